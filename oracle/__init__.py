@@ -1,0 +1,133 @@
+"""Oracle for the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package. The CUDA product path never
+imports it and shares no code with it.
+
+Two independent fp64 CPU implementations live here:
+
+* :func:`recurrence_fwd` / :func:`recurrence_decode_step` -- the plain
+  token-by-token recurrence (the definition), in C (``gdr_oracle.c``), threaded
+  over (sequence, head).  Sources: "Gated DeltaNet: Householder Transitions and
+  the Arithmetic of Forgetting", section "The gated delta rule"; "Linear
+  Attention, Visualized", sections "DeltaNet / Recurrent form", "Gated DeltaNet
+  (GDN)" and "Kimi Delta Attention (KDA)".
+* :func:`oracle.chunked.chunked_fwd` -- the chunkwise WY/UT algorithm written
+  from "Linear Attention, Visualized", sections "Gated DeltaNet (GDN) /
+  Complete per-chunk algorithm" and "Kimi Delta Attention (KDA) / Complete
+  per-chunk algorithm".  It is used only to pin the recurrence (the pages state
+  that every chunk size gives the exact result).
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against closed
+forms, invariants and exact-rational brute force that the pages fix.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (strict IEEE fp64: no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared",
+               "-o", _LIB, _SRC, "-lm", "-lpthread"]
+        subprocess.check_call(cmd)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            dp = ctypes.POINTER(ctypes.c_double)
+            ip = ctypes.POINTER(ctypes.c_int)
+            lib.oracle_gdr_fwd.restype = ctypes.c_int
+            lib.oracle_gdr_fwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ip, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int]
+            lib.oracle_gdr_decode_step.restype = ctypes.c_int
+            lib.oracle_gdr_decode_step.argtypes = [dp, dp, dp, dp, dp, dp, dp,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def recurrence_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, threads=None):
+    """Token-by-token fp64 recurrence over whole sequences.
+
+    Shapes: q, k ``[B, T, H, d_k]``; v ``[B, T, H, d_v]``; g ``[B, T, H]``
+    (scalar gate) or ``[B, T, H, d_k]`` (per-key-channel gate), the log of the
+    decay; beta ``[B, T, H]``; S0 ``[N, H, d_v, d_k]`` or None (zero state).
+    With ``cu_seqlens`` (length N+1 token offsets) B must be 1 and the state is
+    reset at every sequence boundary.  Returns ``(O [B,T,H,d_v], S_final
+    [N,H,d_v,d_k])`` in float64.
+    """
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    per_channel = 1 if g.ndim == 4 else 0
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        n_seq = len(cu) - 1
+        cu_p = cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    else:
+        cu = None
+        n_seq = B
+        cu_p = None
+    S0a = None if S0 is None else _f64(S0)
+    out = np.zeros((B, T, H, dv), dtype=np.float64)
+    S_final = np.zeros((n_seq, H, dv, dk), dtype=np.float64)
+    rc = _load().oracle_gdr_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0a),
+                                _ptr(out), _ptr(S_final), B, T, H, dk, dv, cu_p, n_seq,
+                                per_channel, int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError("oracle_gdr_fwd rejected its arguments")
+    return out, S_final
+
+
+def recurrence_decode_step(q, k, v, g, beta, S):
+    """One decode step for N sequences; returns ``(out [N,H,d_v], S_new)``.
+
+    q, k ``[N, H, d_k]``; v ``[N, H, d_v]``; g ``[N, H]`` or ``[N, H, d_k]``;
+    beta ``[N, H]``; S ``[N, H, d_v, d_k]`` (not modified; a copy is updated).
+    """
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    S_new = _f64(S).copy()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    out = np.zeros((N, H, dv), dtype=np.float64)
+    rc = _load().oracle_gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                        _ptr(S_new), _ptr(out), N, H, dk, dv,
+                                        1 if g.ndim == 3 else 0)
+    if rc != 0:
+        raise ValueError("oracle_gdr_decode_step rejected its arguments")
+    return out, S_new
