@@ -1,0 +1,538 @@
+"""Benchmark of the gated delta rule forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one gdr_fwd over the workload's whole batch (prefill workloads) or
+one gdr_decode_step over all sequences (decode).  Inputs are seeded synthetic
+data of the workload's shapes and distributions (gated_delta_rule_90_b200.inputs),
+resident in HBM before the timed region.  Prints ONE JSON line on rank 0.
+
+Multi-GPU (launched by torch.distributed.run): the (sequence, head) units of
+the method are independent, so every rank runs its own copy of the workload
+(weak scaling) with no collective on the data path; only the timing is reduced
+(max over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_90_b200 import binding, inputs  # noqa: E402
+
+METRIC = "gated-delta-rule fwd tokens/s; % roofline (TC TFLOP/s prefill, HBM GB/s decode)"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SM_COUNT = 148
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- algorithmic work
+def prefill_flops_per_token_head(C, dk, dv):
+    """The 8 chunk GEMMs counted dense: K K^T, Q K^T (2 C d_k each), T V (2 C d_v),
+    T K<- (2 C d_k), A Z (2 C d_v), W<- S^T, Q<- S^T, Z^T K-> (2 d_k d_v each)."""
+    return 2 * C * (3 * dk + 2 * dv) + 6 * dk * dv
+
+
+def prefill_flops_split(C, dk, dv):
+    """(WY-transform share, state-pass share) of the flops per token-head."""
+    wy = 2 * C * dk * 2 + 2 * C * dv + 2 * C * dk
+    return wy, prefill_flops_per_token_head(C, dk, dv) - wy
+
+
+def prefill_min_bytes(cfg, n_seq):
+    """One read of q, k, v, g, beta, S0 and one write of out and S_final."""
+    e = 2 if cfg.dtype == "bf16" else 4
+    th = cfg.B * cfg.T * cfg.H
+    per = (2 * cfg.d_k + cfg.d_v) * e + cfg.d_v * e + 4 + (4 * cfg.d_k if cfg.gate == "channel" else 4)
+    states = n_seq * cfg.H * cfg.d_k * cfg.d_v * 4 * ((1 if cfg.s0_var > 0 else 0) + 1)
+    return th * per + states
+
+
+def decode_bytes(cfg):
+    e = 2 if cfg.dtype == "bf16" else 4
+    heads = cfg.N * cfg.H
+    gb = 4 * cfg.d_k if cfg.gate == "channel" else 4
+    return 2 * heads * cfg.d_k * cfg.d_v * 4 + heads * ((2 * cfg.d_k + 2 * cfg.d_v) * e + gb + 4)
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = os.path.join("/tmp", f"gdr_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        busy = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- helpers
+def dev_tensor(x, dtype, device):
+    if x is None:
+        return None
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    if dtype == "bf16":
+        t = t.to(torch.bfloat16)
+    return t.to(device)
+
+
+def max_over_ranks(x, world):
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.distributed.get_backend() == "nccl" else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ----------------------------------------------------------------- prefill
+class PrefillRun:
+    def __init__(self, cfg, device, seed, path):
+        self.cfg = cfg
+        self.device = device
+        self.inp = inputs.prefill_inputs(cfg, seed=seed)
+        inp = self.inp
+        self.n_seq = inp.n_seq
+        self.q, self.k, self.v = (dev_tensor(x, cfg.dtype, device) for x in (inp.q, inp.k, inp.v))
+        self.g, self.beta = dev_tensor(inp.g, "f32", device), dev_tensor(inp.beta, "f32", device)
+        self.S0 = dev_tensor(inp.S0, "f32", device)
+        self.cu = None if inp.cu_seqlens is None else torch.from_numpy(inp.cu_seqlens).to(device)
+        self.path = path
+        self.out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.d_v), dtype=self.q.dtype, device=device)
+        self.SF = torch.empty((self.n_seq, cfg.H, cfg.d_v, cfg.d_k), dtype=torch.float32,
+                              device=device)
+        gate = 1 if cfg.gate == "channel" else 0
+        dt = 1 if cfg.dtype == "bf16" else 0
+        ws = binding.fwd_workspace_size(cfg.B, cfg.T, cfg.H, cfg.d_k, cfg.d_v, cfg.chunk,
+                                        self.n_seq, self.cu is not None, dt, gate, path)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+
+    def step(self):
+        binding.gdr_fwd(self.q, self.k, self.v, self.g, self.beta, self.S0, chunk=self.cfg.chunk,
+                        cu_seqlens=self.cu, out=self.out, S_final=self.SF, path=self.path,
+                        workspace=self.ws)
+
+    def tokens(self):
+        return self.cfg.B * self.cfg.T
+
+    def e2e(self, steps):
+        """Same step through the C-ABI with pinned HOST buffers: H2D of every
+        input, the call, D2H of out and S_final, all inside the timed region."""
+        cfg, inp, dev = self.cfg, self.inp, self.device
+
+        def host(x, dtype):
+            if x is None:
+                return None
+            t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+            if dtype == "bf16":
+                t = t.to(torch.bfloat16)
+            return t.pin_memory()
+
+        hq, hk, hv = (host(x, cfg.dtype) for x in (inp.q, inp.k, inp.v))
+        hg, hb, hS0 = host(inp.g, "f32"), host(inp.beta, "f32"), host(inp.S0, "f32")
+        hcu = None if inp.cu_seqlens is None else torch.from_numpy(inp.cu_seqlens).pin_memory()
+        hout = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        hSF = torch.empty(self.SF.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hS0, hcu)
+                  if t is not None)
+        d2h = hout.numel() * hout.element_size() + hSF.numel() * hSF.element_size()
+        st = torch.cuda.current_stream()
+
+        def one():
+            q = hq.to(dev, non_blocking=True)
+            k = hk.to(dev, non_blocking=True)
+            v = hv.to(dev, non_blocking=True)
+            g = hg.to(dev, non_blocking=True)
+            b = hb.to(dev, non_blocking=True)
+            S0 = None if hS0 is None else hS0.to(dev, non_blocking=True)
+            cu = None if hcu is None else hcu.to(dev, non_blocking=True)
+            out, SF = binding.gdr_fwd(q, k, v, g, b, S0, chunk=cfg.chunk, cu_seqlens=cu,
+                                      path=self.path, workspace=self.ws)
+            hout.copy_(out, non_blocking=True)
+            hSF.copy_(SF, non_blocking=True)
+
+        one()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            one()
+        e1.record(st)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        return ms, h2d, d2h
+
+
+# ----------------------------------------------------------------- decode
+class DecodeRun:
+    """The decode workload: fresh tokens every step (drawn on the device from a
+    seeded generator before the timed region), state updated in place."""
+
+    def __init__(self, cfg, device, seed, n_steps):
+        self.cfg = cfg
+        self.device = device
+        self.S = torch.from_numpy(inputs.decode_state(cfg, seed=seed)).to(device)
+        gen = torch.Generator(device=device)
+        gen.manual_seed(seed)
+        N, H, dk, dv = cfg.N, cfg.H, cfg.d_k, cfg.d_v
+        tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+
+        def unit(shape):
+            x = torch.randn(shape, generator=gen, device=device)
+            return (x / x.norm(dim=-1, keepdim=True)).to(tdt)
+
+        P = self.pool = max(1, n_steps)
+        self.q = unit((P, N, H, dk))
+        self.k = unit((P, N, H, dk))
+        self.v = torch.randn((P, N, H, dv), generator=gen, device=device).to(tdt)
+        self.b = torch.sigmoid(torch.randn((P, N, H), generator=gen, device=device))
+        gshape = (P, N, H, dk) if cfg.gate == "channel" else (P, N, H)
+        self.g = -torch.nn.functional.softplus(torch.randn(gshape, generator=gen, device=device)) * cfg.gate_scale
+        self.out = torch.empty((N, H, dv), dtype=tdt, device=device)
+        self.i = 0
+
+    def step(self):
+        j = self.i % self.pool
+        self.i += 1
+        binding.gdr_decode_step(self.q[j], self.k[j], self.v[j], self.g[j], self.b[j], self.S,
+                                out=self.out)
+
+    def tokens(self):
+        return self.cfg.N
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_prefill_sample(cfg, seed, budget_s):
+    """Time the fp64 oracle on a bounded sample of the workload: the first h
+    heads of every sequence, h chosen so the run takes about budget_s seconds.
+    Returns (equivalent tokens/s, cores, description)."""
+    import oracle  # CPU baseline leg only
+
+    inp = inputs.prefill_inputs(cfg, seed=seed)
+    cores = oracle.default_threads()
+    n_seq = inp.n_seq
+
+    def run(h):
+        sl = lambda x: None if x is None else np.ascontiguousarray(x[:, :, :h])
+        S0 = None if inp.S0 is None else np.ascontiguousarray(inp.S0[:, :h])
+        t = time.perf_counter()
+        oracle.recurrence_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.g), sl(inp.beta), S0=S0,
+                              cu_seqlens=inp.cu_seqlens, threads=cores)
+        return time.perf_counter() - t
+
+    t1 = run(1)
+    per_head = t1  # one head of every sequence
+    h = int(max(1, min(cfg.H, budget_s / max(per_head, 1e-6))))
+    if h > 1:
+        dt = run(h)
+    else:
+        dt = t1
+    token_heads = cfg.B * cfg.T * h
+    return (token_heads / cfg.H) / dt, cores, (f"{h} of {cfg.H} heads x all {cfg.B * cfg.T} "
+                                               f"tokens ({token_heads} token-heads, {dt:.2f} s)"), dt
+
+
+def oracle_decode_sample(cfg, seed, budget_s):
+    import oracle
+
+    S = inputs.decode_state(cfg, seed=seed).astype(np.float64)
+    t0 = time.perf_counter()
+    steps = 0
+    while time.perf_counter() - t0 < budget_s and steps < cfg.steps:
+        tok = inputs.decode_token(cfg, steps, seed=seed)
+        t = time.perf_counter()
+        _, S = oracle.recurrence_decode_step(tok.q, tok.k, tok.v, tok.g, tok.beta, S)
+        steps += 1
+        if steps == 1:
+            t_compute = time.perf_counter() - t
+        else:
+            t_compute += time.perf_counter() - t
+    return cfg.N * steps / t_compute, 1, f"{steps} full decode steps ({cfg.N}x{cfg.H} heads)", t_compute
+
+
+# ----------------------------------------------------------------- main
+def workload_config(name):
+    if name in inputs.PREFILL:
+        c = inputs.PREFILL[name]
+        return c, {"workload": name, "B": c.B, "T": c.T, "H": c.H, "d_k": c.d_k, "d_v": c.d_v,
+                   "chunk": c.chunk, "gate": c.gate, "dtype_io": c.dtype,
+                   **({"n_seq": c.n_seq} if c.n_seq else {})}
+    c = inputs.DECODE[name]
+    return c, {"workload": name, "N": c.N, "H": c.H, "d_k": c.d_k, "d_v": c.d_v, "gate": c.gate,
+               "dtype_io": c.dtype, "steps_per_sequence": c.steps}
+
+
+def time_steps(run, steps, flush):
+    """Per-step CUDA-event times (ms) on the launching stream; L2 flushed
+    between steps (outside the timed intervals) when `flush` is given."""
+    st = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        if flush is not None:
+            flush.zero_()
+        a.record(st)
+        run.step()
+        b.record(st)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 CPU oracle, timed as it stands on the host cores."""
+    if rank != 0:
+        return
+    cfg, conf = workload_config(args.workload)
+    budget = max(0.5, args.ref_budget_s / max(1, args.steps + args.warmup))
+    vals = []
+    if isinstance(cfg, inputs.DecodeConfig):
+        for i in range(args.warmup + args.steps):
+            v, cores, sample, _ = oracle_decode_sample(cfg, inputs.BASE_SEED + cfg.seed_index,
+                                                       budget)
+            if i >= args.warmup:
+                vals.append(v)
+    else:
+        for i in range(args.warmup + args.steps):
+            v, cores, sample, _ = oracle_prefill_sample(cfg, inputs.BASE_SEED + cfg.seed_index,
+                                                        budget)
+            if i >= args.warmup:
+                vals.append(v)
+    value = statistics.median(vals)
+    tok = cfg.N if isinstance(cfg, inputs.DecodeConfig) else cfg.B * cfg.T
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tok / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": conf,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warmup,
+            with_cpu, with_e2e, sampler=None):
+    cfg, conf = workload_config(name)
+    seed = (inputs.BASE_SEED + cfg.seed_index) * 1000 + rank
+    is_decode = isinstance(cfg, inputs.DecodeConfig)
+    run = (DecodeRun(cfg, device, seed, steps + warmup) if is_decode
+           else PrefillRun(cfg, device, seed, path))
+    flush = None if is_decode else torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32,
+                                               device=device)
+    for _ in range(warmup):
+        if flush is not None:
+            flush.zero_()
+        run.step()
+    torch.cuda.synchronize()
+    binding.profile_read()  # reset counters
+    binding.profile_enable(True)
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    times = time_steps(run, steps, flush)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - w0
+    clocks = sampler.stop() if sampler else None
+    binding.profile_enable(False)
+    prof = binding.profile_read()
+    assert binding.device_status() == binding.GDR_OK
+    ms = max_over_ranks(sum(times) / len(times), world)
+    tokens_all = run.tokens() * world
+    value = tokens_all / (ms * 1e-3)
+    kernels = {k: {"launches": n, "avg_ms": (t / n if n else 0.0)} for k, (n, t) in prof.items()
+               if n}
+    launches = sum(n for n, _ in prof.values())
+
+    # roofline of the dominant kernel
+    dom = max(kernels.items(), key=lambda kv: kv[1]["avg_ms"] * kv[1]["launches"])[0]
+    dom_ms = kernels[dom]["avg_ms"]
+    if is_decode:
+        B_ = decode_bytes(cfg)
+        ach = B_ / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": peak_kind + " hbm_gbs", "algorithmic_bytes_per_launch": B_,
+                "frac_of_8TBps_spec": ach / 8000.0}
+        conf["l2"] = "no flush: the 512 MiB state is larger than L2 and is streamed every step"
+    else:
+        th = cfg.B * cfg.T * cfg.H
+        f_all = prefill_flops_per_token_head(cfg.chunk, cfg.d_k, cfg.d_v)
+        wy, st_ = prefill_flops_split(cfg.chunk, cfg.d_k, cfg.d_v)
+        share = {"fwd_simt": f_all, "tc_wy": wy, "tc_state": st_}.get(dom, 0)
+        flops = share * th
+        if dom == "fwd_simt":
+            peak = SM_COUNT * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            ach = flops / (dom_ms * 1e-3) / 1e12
+            roof = {"bound": "alu", "kernel": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                    "frac": ach / peak, "traffic": None,
+                    "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
+                    "algorithmic_flops_per_launch": flops}
+        else:
+            peak = peaks["bf16_tflops"]
+            ach = flops / (dom_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak,
+                    "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                    "peak_source": peak_kind + " bf16_tflops (burst)",
+                    "algorithmic_flops_per_launch": flops}
+        min_bytes = prefill_min_bytes(cfg, run.n_seq)
+        roof["step"] = {"tflops": f_all * th / (ms * 1e-3) / 1e12,
+                        "tc_frac": f_all * th / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                        "hbm_gbs_min_bytes": min_bytes / (ms * 1e-3) / 1e9,
+                        "hbm_frac": min_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                        "flops_per_step": f_all * th, "min_bytes_per_step": min_bytes}
+        conf["l2"] = (f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the "
+                      "per-step CUDA-event intervals)")
+        conf["path"] = path
+    res = {"value": value, "ms_per_step": ms, "wall_s_incl_flush": wall, "roofline": roof,
+           "kernels": kernels, "gpu_launches": launches, "clocks": clocks, "config": conf,
+           "cfg": cfg, "run": run}
+    if with_e2e and not is_decode:
+        e_ms, h2d, d2h = run.e2e(max(1, min(steps, 5)))
+        e_ms = max_over_ranks(e_ms, world)
+        res["e2e"] = {"value": tokens_all / (e_ms * 1e-3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    if with_cpu and rank == 0 and world == 1:
+        if is_decode:
+            v, cores, sample, _ = oracle_decode_sample(cfg, seed, 10.0)
+        else:
+            v, cores, sample, _ = oracle_prefill_sample(cfg, seed, 10.0)
+        res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": sample}
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gdn_prefill",
+                    choices=list(inputs.PREFILL) + list(inputs.DECODE))
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill",
+                    help="comma-separated workloads measured after the main one ('' for none)")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--ref-budget-s", type=float, default=90.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+            return
+        device = torch.device("cuda", local)
+        torch.cuda.set_device(device)
+        binding.lib()
+        peaks, peak_kind = load_peaks()
+        sampler = ClockSampler(local) if rank == 0 else None
+        main_res = measure(args, args.workload, device, rank, world, peaks, peak_kind, args.path,
+                           args.steps, args.warmup, not args.no_cpu, True, sampler)
+        extra = {}
+        for name in [x for x in args.extra.split(",") if x and x != args.workload]:
+            steps = 20 if name != "decode" else 200
+            r = measure(args, name, device, rank, world, peaks, peak_kind, args.path, steps, 3,
+                        False, False, None)
+            extra[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
+                           "steps": steps, "config": r["config"], "roofline": r["roofline"],
+                           "kernels": r["kernels"]}
+            del r
+            torch.cuda.empty_cache()
+        if rank == 0:
+            cfg = main_res["cfg"]
+            line = {"metric": METRIC, "value": main_res["value"], "unit": "tokens/s",
+                    "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                    "ms_per_step": main_res["ms_per_step"], "higher_is_better": True,
+                    "scaling": "weak", "vs_baseline": None,
+                    "dtype": "bf16" if getattr(cfg, "dtype", "bf16") == "bf16" else "f32",
+                    "data": "synthetic (seeded; shapes and distributions of the workload)",
+                    "config": {**main_res["config"], "parallelism": f"replicas x{world}"},
+                    "roofline": main_res["roofline"], "e2e": main_res.get("e2e"),
+                    "gpu_launches": main_res["gpu_launches"], "clocks": main_res["clocks"],
+                    "kernels": main_res["kernels"], "cpu_baseline": main_res.get("cpu_baseline"),
+                    "extra": extra}
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

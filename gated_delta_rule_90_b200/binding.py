@@ -1,0 +1,162 @@
+"""ctypes binding of libgdr (include/gdr.h) for torch tensors.
+
+Argument marshalling only: shapes are read off the tensors, outputs and the
+workspace are allocated with torch, and every step of the computation runs
+in libgdr's CUDA kernels.  There is no fallback: if the library is missing
+the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdr.so")
+
+GDR_OK, GDR_ERR_INVALID, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT = range(5)
+GDR_F32, GDR_BF16 = 0, 1
+GDR_GATE_SCALAR, GDR_GATE_PER_KEY_CHANNEL = 0, 1
+PATHS = {"auto": 0, "simt": 1, "tc": 2}
+KERNELS = {"decode": 0, "fwd_simt": 1, "tc_plan": 2, "tc_wy": 3, "tc_state": 4}
+
+_lib = None
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdr.so (built in-tree by __graft_entry__.build())."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgdr.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.gdr_status_string.restype = ctypes.c_char_p
+        L.gdr_status_string.argtypes = [i]
+        L.gdr_fwd_workspace_size.restype = sz
+        L.gdr_fwd_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i, i, i]
+        L.gdr_fwd.restype = i
+        L.gdr_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, i, i, i,
+                              vp, sz, vp]
+        L.gdr_decode_step.restype = i
+        L.gdr_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+        L.gdr_device_status.restype = i
+        L.gdr_device_status.argtypes = [vp]
+        L.gdr_selftest_wait_timeout.restype = i
+        L.gdr_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+        L.gdr_profile_enable.restype = None
+        L.gdr_profile_enable.argtypes = [i]
+        L.gdr_profile_read.restype = i
+        L.gdr_profile_read.argtypes = [i, ctypes.POINTER(ctypes.c_longlong),
+                                       ctypes.POINTER(ctypes.c_double)]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdr_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDR_BF16
+    if t.dtype == torch.float32:
+        return GDR_F32
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _need_contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def fwd_workspace_size(B, T, H, d_k, d_v, chunk, n_seq, varlen, dtype, gate, path="auto") -> int:
+    return int(lib().gdr_fwd_workspace_size(B, T, H, d_k, d_v, chunk, n_seq, int(bool(varlen)),
+                                            dtype, gate, PATHS[path]))
+
+
+def gdr_fwd(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, out=None,
+            S_final=None, want_final: bool = True, path: str = "auto", workspace=None,
+            stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Prefill: returns ``(out [B,T,H,d_v], S_final [N,H,d_v,d_k] or None)``."""
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    dtype = _dtype_code(q)
+    gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
+    n_seq = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+    _need_contig(q, k, v, g, beta, S0, cu_seqlens)
+    if out is None:
+        out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
+    if S_final is None and want_final:
+        S_final = torch.empty((n_seq, H, d_v, d_k), dtype=torch.float32, device=q.device)
+    ws_bytes = fwd_workspace_size(B, T, H, d_k, d_v, chunk, n_seq, cu_seqlens is not None, dtype,
+                                  gate, path)
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    ws_avail = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdr_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out),
+                       _ptr(S_final), B, T, H, d_k, d_v, chunk, _ptr(cu_seqlens), n_seq, dtype,
+                       gate, PATHS[path], _ptr(workspace), ws_avail, _stream(stream))
+    if st != GDR_OK:
+        raise GdrError(st, "gdr_fwd")
+    return out, S_final
+
+
+def gdr_decode_step(q, k, v, g, beta, S, *, out=None, stream=None) -> torch.Tensor:
+    """Decode one token per sequence, updating ``S`` in place; returns out [N,H,d_v]."""
+    N, H, d_k = q.shape
+    d_v = v.shape[-1]
+    dtype = _dtype_code(q)
+    gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 3 else GDR_GATE_SCALAR
+    _need_contig(q, k, v, g, beta, S)
+    if out is None:
+        out = torch.empty((N, H, d_v), dtype=q.dtype, device=q.device)
+    st = lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                               _ptr(out), N, H, d_k, d_v, dtype, gate, _stream(stream))
+    if st != GDR_OK:
+        raise GdrError(st, "gdr_decode_step")
+    return out
+
+
+def device_status(stream=None) -> int:
+    return int(lib().gdr_device_status(_stream(stream)))
+
+
+def selftest_wait_timeout(spin_limit: int, stream=None) -> int:
+    return int(lib().gdr_selftest_wait_timeout(spin_limit, _stream(stream)))
+
+
+def profile_enable(on: bool = True) -> None:
+    lib().gdr_profile_enable(1 if on else 0)
+
+
+def profile_read() -> dict:
+    """{kernel: (launches, total_ms)} since the previous read (then reset)."""
+    res = {}
+    for name, kid in KERNELS.items():
+        n = ctypes.c_longlong(0)
+        ms = ctypes.c_double(0.0)
+        st = lib().gdr_profile_read(kid, ctypes.byref(n), ctypes.byref(ms))
+        if st != GDR_OK:
+            raise GdrError(st, "gdr_profile_read")
+        res[name] = (int(n.value), float(ms.value))
+    return res

@@ -1,0 +1,56 @@
+// Shared device helpers of the gated delta rule kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdr.h"
+
+namespace gdr {
+
+// Device error word bits (see gdr_device_status).
+enum : unsigned int { kErrTimeout = 1u };
+
+// Token-storage loads/stores: fp32 or bf16, converted to/from fp32.
+__device__ __forceinline__ float ld_in(const float *p, size_t i) { return p[i]; }
+__device__ __forceinline__ float ld_in(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void st_out(float *p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void st_out(__nv_bfloat16 *p, size_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+// Sequence bounds [t0, t1) of sequence s, in token rows of the [B*T] view.
+// Packed offsets are clamped into [0, T_total] and made non-decreasing so a
+// malformed array can never send a kernel out of bounds.
+__device__ __forceinline__ void seq_bounds(const int32_t *cu, int s, int T, int T_total,
+                                           long &t0, long &t1) {
+    if (cu) {
+        int a = cu[s], b = cu[s + 1];
+        a = a < 0 ? 0 : (a > T_total ? T_total : a);
+        b = b < a ? a : (b > T_total ? T_total : b);
+        t0 = a;
+        t1 = b;
+    } else {
+        t0 = (long)s * T;
+        t1 = t0 + T;
+    }
+}
+
+}  // namespace gdr
+
+// Host-side launch helpers shared by the translation units.
+namespace gdr_host {
+// Address of the device error word on the current device (cached per device).
+unsigned int *device_error_word();
+// Launch accounting: call prof_begin before and prof_end after a launch of
+// kernel `id` on stream `st` (events are recorded only while timing is on).
+struct ProfToken {
+    int id;
+    int slot;
+};
+ProfToken prof_begin(int id, cudaStream_t st);
+void prof_end(ProfToken tok, cudaStream_t st);
+}  // namespace gdr_host

@@ -1,0 +1,271 @@
+// SIMT (fp32 CUDA-core) chunkwise prefill of the gated delta rule.
+//
+// The path for fp32 inputs (where bf16 tensor-core operands would not meet an
+// fp32 tolerance) and for shapes outside the tensor-core path; it is also the
+// GPU-side cross-check of that path.  One CTA owns one (sequence, head, slice of
+// 32 state rows) and walks the sequence's chunks in order.  Per chunk r it takes
+// the steps of "Linear Attention, Visualized", "Gated DeltaNet (GDN) / Complete
+// per-chunk algorithm" and "Kimi Delta Attention (KDA) / Complete per-chunk
+// algorithm", transposed to the column convention (S is d_v x d_k; only the
+// CTA's rows of S are held):
+//   G_l       = sum_{s<=l} g_s                       (cumulative log-decay)
+//   L[l,m]    = sum_c k_lc k_mc exp(G_lc - G_mc)      (m < l)
+//   A[l,m]    = sum_c q_lc k_mc exp(G_lc - G_mc)      (m <= l)
+//   (I + diag(beta) L) T = diag(beta)                 (column-wise forward substitution)
+//   Z         = T (V - K<- S^T)          (= U - W<- S^T with U = T V, W<- = T K<-)
+//   O         = Q<- S^T + A Z
+//   S         <- S Diag(exp(G_C)) + Z^T K->
+// with K<- = exp(G) . K, Q<- = exp(G) . Q, K-> = exp(G_C - G) . K.  Decay ratios
+// are always formed as exp of a difference of cumulative sums, never as a ratio
+// of products.  A chunk that runs past the end of its sequence treats the
+// missing tokens as k = q = v = 0, beta = 0, g = 0, which leaves every valid
+// row unchanged (the pages assume the chunk size divides the length).
+#include "common.cuh"
+
+namespace gdr {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtRows = 32;  // state rows (d_v) per CTA
+
+struct SimtSmem {
+    // offsets in floats
+    int Kc, Qc, Gc, Kx, bt, Nm, Am, Tm, Pm, Zm, Ss, total;
+    int kst;  // padded row stride of the [C][d_k] buffers
+};
+
+__host__ __device__ inline SimtSmem simt_layout(int C, int dk, bool channel) {
+    SimtSmem L;
+    L.kst = dk + 1;
+    int o = 0;
+    L.Kc = o; o += C * L.kst;
+    L.Qc = o; o += C * L.kst;
+    L.Gc = o; o += channel ? C * L.kst : C;
+    L.Kx = o; o += channel ? C * L.kst : 0;
+    L.bt = o; o += C;
+    L.Nm = o; o += C * C;
+    L.Am = o; o += C * C;
+    L.Tm = o; o += C * C;
+    L.Pm = o; o += C * kSimtRows;
+    L.Zm = o; o += C * kSimtRows;
+    L.Ss = o; o += kSimtRows * L.kst;
+    L.total = o;
+    return L;
+}
+
+template <typename Tin, bool CH>
+__global__ void __launch_bounds__(kSimtThreads)
+fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                const float *__restrict__ g, const float *__restrict__ beta,
+                const float *__restrict__ S0, Tin *__restrict__ out, float *__restrict__ S_final,
+                int T, int H, int dk, int dv, int C, const int32_t *__restrict__ cu, int T_total) {
+    extern __shared__ float sm[];
+    const SimtSmem L = simt_layout(C, dk, CH);
+    float *Kc = sm + L.Kc, *Qc = sm + L.Qc, *Gc = sm + L.Gc, *Kx = sm + L.Kx, *bt = sm + L.bt;
+    float *Nm = sm + L.Nm, *Am = sm + L.Am, *Tm = sm + L.Tm, *Pm = sm + L.Pm, *Zm = sm + L.Zm;
+    float *Ss = sm + L.Ss;
+    const int kst = L.kst;
+    const int tid = threadIdx.x;
+    const int s = blockIdx.x / H, h = blockIdx.x % H;
+    const int r0 = blockIdx.y * kSimtRows;
+    const int nr = min(kSimtRows, dv - r0);
+    long t0, t1;
+    seq_bounds(cu, s, T, T_total, t0, t1);
+
+    // state slice: rows r0 .. r0+nr of S (d_v x d_k)
+    const size_t soff = ((size_t)s * H + h) * (size_t)dv * dk;
+    for (int e = tid; e < kSimtRows * dk; e += kSimtThreads) {
+        const int r = e / dk, c = e % dk;
+        Ss[r * kst + c] = (S0 && r < nr) ? S0[soff + (size_t)(r0 + r) * dk + c] : 0.f;
+    }
+
+    for (long c0 = t0; c0 < t1; c0 += C) {
+        const int len = (int)min((long)C, t1 - c0);
+        __syncthreads();
+        // ---- load the chunk (missing tokens are zero) ----
+        for (int e = tid; e < C * dk; e += kSimtThreads) {
+            const int l = e / dk, c = e % dk;
+            float kv = 0.f, qv = 0.f;
+            if (l < len) {
+                const size_t off = ((size_t)(c0 + l) * H + h) * dk + c;
+                kv = ld_in(k, off);
+                qv = ld_in(q, off);
+            }
+            Kc[l * kst + c] = kv;
+            Qc[l * kst + c] = qv;
+            if (CH) Gc[l * kst + c] = (l < len) ? g[((size_t)(c0 + l) * H + h) * dk + c] : 0.f;
+        }
+        for (int l = tid; l < C; l += kSimtThreads) {
+            const size_t off = (size_t)(c0 + l) * H + h;
+            bt[l] = (l < len) ? beta[off] : 0.f;
+            if (!CH) Gc[l] = (l < len) ? g[off] : 0.f;
+        }
+        __syncthreads();
+        // ---- cumulative log-decay G (in place) ----
+        if (CH) {
+            for (int c = tid; c < dk; c += kSimtThreads) {
+                float acc = 0.f;
+                for (int l = 0; l < C; ++l) {
+                    acc += Gc[l * kst + c];
+                    Gc[l * kst + c] = acc;
+                }
+            }
+        } else if (tid == 0) {
+            float acc = 0.f;
+            for (int l = 0; l < C; ++l) {
+                acc += Gc[l];
+                Gc[l] = acc;
+            }
+        }
+        __syncthreads();
+        // ---- L (scaled by beta into N = diag(beta) L) and A ----
+        for (int p = tid; p < C * C; p += kSimtThreads) {
+            const int l = p / C, m = p % C;
+            float lv = 0.f, av = 0.f;
+            if (m <= l) {
+                const float *kl = Kc + l * kst, *km = Kc + m * kst, *ql = Qc + l * kst;
+                if (CH) {
+                    const float *gl = Gc + l * kst, *gm = Gc + m * kst;
+                    for (int c = 0; c < dk; ++c) {
+                        const float w = km[c] * expf(gl[c] - gm[c]);
+                        lv = fmaf(kl[c], w, lv);
+                        av = fmaf(ql[c], w, av);
+                    }
+                } else {
+                    for (int c = 0; c < dk; ++c) {
+                        lv = fmaf(kl[c], km[c], lv);
+                        av = fmaf(ql[c], km[c], av);
+                    }
+                    const float w = expf(Gc[l] - Gc[m]);
+                    lv *= w;
+                    av *= w;
+                }
+            }
+            Nm[p] = (m < l) ? bt[l] * lv : 0.f;
+            Am[p] = av;
+        }
+        __syncthreads();
+        // ---- T: (I + N) T = diag(beta), thread j solves column j ----
+        for (int j = tid; j < C; j += kSimtThreads) {
+            for (int i = 0; i < C; ++i) {
+                float acc = (i == j) ? bt[j] : 0.f;
+                for (int m = 0; m < i; ++m) acc = fmaf(-Nm[i * C + m], Tm[m * C + j], acc);
+                Tm[i * C + j] = (i < j) ? 0.f : acc;
+            }
+        }
+        // decayed copies: Q<- in place; K<- into Kx (per channel) -- A and L are done
+        for (int e = tid; e < C * dk; e += kSimtThreads) {
+            const int l = e / dk, c = e % dk;
+            const float w = expf(CH ? Gc[l * kst + c] : Gc[l]);
+            Qc[l * kst + c] *= w;
+            if (CH) Kx[l * kst + c] = Kc[l * kst + c] * w;
+        }
+        __syncthreads();
+        // ---- P = V - K<- S^T  (C x nr) ----
+        for (int e = tid; e < C * kSimtRows; e += kSimtThreads) {
+            const int l = e / kSimtRows, r = e % kSimtRows;
+            float acc = 0.f;
+            if (r < nr && l < len) {
+                const float *kl = CH ? Kx + l * kst : Kc + l * kst;
+                const float *sr = Ss + r * kst;
+                for (int c = 0; c < dk; ++c) acc = fmaf(kl[c], sr[c], acc);
+                if (!CH) acc *= expf(Gc[l]);
+                acc = ld_in(v, ((size_t)(c0 + l) * H + h) * dv + r0 + r) - acc;
+            }
+            Pm[e] = acc;
+        }
+        __syncthreads();
+        // ---- Z = T P ----
+        for (int e = tid; e < C * kSimtRows; e += kSimtThreads) {
+            const int l = e / kSimtRows, r = e % kSimtRows;
+            float acc = 0.f;
+            for (int m = 0; m <= l; ++m) acc = fmaf(Tm[l * C + m], Pm[m * kSimtRows + r], acc);
+            Zm[e] = acc;
+        }
+        __syncthreads();
+        // ---- O = Q<- S^T + A Z ----
+        for (int e = tid; e < C * kSimtRows; e += kSimtThreads) {
+            const int l = e / kSimtRows, r = e % kSimtRows;
+            if (r < nr && l < len) {
+                float acc = 0.f;
+                const float *ql = Qc + l * kst, *sr = Ss + r * kst;
+                for (int c = 0; c < dk; ++c) acc = fmaf(ql[c], sr[c], acc);
+                for (int m = 0; m <= l; ++m) acc = fmaf(Am[l * C + m], Zm[m * kSimtRows + r], acc);
+                st_out(out, ((size_t)(c0 + l) * H + h) * dv + r0 + r, acc);
+            }
+        }
+        // K-> = exp(G_C - G) . K into Kx (Kx's K<- is no longer read after P)
+        const int last = C - 1;
+        if (CH) {
+            for (int e = tid; e < C * dk; e += kSimtThreads) {
+                const int l = e / dk, c = e % dk;
+                Kx[l * kst + c] = Kc[l * kst + c] * expf(Gc[last * kst + c] - Gc[l * kst + c]);
+            }
+        }
+        __syncthreads();
+        // ---- S <- S Diag(exp(G_C)) + Z^T K-> ----
+        for (int e = tid; e < kSimtRows * dk; e += kSimtThreads) {
+            const int r = e / dk, c = e % dk;
+            float acc;
+            if (CH) {
+                acc = Ss[r * kst + c] * expf(Gc[last * kst + c]);
+                for (int l = 0; l < C; ++l) acc = fmaf(Zm[l * kSimtRows + r], Kx[l * kst + c], acc);
+            } else {
+                acc = Ss[r * kst + c] * expf(Gc[last]);
+                for (int l = 0; l < C; ++l)
+                    acc = fmaf(Zm[l * kSimtRows + r] * expf(Gc[last] - Gc[l]), Kc[l * kst + c], acc);
+            }
+            Ss[r * kst + c] = acc;
+        }
+    }
+    __syncthreads();
+    if (S_final) {
+        for (int e = tid; e < nr * dk; e += kSimtThreads) {
+            const int r = e / dk, c = e % dk;
+            S_final[soff + (size_t)(r0 + r) * dk + c] = Ss[r * kst + c];
+        }
+    }
+}
+
+}  // namespace gdr
+
+using namespace gdr;
+
+namespace gdr_host {
+
+size_t simt_smem_bytes(int C, int dk, bool channel) {
+    return sizeof(float) * (size_t)simt_layout(C, dk, channel).total;
+}
+
+template <typename Tin, bool CH>
+static cudaError_t launch_simt(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *S0, void *out, float *S_final,
+                               int T, int H, int dk, int dv, int C, const int32_t *cu, int n_seq,
+                               int T_total, cudaStream_t st) {
+    const size_t smem = simt_smem_bytes(C, dk, CH);
+    cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<Tin, CH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)(n_seq * H), (unsigned)((dv + kSimtRows - 1) / kSimtRows));
+    fwd_simt_kernel<Tin, CH><<<grid, kSimtThreads, smem, st>>>(
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, S0, (Tin *)out, S_final, T, H,
+        dk, dv, C, cu, T_total);
+    return cudaGetLastError();
+}
+
+cudaError_t fwd_simt_dispatch(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *S0, void *out, float *S_final,
+                              int T, int H, int dk, int dv, int C, const int32_t *cu, int n_seq,
+                              int T_total, gdr_dtype dtype, gdr_gate gate, cudaStream_t st) {
+    const bool ch = gate == GDR_GATE_PER_KEY_CHANNEL;
+    if (dtype == GDR_BF16)
+        return ch ? launch_simt<__nv_bfloat16, true>(q, k, v, g, beta, S0, out, S_final, T, H, dk,
+                                                     dv, C, cu, n_seq, T_total, st)
+                  : launch_simt<__nv_bfloat16, false>(q, k, v, g, beta, S0, out, S_final, T, H,
+                                                      dk, dv, C, cu, n_seq, T_total, st);
+    return ch ? launch_simt<float, true>(q, k, v, g, beta, S0, out, S_final, T, H, dk, dv, C, cu,
+                                         n_seq, T_total, st)
+              : launch_simt<float, false>(q, k, v, g, beta, S0, out, S_final, T, H, dk, dv, C, cu,
+                                          n_seq, T_total, st);
+}
+
+}  // namespace gdr_host

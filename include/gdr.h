@@ -1,0 +1,166 @@
+/*
+ * gdr.h -- C-ABI of the B200 (sm_100a) gated delta rule forward pass.
+ *
+ * The operation (column convention; the state S of one (sequence, head) is a
+ * d_v x d_k fp32 matrix, q_t, k_t in R^{d_k}, v_t in R^{d_v}):
+ *
+ *     S_t = (S_{t-1} D_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,    o_t = S_t q_t
+ *
+ * with D_t = exp(g_t) I  (GDR_GATE_SCALAR, Gated DeltaNet) or
+ *      D_t = Diag(exp(g_t)) (GDR_GATE_PER_KEY_CHANNEL, Kimi Delta Attention:
+ *      the state is decayed channel by channel first, then corrected).
+ * Sources: "Gated DeltaNet: Householder Transitions and the Arithmetic of
+ * Forgetting", section "The gated delta rule"; "Linear Attention, Visualized",
+ * sections "Gated DeltaNet (GDN)" and "Kimi Delta Attention (KDA)".
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or keeps them.  Tensors are dense row-major
+ *    (contiguous) and 16-byte aligned.
+ *  - q, k, v and out are fp32 (GDR_F32) or bf16 (GDR_BF16) as `dtype` says;
+ *    g, beta and all states are fp32.
+ *  - g is the log of the decay: alpha = exp(g) (g <= 0 for a decay).  beta is
+ *    used as given (no clamp; beta = 2 makes the reflection I - 2 k k^T).
+ *    No 1/sqrt(d) scale and no normalisation is applied: q and k are used as
+ *    given ("Linear Attention, Visualized", Notation: the scale is absorbed
+ *    into q or k).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Argument validation happens on the host before any launch; a
+ *    failed validation launches nothing and leaves every output untouched.
+ *  - `out` must not overlap any input.  S0 may equal S_final (in-place
+ *    continuation); other overlaps are not allowed.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID = 1,      /* bad shape, NULL where required, misalignment, bad enum */
+    GDR_ERR_UNSUPPORTED = 2,  /* valid but not built: sizes or path outside the instantiated set */
+    GDR_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    GDR_ERR_TIMEOUT = 4       /* a bounded device-side wait expired (see gdr_device_status) */
+} gdr_status;
+
+typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+typedef enum { GDR_GATE_SCALAR = 0, GDR_GATE_PER_KEY_CHANNEL = 1 } gdr_gate;
+
+/* Which kernels run the prefill.
+ *  GDR_PATH_AUTO        tensor-core path when it applies (bf16, d_k = d_v = 128,
+ *                       chunk = 64), else the SIMT path.
+ *  GDR_PATH_SIMT        fp32 CUDA-core kernels (any supported shape; the only
+ *                       path for fp32 inputs).
+ *  GDR_PATH_TENSORCORE  tcgen05/TMEM + TMA kernels; GDR_ERR_UNSUPPORTED where
+ *                       they do not apply. */
+typedef enum { GDR_PATH_AUTO = 0, GDR_PATH_SIMT = 1, GDR_PATH_TENSORCORE = 2 } gdr_path;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *gdr_status_string(gdr_status s);
+
+/*
+ * Bytes of device workspace gdr_fwd needs for these arguments and this path
+ * (0 if none).  Returns 0 as well for arguments gdr_fwd would reject.
+ * `n_seq` is the number of packed sequences when cu_seqlens is used, else
+ * ignored (pass 0).
+ */
+size_t gdr_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk, int n_seq,
+                              int varlen, gdr_dtype dtype, gdr_gate gate, gdr_path path);
+
+/*
+ * Chunkwise-parallel prefill over whole sequences (the chunked WY/UT form of
+ * "Linear Attention, Visualized", sections "Gated DeltaNet (GDN) / Complete
+ * per-chunk algorithm" and "Kimi Delta Attention (KDA) / Complete per-chunk
+ * algorithm"; the result equals the token recurrence above for every chunk
+ * size, section "Chunkwise algorithm / Cost").
+ *
+ *  q, k     [B, T, H, d_k]   dtype
+ *  v        [B, T, H, d_v]   dtype
+ *  g        [B, T, H] (GDR_GATE_SCALAR) or [B, T, H, d_k] (per channel), fp32
+ *  beta     [B, T, H]        fp32
+ *  S0       [N, H, d_v, d_k] fp32 initial states, or NULL for zero states
+ *  out      [B, T, H, d_v]   dtype, written for every token
+ *           (with B*T == 0 the token tensors may be NULL; S_final = S0)
+ *  S_final  [N, H, d_v, d_k] fp32 final states, or NULL to skip
+ *  chunk    16, 32 or 64 (SIMT); 64 (tensor-core path)
+ *  cu_seqlens  NULL: N = B sequences of length T.  Otherwise a DEVICE int32
+ *           array [n_seq + 1] of token offsets into a packed batch (B must be
+ *           1, cu_seqlens[0] = 0, cu_seqlens[n_seq] = T, non-decreasing); the
+ *           state restarts from S0[i] (or zero) at every sequence start and
+ *           N = n_seq.  Offsets live on the device and are not read by the
+ *           host; out-of-range or decreasing offsets are clamped into [0, T] by
+ *           the kernels (never an out-of-bounds access; such results are
+ *           unspecified).
+ *  d_k, d_v multiples of 16 in [16, 128] (SIMT); 128 (tensor-core path).
+ *  workspace / workspace_bytes: device scratch of at least
+ *           gdr_fwd_workspace_size(...) bytes, 256-byte aligned, owned by the
+ *           caller, not used by anything else until the call has completed on
+ *           `stream`.  May be NULL when that size is 0.
+ * Returns GDR_OK once the work is enqueued.
+ */
+gdr_status gdr_fwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const float *S0, void *out, float *S_final, int B, int T,
+                   int H, int d_k, int d_v, int chunk, const int32_t *cu_seqlens, int n_seq,
+                   gdr_dtype dtype, gdr_gate gate, gdr_path path, void *workspace,
+                   size_t workspace_bytes, void *stream);
+
+/*
+ * One decode step for N independent sequences, updating the states in place
+ * (the token recurrence above applied once; "Linear Attention, Visualized",
+ * DeltaNet / Recurrent form, with the decay of section "Gated DeltaNet (GDN)"
+ * or "Kimi Delta Attention (KDA)").
+ *
+ *  q, k     [N, H, d_k]        dtype
+ *  v        [N, H, d_v]        dtype
+ *  g        [N, H] or [N, H, d_k]  fp32 log-decay
+ *  beta     [N, H]             fp32
+ *  S_inout  [N, H, d_v, d_k]   fp32, read and overwritten
+ *  out      [N, H, d_v]        dtype
+ *  d_k in {64, 128}; d_v a multiple of 32 in [32, 256].
+ */
+gdr_status gdr_decode_step(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, float *S_inout, void *out, int N, int H, int d_k,
+                           int d_v, gdr_dtype dtype, gdr_gate gate, void *stream);
+
+/*
+ * Synchronises `stream`, then reports (and clears) the device-side error word
+ * of the current device: GDR_ERR_TIMEOUT if a bounded wait inside a kernel
+ * gave up since the last call (that kernel skipped its remaining work and
+ * returned), GDR_ERR_CUDA if the stream reports an error, else GDR_OK.
+ */
+gdr_status gdr_device_status(void *stream);
+
+/*
+ * Self-test of the bounded-wait error path: launches one tiny kernel that
+ * waits on a shared-memory barrier nobody arrives at, gives up after
+ * about `spin_limit` polls, records GDR_ERR_TIMEOUT in the device error word and
+ * returns normally (the context stays usable).  Follow with gdr_device_status.
+ */
+gdr_status gdr_selftest_wait_timeout(unsigned int spin_limit, void *stream);
+
+/*
+ * Per-kernel launch accounting and timing (a small built-in profiler).
+ * Kernel ids: GDR_K_DECODE, GDR_K_FWD_SIMT, GDR_K_TC_PLAN, GDR_K_TC_WY,
+ * GDR_K_TC_STATE.  Launches are always counted.  While timing is enabled,
+ * every launch is bracketed by two CUDA events recorded on the launch's own
+ * stream.  gdr_profile_read waits for the recorded events, returns the
+ * launches and the summed device time (ms) of kernel `id` since the last read
+ * of that id, and resets both.  Not thread-safe against concurrent gdr_* calls
+ * from other host threads.
+ */
+enum { GDR_K_DECODE = 0, GDR_K_FWD_SIMT = 1, GDR_K_TC_PLAN = 2, GDR_K_TC_WY = 3,
+       GDR_K_TC_STATE = 4, GDR_K_COUNT = 5 };
+void gdr_profile_enable(int on);
+gdr_status gdr_profile_read(int id, long long *launches, double *total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H */
