@@ -207,3 +207,90 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
     assert binding.device_status() == binding.GDR_ERR_TIMEOUT
     assert binding.device_status() == binding.GDR_OK  # cleared
     check(inputs.prefill_inputs(inputs.PREFILL["tiny_fp32"]), cuda_device)
+
+
+# ------------------------------------------------------------------ tensor-core prefill
+def sample_oracle(inp, heads, seqs=None):
+    """Oracle on a sample of (sequence, head) units: all tokens of the chosen
+    heads (and, for a regular batch, the chosen batch rows)."""
+    cfg = inp.cfg
+    hs = np.asarray(heads)
+    if inp.cu_seqlens is None:
+        bs = np.arange(cfg.B) if seqs is None else np.asarray(seqs)
+        sl = lambda x: np.ascontiguousarray(x[bs][:, :, hs])
+        S0 = None if inp.S0 is None else np.ascontiguousarray(inp.S0[bs][:, hs])
+        O, SF = oracle.recurrence_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.g), sl(inp.beta),
+                                      S0=S0)
+        return O, SF, (bs, hs)
+    sl = lambda x: np.ascontiguousarray(x[:, :, hs])
+    S0 = None if inp.S0 is None else np.ascontiguousarray(inp.S0[:, hs])
+    O, SF = oracle.recurrence_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.g), sl(inp.beta), S0=S0,
+                                  cu_seqlens=inp.cu_seqlens)
+    return O, SF, (None, hs)
+
+
+def check_sampled(inp, dev, heads, seqs=None, path="tc", tol=1e-2):
+    O, SF = run_fwd(inp, dev, path)
+    Or, SFr, (bs, hs) = sample_oracle(inp, heads, seqs)
+    if bs is None:
+        Og, SFg = O[:, :, hs], SF[:, hs]
+    else:
+        Og, SFg = O[bs][:, :, hs], SF[bs][:, hs]
+    eo, es = prefill_out_rel(Og, Or, inp.cu_seqlens), state_rel(SFg, SFr)
+    assert np.isfinite(O).all() and np.isfinite(SF).all()
+    assert eo <= tol and es <= tol, (eo, es)
+    return eo, es
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("T", [64, 300, 1])
+def test_tc_small_against_oracle(cuda_device, gate, T):
+    cfg = small_cfg(B=2, T=T, H=3, gate=gate, gate_scale=0.1 if gate == "scalar" else 0.05)
+    check(inputs.prefill_inputs(cfg, seed=301), cuda_device, path="tc")
+
+
+def test_tc_varlen_with_empty_and_unit_sequences(cuda_device):
+    cfg = inputs.PREFILL["varlen_prefill"].replace(T=600, H=2, n_seq=0, s0_var=0.01)
+    inp = inputs.prefill_inputs(cfg, seed=302)
+    inp.cu_seqlens = np.array([0, 0, 1, 65, 129, 200, 200, 600], dtype=np.int32)
+    inp.S0 = np.random.default_rng(6).standard_normal((7, 2, 128, 128)).astype(np.float32) * 0.1
+    check(inp, cuda_device, path="tc")
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_tc_matches_simt(cuda_device, gate):
+    cfg = small_cfg(B=1, T=515, H=4, gate=gate, gate_scale=0.1 if gate == "scalar" else 0.05)
+    inp = inputs.prefill_inputs(cfg, seed=303)
+    O1, S1 = run_fwd(inp, cuda_device, path="tc")
+    O2, S2 = run_fwd(inp, cuda_device, path="simt")
+    assert prefill_out_rel(O1, O2) < 1e-2 and state_rel(S1, S2) < 1e-2
+
+
+def test_tc_gdn_prefill_full_size_sampled(cuda_device):
+    """Gated DeltaNet prefill workload at full size (B=4, H=16, T=4096) in the
+    launch configuration the benchmark times; oracle on 3 heads x 4 sequences."""
+    inp = inputs.prefill_inputs(inputs.PREFILL["gdn_prefill"])
+    check_sampled(inp, cuda_device, heads=[0, 7, 15])
+
+
+def test_tc_kda_prefill_full_size_sampled(cuda_device):
+    """Per-channel-gate workload at full size (B=2, H=32, T=8192)."""
+    inp = inputs.prefill_inputs(inputs.PREFILL["kda_prefill"])
+    check_sampled(inp, cuda_device, heads=[0, 31])
+
+
+def test_tc_kda_prefill_nonzero_state_sampled(cuda_device):
+    cfg = inputs.PREFILL["kda_prefill"].replace(T=2048)
+    inp = inputs.prefill_inputs(cfg, s0_var=0.01)
+    check_sampled(inp, cuda_device, heads=[3, 17])
+
+
+def test_tc_varlen_prefill_full_size_sampled(cuda_device):
+    """Packed variable-length workload at full size (16 sequences, 65536 tokens)."""
+    inp = inputs.prefill_inputs(inputs.PREFILL["varlen_prefill"])
+    check_sampled(inp, cuda_device, heads=[5, 12])
+
+
+def test_tc_varlen_nonzero_state_sampled(cuda_device):
+    inp = inputs.prefill_inputs(inputs.PREFILL["varlen_prefill"], s0_var=0.01)
+    check_sampled(inp, cuda_device, heads=[1])
