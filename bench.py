@@ -481,6 +481,7 @@ def main():
     ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill",
                     help="comma-separated workloads measured after the main one ('' for none)")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-budget-s", type=float, default=90.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -504,7 +505,7 @@ def main():
         peaks, peak_kind = load_peaks()
         sampler = ClockSampler(local) if rank == 0 else None
         main_res = measure(args, args.workload, device, rank, world, peaks, peak_kind, args.path,
-                           args.steps, args.warmup, not args.no_cpu, True, sampler)
+                           args.steps, args.warmup, not args.no_cpu, not args.no_e2e, sampler)
         extra = {}
         for name in [x for x in args.extra.split(",") if x and x != args.workload]:
             steps = 20 if name != "decode" else 200

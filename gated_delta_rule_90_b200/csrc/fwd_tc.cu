@@ -48,7 +48,6 @@ using namespace sm100;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int kThreads = 128;
 constexpr uint32_t kSpin = 1u << 24;  // poll limit of every mbarrier wait
 constexpr uint32_t kTmemCols = 256;
 
@@ -65,7 +64,8 @@ struct Ws {
     int *chunk_start;  // [n_seq + 1] (varlen)
     int *order;        // [n_seq] longest first (varlen)
     float *dec;        // [slots*H][128]
-    __nv_bfloat16 *W, *U, *Q, *K;  // [slots*H][64][128]
+    __nv_bfloat16 *W, *U;          // transposed: [slots*H][128 (d)][64 (token)]
+    __nv_bfloat16 *Q, *K;          // [slots*H][64 (token)][128 (d)]
     __nv_bfloat16 *A;              // [slots*H][64][64]
 };
 
@@ -153,34 +153,44 @@ __global__ void plan_kernel(const int32_t *cu, int n_seq, int T_total, int *chun
 }
 
 // ------------------------------------------------------------------ WY kernel
+// 256 threads.  For accumulator epilogues, warp w serves TMEM lane quadrant
+// (w & 3) and column half (w >> 2).
+constexpr int kWyThreads = 256;
+
 struct WySmem {
-    static constexpr uint32_t KQ = 0;                    // [K;Q] raw, 2 atoms x 128 rows
+    static constexpr uint32_t KQ = 0;                    // [K;Q] raw, 2 atoms x 128 rows; later U^T|W^T staging
     static constexpr uint32_t V = KQ + 2 * 16384;        // 2 atoms x 64 rows
     static constexpr uint32_t KL = V + 2 * 8192;         // K<- (MMA A operand, MN-major)
-    static constexpr uint32_t TT = KL + 2 * 8192;        // T, K-major B operand
+    static constexpr uint32_t TT = KL + 2 * 8192;        // T (K-major B operand); A staging before
     static constexpr uint32_t KH = TT + 8192;            // KDA: [K^;Q^] scaled Gram A
     static constexpr uint32_t KC = KH + 2 * 16384;       // KDA: K-check, Gram B
     static constexpr uint32_t end_tc(bool ch) { return ch ? KC + 2 * 8192 : KH; }
-    static constexpr int NST = 68;                       // fp32 row stride of N
+    static constexpr int NST = 68;                       // fp32 row stride of N and X
 };
 
 template <bool CH>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kWyThreads)
 wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-          const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
+          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+          const __grid_constant__ CUtensorMap tm_Ust, const __grid_constant__ CUtensorMap tm_Wst,
+          const __grid_constant__ CUtensorMap tm_Ast, const float *__restrict__ g,
           const float *__restrict__ beta, const int32_t *__restrict__ cu, Geo geo, Ws ws,
           unsigned int *err) {
+    constexpr int NST = WySmem::NST;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint8_t *sKQ = sm + WySmem::KQ, *sV = sm + WySmem::V, *sKL = sm + WySmem::KL;
     uint8_t *sT = sm + WySmem::TT, *sKH = sm + WySmem::KH, *sKC = sm + WySmem::KC;
     float *sN = reinterpret_cast<float *>(sm + WySmem::end_tc(CH));   // [64][NST]
-    float *sG = sN + 64 * WySmem::NST;                                 // CH ? [64][128] : [64]
-    float *sB = sG + (CH ? 64 * D : 64);                               // beta [64]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 64);           // [2]
+    float *sX = sN + 64 * NST;                                          // [64][NST]
+    float *sG = sX + 64 * NST;                                          // CH ? [64][128] : [64]
+    float *sB = sG + (CH ? 64 * D : 64);                                // beta [64]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 64);            // [2]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qd = warp & 3, hf = warp >> 2;
+    const uint32_t lb = (uint32_t)(qd * 32) << 16;
     const int gcid = blockIdx.x, h = blockIdx.y;
     long tstart;
     int len;
@@ -205,7 +215,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_arrive_expect_tx(&bars[0], 6 * kHalfBytes);
+        mbar_arrive_expect_tx(&bars[0], 6 * kHalfBytes + (CH ? C * D * 4 : 0));
         const int x0 = h * D, y = (int)tstart;
         tma_load_2d(sKQ, &tm_k, &bars[0], x0, y);
         tma_load_2d(sKQ + 16384, &tm_k, &bars[0], x0 + 64, y);
@@ -213,25 +223,13 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         tma_load_2d(sKQ + 16384 + 8192, &tm_q, &bars[0], x0 + 64, y);
         tma_load_2d(sV, &tm_v, &bars[0], x0, y);
         tma_load_2d(sV + 8192, &tm_v, &bars[0], x0 + 64, y);
+        if (CH) tma_load_2d(sG, &tm_g, &bars[0], x0, y);  // [64][128] fp32 per-channel gates
     }
     // gates and beta (zero beyond the sequence end), cumulative log-decay G
-    if (CH) {
-        for (int e = tid; e < C * D; e += kThreads) {
-            const int l = e >> 7, c = e & 127;
-            sG[e] = (l < len) ? g[((size_t)(tstart + l) * geo.H + h) * D + c] : 0.f;
-        }
-    } else if (tid < C) {
-        sG[tid] = (tid < len) ? g[(size_t)(tstart + tid) * geo.H + h] : 0.f;
-    }
+    if (!CH && tid < C) sG[tid] = (tid < len) ? g[(size_t)(tstart + tid) * geo.H + h] : 0.f;
     if (tid < C) sB[tid] = (tid < len) ? beta[(size_t)(tstart + tid) * geo.H + h] : 0.f;
     __syncthreads();
-    if (CH) {
-        float acc = 0.f;  // thread = channel
-        for (int l = 0; l < C; ++l) {
-            acc += sG[l * D + tid];
-            sG[l * D + tid] = acc;
-        }
-    } else if (warp == 0) {
+    if (!CH && warp == 0) {
         float a = sG[lane], b = sG[lane + 32];
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -246,21 +244,37 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         sG[lane] = a;
         sG[lane + 32] = b;
     }
-    const bool ok_ld = mbar_wait_bounded(&bars[0], 0, kSpin, err);
-    if (!__syncthreads_and(ok_ld)) goto cleanup;
-
+    {
+        const bool ok_ld = mbar_wait_bounded(&bars[0], 0, kSpin, err);
+        if (!__syncthreads_and(ok_ld)) goto cleanup;
+    }
+    if (CH) {
+        // per-channel scan, rows past the sequence end count as g = 0: thread
+        // (c, half) scans 32 rows, the upper half then adds the lower half's total
+        const int c = tid & 127, r0 = (tid >> 7) * 32;
+        float acc = 0.f;
+        for (int l = r0; l < r0 + 32; ++l) {
+            if (l < len) acc += sG[l * D + c];
+            sG[l * D + c] = acc;
+        }
+        __syncthreads();
+        if (r0) {
+            const float base = sG[31 * D + c];
+            for (int l = 32; l < 64; ++l) sG[l * D + c] += base;
+        }
+    }
     // zero the rows beyond the sequence end (whole 128-byte rows: swizzle-agnostic)
     if (len < C) {
-        for (int e = tid; e < (C - len) * 8 * 6; e += kThreads) {
+        for (int e = tid; e < (C - len) * 8 * 6; e += kWyThreads) {
             const int r = len + e / 48, part = e % 48, tile = part >> 3, ch16 = part & 7;
             uint8_t *base = tile < 4 ? sKQ + (tile & 1) * 16384 + (tile >> 1) * 8192
                                      : sV + (tile & 1) * 8192;
             *reinterpret_cast<uint4 *>(base + r * 128 + ch16 * 16) = make_uint4(0, 0, 0, 0);
         }
-        __syncthreads();
     }
+    __syncthreads();
     // decayed operands: K<- = e^G . k (all gates); KDA also the scaled Gram operands
-    for (int e = tid; e < C * 16; e += kThreads) {
+    for (int e = tid; e < C * 16; e += kWyThreads) {
         const int l = e >> 4, a = (e >> 3) & 1, j = e & 7;
         const int c0 = a * 64 + ((j ^ (l & 7)) << 3);
         const uint32_t off = a * 16384 + l * 128 + j * 16;
@@ -270,9 +284,9 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll
             for (int i = 0; i < 8; ++i) w[i] = __expf(sG[l * D + c0 + i]);
         } else {
-            const float s = __expf(sG[l]);
+            const float sc = __expf(sG[l]);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = s;
+            for (int i = 0; i < 8; ++i) w[i] = sc;
         }
         float o[8];
 #pragma unroll
@@ -283,9 +297,9 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             unpack8(*reinterpret_cast<const uint4 *>(sKQ + off + 8192), qv);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float d = sG[l * D + c0 + i] - sG[31 * D + c0 + i];
-                e1[i] = __expf(d);
-                e2[i] = __expf(-d);
+                const float dlt = sG[l * D + c0 + i] - sG[31 * D + c0 + i];
+                e1[i] = __expf(dlt);
+                e2[i] = __expf(-dlt);
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) o[i] = kv[i] * e1[i];
@@ -324,59 +338,136 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     }
     tc_fence_after();
     {
-        // rows 0..63 of the accumulator: K K^T; rows 64..127: Q K^T
-        const int l = (warp & 1) * 32 + lane;
-        float gr[64];
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb)
-            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + cb * 16, gr + cb * 16);
+        // accumulator rows 0..63: K K^T -> N = diag(beta) tril_-1(. Gamma);
+        // rows 64..127: Q K^T -> A = tril_0(. Gamma), bf16, staged in the T tile
+        const int l = (qd & 1) * 32 + lane, m0 = hf * 32;
+        float gr[32];
+        tmem_ld16(tmem + lb + m0, gr);
+        tmem_ld16(tmem + lb + m0 + 16, gr + 16);
         tmem_wait_ld();
         const float Gl = CH ? 0.f : sG[l];
-        if (warp < 2) {
+        if (qd < 2) {
             const float bl = sB[l];
 #pragma unroll
-            for (int m = 0; m < 64; ++m) {
+            for (int i = 0; i < 32; ++i) {
+                const int m = m0 + i;
                 const float w = CH ? 1.f : __expf(Gl - sG[m]);
-                sN[l * WySmem::NST + m] = (m < l) ? bl * gr[m] * w : 0.f;
+                sN[l * NST + m] = (m < l) ? bl * gr[i] * w : 0.f;
             }
         } else {
-            __nv_bfloat16 *Ag = ws.A + slot * (C * C) + (size_t)l * C;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int jj = 0; jj < 4; ++jj) {
                 float o[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const int m = j * 8 + i;
+                    const int m = m0 + jj * 8 + i;
                     const float w = CH ? 1.f : __expf(Gl - sG[m]);
-                    o[i] = (m <= l) ? gr[m] * w : 0.f;
+                    o[i] = (m <= l) ? gr[jj * 8 + i] * w : 0.f;
                 }
-                *reinterpret_cast<uint4 *>(Ag + j * 8) = pack8(o);
+                const int j = hf * 4 + jj;
+                *reinterpret_cast<uint4 *>(sT + l * 128 + ((j ^ (l & 7)) << 4)) = pack8(o);
             }
         }
     }
+    fence_proxy_async_smem();
     __syncthreads();
-    // T: (I + N) T = diag(beta); thread j < 64 solves column j by forward substitution
-    if (tid < C) {
-        const int j = tid;
-        float t[C];
+    if (tid == 0) {  // A -> workspace
+        tma_store_2d(&tm_Ast, sT, 0, (int)(slot * C));
+        bulk_commit_group();
+    }
+    // T = (I + N)^{-1} diag(beta), N = diag(beta) L strictly lower, by 16 x 16
+    // blocks: X_ii = (I + N_ii)^{-1} by forward substitution (one column per
+    // thread), then X_ij = -X_ii sum_{k=j}^{i-1} N_ik X_kj, one block
+    // diagonal at a time (all fp32 in shared memory).
+    {
+        if (tid < C) {
+            const int b = tid >> 4, j = tid & 15;
+            const float *Nb = sN + (16 * b) * NST + 16 * b;
+            float x[16];
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            float acc = 0.f;
-            const float4 *row = reinterpret_cast<const float4 *>(sN + i * WySmem::NST);
+            for (int i = 0; i < 16; ++i) {
+                float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-            for (int m4 = 0; m4 < (i + 3) / 4; ++m4) {
-                const float4 nv = row[m4];
-                if (4 * m4 + 0 < i) acc = fmaf(nv.x, t[4 * m4 + 0], acc);
-                if (4 * m4 + 1 < i) acc = fmaf(nv.y, t[4 * m4 + 1], acc);
-                if (4 * m4 + 2 < i) acc = fmaf(nv.z, t[4 * m4 + 2], acc);
-                if (4 * m4 + 3 < i) acc = fmaf(nv.w, t[4 * m4 + 3], acc);
+                for (int m = 0; m < i; ++m) {
+                    if (m & 1) p1 = fmaf(Nb[i * NST + m], x[m], p1);
+                    else p0 = fmaf(Nb[i * NST + m], x[m], p0);
+                }
+                x[i] = ((i == j) ? 1.f : 0.f) - (p0 + p1);
             }
-            t[i] = ((i == j) ? sB[j] : 0.f) - acc;
-        }
-        // T[i][j] -> K-major SW128 tile (row i, column j)
 #pragma unroll
-        for (int i = 0; i < C; ++i)
-            *reinterpret_cast<__nv_bfloat16 *>(sT + sw128_off(i, j)) = __float2bfloat16_rn(t[i]);
+            for (int i = 0; i < 16; ++i) sX[(16 * b + i) * NST + 16 * b + j] = x[i];
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int dd = 1; dd < 4; ++dd) {
+            const int nout = (4 - dd) * 256;
+            // P_ij = sum_k N_ik X_kj, written into block (i, j) of X (not read in this pass)
+#pragma unroll
+            for (int kq = 0; kq < 3; ++kq) {
+                const int e = tid + kq * kWyThreads;
+                if (e < nout) {
+                    const int j = e >> 8, i = j + dd, r = (e >> 4) & 15, c = e & 15;
+                    float p0 = 0.f, p1 = 0.f;
+                    for (int kb = j; kb < i; ++kb) {
+                        const float4 *nr = reinterpret_cast<const float4 *>(sN + (16 * i + r) * NST + 16 * kb);
+                        const float *xc = sX + (16 * kb) * NST + 16 * j + c;
+#pragma unroll
+                        for (int m4 = 0; m4 < 4; ++m4) {
+                            const float4 nv = nr[m4];
+                            p0 = fmaf(nv.x, xc[(4 * m4 + 0) * NST], p0);
+                            p1 = fmaf(nv.y, xc[(4 * m4 + 1) * NST], p1);
+                            p0 = fmaf(nv.z, xc[(4 * m4 + 2) * NST], p0);
+                            p1 = fmaf(nv.w, xc[(4 * m4 + 3) * NST], p1);
+                        }
+                    }
+                    sX[(16 * i + r) * NST + 16 * j + c] = p0 + p1;
+                }
+            }
+            __syncthreads();
+            float res[3];
+#pragma unroll
+            for (int kq = 0; kq < 3; ++kq) {
+                const int e = tid + kq * kWyThreads;
+                res[kq] = 0.f;
+                if (e < nout) {
+                    const int j = e >> 8, i = j + dd, r = (e >> 4) & 15, c = e & 15;
+                    const float4 *xr = reinterpret_cast<const float4 *>(sX + (16 * i + r) * NST + 16 * i);
+                    const float *pc = sX + (16 * i) * NST + 16 * j + c;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m4 = 0; m4 < 4; ++m4) {
+                        const float4 xv = xr[m4];  // X_ii is lower triangular: zeros above
+                        acc = fmaf(xv.x, pc[(4 * m4 + 0) * NST], acc);
+                        acc = fmaf(xv.y, pc[(4 * m4 + 1) * NST], acc);
+                        acc = fmaf(xv.z, pc[(4 * m4 + 2) * NST], acc);
+                        acc = fmaf(xv.w, pc[(4 * m4 + 3) * NST], acc);
+                    }
+                    res[kq] = -acc;
+                }
+            }
+            if (dd == 3 && tid == 0) bulk_wait_group_read<0>();  // the A staging is read
+            __syncthreads();
+#pragma unroll
+            for (int kq = 0; kq < 3; ++kq) {
+                const int e = tid + kq * kWyThreads;
+                if (e < nout) {
+                    const int j = e >> 8, i = j + dd, r = (e >> 4) & 15, c = e & 15;
+                    sX[(16 * i + r) * NST + 16 * j + c] = res[kq];
+                }
+            }
+            __syncthreads();
+        }
+        // T[i][j] = X[i][j] beta_j (lower triangle) -> bf16, K-major SW128 tile
+        for (int e = tid; e < C * 8; e += kWyThreads) {
+            const int i = e >> 3, j8 = e & 7;
+            float o[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j8 * 8 + u;
+                o[u] = (j <= i) ? sX[i * NST + j] * sB[j] : 0.f;
+            }
+            *reinterpret_cast<uint4 *>(sT + i * 128 + ((j8 ^ (i & 7)) << 4)) = pack8(o);
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -398,87 +489,118 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     // meanwhile: Q<- and K-> to the workspace, and the chunk decay
     {
         __nv_bfloat16 *Qg = ws.Q + slot * (C * D), *Kg = ws.K + slot * (C * D);
-        for (int e = tid; e < C * 16; e += kThreads) {
+        for (int e = tid; e < C * 16; e += kWyThreads) {
             const int l = e >> 4, a = (e >> 3) & 1, j = e & 7;
             const int c0 = a * 64 + ((j ^ (l & 7)) << 3);
             const uint32_t off = a * 16384 + l * 128 + j * 16;
             float kv[8], qv[8], wq[8], wk[8];
             unpack8(*reinterpret_cast<const uint4 *>(sKQ + off), kv);
             unpack8(*reinterpret_cast<const uint4 *>(sKQ + off + 8192), qv);
+            if (CH) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float Gl = CH ? sG[l * D + c0 + i] : sG[l];
-                const float Gc = CH ? sG[(C - 1) * D + c0 + i] : sG[C - 1];
-                wq[i] = qv[i] * __expf(Gl);
-                wk[i] = kv[i] * __expf(Gc - Gl);
+                for (int i = 0; i < 8; ++i) {
+                    const float Gl = sG[l * D + c0 + i];
+                    wq[i] = qv[i] * __expf(Gl);
+                    wk[i] = kv[i] * __expf(sG[(C - 1) * D + c0 + i] - Gl);
+                }
+            } else {
+                const float eq = __expf(sG[l]), ek = __expf(sG[C - 1] - sG[l]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    wq[i] = qv[i] * eq;
+                    wk[i] = kv[i] * ek;
+                }
             }
             *reinterpret_cast<uint4 *>(Qg + l * D + c0) = pack8(wq);
             *reinterpret_cast<uint4 *>(Kg + l * D + c0) = pack8(wk);
         }
-        ws.dec[slot * D + tid] = __expf(CH ? sG[(C - 1) * D + tid] : sG[C - 1]);
+        if (tid < D) ws.dec[slot * D + tid] = __expf(CH ? sG[(C - 1) * D + tid] : sG[C - 1]);
     }
     {
         const bool ok = mbar_wait_bounded(&bars[1], 1, kSpin, err);
-        if (!__syncthreads_and(ok)) goto cleanup;
+        if (!__syncthreads_and(ok)) goto cleanup;  // also: the raw K/Q tiles are no longer read
     }
     tc_fence_after();
     {
-        // thread = feature row d of U^T / W<-^T; write U[l][d], W[l][d]
-        const int d = tid;
-        __nv_bfloat16 *Ug = ws.U + slot * (C * D), *Wg = ws.W + slot * (C * D);
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // U^T, W<-^T rows (feature d, 32 tokens each) -> staging in the K/Q area
+        // (128 x 64 bf16, 128-byte swizzle) -> TMA stores
+        const int d = qd * 32 + lane;
+        float u[32], w[32];
+        tmem_ld16(tmem + lb + 64 + hf * 32, u);
+        tmem_ld16(tmem + lb + 64 + hf * 32 + 16, u + 16);
+        tmem_ld16(tmem + lb + 128 + hf * 32, w);
+        tmem_ld16(tmem + lb + 128 + hf * 32 + 16, w + 16);
+        tmem_wait_ld();
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float u[16], w[16];
-            tmem_ld16(tmem + lane_base + 64 + cb * 16, u);
-            tmem_ld16(tmem + lane_base + 128 + cb * 16, w);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int l = cb * 16 + i;
-                Ug[l * D + d] = __float2bfloat16_rn(u[i]);
-                Wg[l * D + d] = __float2bfloat16_rn(w[i]);
-            }
+        for (int jj = 0; jj < 4; ++jj) {
+            const int j = hf * 4 + jj;
+            const uint32_t off = d * 128 + ((j ^ (d & 7)) << 4);
+            *reinterpret_cast<uint4 *>(sKQ + off) = pack8(u + jj * 8);
+            *reinterpret_cast<uint4 *>(sKQ + 16384 + off) = pack8(w + jj * 8);
         }
     }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tma_store_2d(&tm_Ust, sKQ, 0, (int)(slot * D));
+        tma_store_2d(&tm_Wst, sKQ + 16384, 0, (int)(slot * D));
+        bulk_commit_group();
+    }
 cleanup:
+    if (tid == 0) bulk_wait_group<0>();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------ state kernel
+// Warp roles (13 warps):
+//   warps 0-7   state chain: S epilogue and Z epilogue.  Warp w serves TMEM
+//               lane quadrant (w & 3) -- state rows d = 32 (w & 3) + lane -- and
+//               column half (w >> 2) of the accumulators it touches.
+//   warps 8-11  output: O^T (TMEM) -> shared staging -> TMA store.
+//   warp 12     producer: TMA loads of the next chunks and every tcgen05.mma.
+// The roles hand over through mbarriers only; the chain never waits on the
+// output path.  TMEM columns: S [0,128), Z^T [128,192), O^T x2 [192,320).
 struct StSmem {
-    // per stage: W, Q, K, U (16 KB each, 2 atom columns of 8 KB), A (8 KB), decay (512 B)
-    static constexpr uint32_t W = 0, Q = 16384, K = 32768, U = 49152, A = 65536, DEC = 73728;
-    static constexpr uint32_t STAGE = 74752;  // 73 KB, multiple of 1024
-    static constexpr uint32_t S = 2 * STAGE;  // bf16 S, 2 atom columns x 128 rows
-    static constexpr uint32_t ZT = S + 32768; // bf16 Z^T, 128 rows x 64
-    static constexpr uint32_t BARS = ZT + 16384;
-    static constexpr uint32_t TOTAL = BARS + 64;
+    // per stage: W<-^T (128 x 64, MN-major B), Q<- (64 x 128, K-major B),
+    // K-> (64 x 128, MN-major B), U^T (128 x 64), A (64 x 64, K-major B)
+    static constexpr uint32_t WT = 0, Q = 16384, K = 32768, UT = 49152, A = 65536;
+    static constexpr uint32_t STAGE = 73728;
+    static constexpr uint32_t DEC = 2 * STAGE;      // decay [2][128] fp32
+    static constexpr uint32_t S = DEC + 1024;       // bf16 S, K-major A operand (2 atoms)
+    static constexpr uint32_t ZT = S + 32768;       // bf16 Z^T, K-major A operand
+    static constexpr uint32_t OST = ZT + 16384;     // O staging for the TMA store [64][128]
+    static constexpr uint32_t BARS = OST + 16384;
+    static constexpr uint32_t TOTAL = BARS + 256;
     static constexpr uint32_t TX = 4 * kTileBytes + kHalfBytes + kDecBytes;
 };
+constexpr int kChainThreads = 256, kOutThreads = 128;
+constexpr int kStThreads = kChainThreads + kOutThreads + 32;
+constexpr uint32_t kStTmemCols = 512;
 
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
-                                          uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kStThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ CUtensorMap tm_U,
              const __grid_constant__ CUtensorMap tm_Q, const __grid_constant__ CUtensorMap tm_K,
-             const __grid_constant__ CUtensorMap tm_A, const float *__restrict__ S0,
-             __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
-             const int32_t *__restrict__ cu, Geo geo, Ws ws, unsigned int *err) {
+             const __grid_constant__ CUtensorMap tm_A, const __grid_constant__ CUtensorMap tm_out,
+             const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
+             float *__restrict__ S_final, const int32_t *__restrict__ cu, Geo geo, Ws ws,
+             unsigned int *err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + StSmem::BARS);  // full[2], mma
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 3);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + StSmem::BARS);  // [2] TMA stage loaded
+    uint64_t *opsS = full + 2;   // chain: S operand + decayed S ready    (count 256)
+    uint64_t *opsZ = full + 3;   // chain: Z^T operand ready               (count 256)
+    uint64_t *barZ = full + 4;   // mma: Z^T accumulated
+    uint64_t *barS = full + 5;   // mma: S update accumulated
+    uint64_t *barO = full + 6;   // [2] mma: O^T buffer complete
+    uint64_t *oFree = full + 8;  // [2] output warps: O^T buffer read (count 128)
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(full + 10);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int unit = blockIdx.x;
     const int s = geo.varlen ? ws.order[unit / geo.H] : unit / geo.H;
     const int h = unit % geo.H;
@@ -486,195 +608,231 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
     seq_bounds(cu, s, geo.T, geo.T_total, t0, t1);
     const int gc0 = geo.varlen ? ws.chunk_start[s] : s * geo.nc;
     const int nch = (int)((t1 - t0 + C - 1) / C);
-    const int d = tid;  // state row owned by this thread (TMEM lane)
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const size_t soff = ((size_t)s * geo.H + h) * (size_t)D * D + (size_t)d * D;
 
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_init(&bars[2], 1);
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(opsS, kChainThreads);
+        mbar_init(opsZ, kChainThreads);
+        mbar_init(barZ, 1);
+        mbar_init(barS, 1);
+        mbar_init(&barO[0], 1);
+        mbar_init(&barO[1], 1);
+        mbar_init(&oFree[0], kOutThreads);
+        mbar_init(&oFree[1], kOutThreads);
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tslot, kTmemCols);
+        tmem_alloc(tslot, kStTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t tS = tmem, tZ = tmem + 128, tO = tmem + 192;
+    const uint32_t tS = tmem, tZ = tmem + 128, tO0 = tmem + 192;
+    bool ok = true;
 
-    auto issue = [&](int r) {
-        uint8_t *st = sm + (r & 1) * StSmem::STAGE;
-        uint64_t *bar = &bars[r & 1];
-        const size_t sl = (size_t)(gc0 + r) * geo.H + h;
-        const int y = (int)(sl * C);
-        mbar_arrive_expect_tx(bar, StSmem::TX);
-        tma_load_2d(st + StSmem::W, &tm_W, bar, 0, y);
-        tma_load_2d(st + StSmem::W + 8192, &tm_W, bar, 64, y);
-        tma_load_2d(st + StSmem::Q, &tm_Q, bar, 0, y);
-        tma_load_2d(st + StSmem::Q + 8192, &tm_Q, bar, 64, y);
-        tma_load_2d(st + StSmem::K, &tm_K, bar, 0, y);
-        tma_load_2d(st + StSmem::K + 8192, &tm_K, bar, 64, y);
-        tma_load_2d(st + StSmem::U, &tm_U, bar, 0, y);
-        tma_load_2d(st + StSmem::U + 8192, &tm_U, bar, 64, y);
-        tma_load_2d(st + StSmem::A, &tm_A, bar, 0, y);
-        bulk_load(st + StSmem::DEC, ws.dec + sl * D, kDecBytes, bar);
-    };
-    if (tid == 0 && nch > 0) {
-        prefetch_tmap(&tm_W);
-        prefetch_tmap(&tm_U);
-        prefetch_tmap(&tm_Q);
-        prefetch_tmap(&tm_K);
-        prefetch_tmap(&tm_A);
-        issue(0);
-    }
-    // S <- S0 (or 0) in TMEM
+    if (warp < 8) {
+        // ===================== state chain =====================
+        const int qd = warp & 3, hf = warp >> 2;
+        const int d = qd * 32 + lane;
+        const uint32_t lb = (uint32_t)(qd * 32) << 16;
+        const size_t soff = ((size_t)s * geo.H + h) * (size_t)D * D + (size_t)d * D + hf * 64;
 #pragma unroll
-    for (int cb = 0; cb < 8; ++cb) {
-        float v[16];
+        for (int cb = 0; cb < 4; ++cb) {  // S <- S0 (or 0)
+            float v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = S0 ? S0[soff + cb * 16 + i] : 0.f;
-        tmem_st16(tS + lane_base + cb * 16, v);
-    }
-    tmem_wait_st();
-
-    uint32_t mma_phase = 0;
-    for (int r = 0; r < nch; ++r) {
-        uint8_t *st = sm + (r & 1) * StSmem::STAGE;
-        const long tstart = t0 + (long)r * C;
-        const int len = (int)min((long)C, t1 - tstart);
-        if (tid == 0 && r + 1 < nch) {
-            fence_proxy_async_smem();
-            issue(r + 1);
+            for (int i = 0; i < 16; ++i) v[i] = S0 ? S0[soff + cb * 16 + i] : 0.f;
+            tmem_st16(tS + lb + hf * 64 + cb * 16, v);
         }
-        {
-            const bool ok = mbar_wait_bounded(&bars[r & 1], (r >> 1) & 1, kSpin, err);
-            if (!__syncthreads_and(ok)) goto cleanup;
-        }
-        // S (fp32, TMEM) -> bf16 operand in smem; S <- S Diag(decay) in TMEM
-        {
-            const float *dec = reinterpret_cast<const float *>(st + StSmem::DEC);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+        tmem_wait_st();
+        for (int r = 0; r < nch && ok; ++r) {
+            const uint8_t *st = sm + (r & 1) * StSmem::STAGE;
+            ok = mbar_wait_bounded(&full[r & 1], (r >> 1) & 1, kSpin, err);
+            if (r > 0) ok = ok && mbar_wait_bounded(barS, (r - 1) & 1, kSpin, err);
+            if (!ok) break;
+            tc_fence_after();
+            {   // S (fp32) -> bf16 operand; S <- S Diag(decay) in TMEM
+                const float *dec = reinterpret_cast<const float *>(sm + StSmem::DEC) +
+                                   (r & 1) * D + hf * 64;
                 float v[64];
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb)
-                    tmem_ld16(tS + lane_base + half * 64 + cb * 16, v + cb * 16);
+                for (int cb = 0; cb < 4; ++cb) tmem_ld16(tS + lb + hf * 64 + cb * 16, v + cb * 16);
                 tmem_wait_ld();
-                uint8_t *rowp = sm + StSmem::S + half * 16384 + d * 128;
+                uint8_t *rowp = sm + StSmem::S + hf * 16384 + d * 128;
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     *reinterpret_cast<uint4 *>(rowp + ((j ^ (d & 7)) << 4)) = pack8(v + j * 8);
 #pragma unroll
-                for (int i = 0; i < 64; ++i) v[i] *= dec[half * 64 + i];
+                for (int i = 0; i < 64; ++i) v[i] *= dec[i];
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) tmem_st16(tS + lane_base + half * 64 + cb * 16, v + cb * 16);
+                for (int cb = 0; cb < 4; ++cb) tmem_st16(tS + lb + hf * 64 + cb * 16, v + cb * 16);
+                tmem_wait_st();
             }
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(opsS);
+            ok = mbar_wait_bounded(barZ, r & 1, kSpin, err);
+            if (!ok) break;
             tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk & 3) * 32;
-                const uint64_t a =
-                    sdesc_sw128(smem_u32(sm + StSmem::S + (kk >> 2) * 16384 + koff), 16, 1024);
-                const uint64_t bw =
-                    sdesc_sw128(smem_u32(st + StSmem::W + (kk >> 2) * 8192 + koff), 16, 1024);
-                const uint64_t bq =
-                    sdesc_sw128(smem_u32(st + StSmem::Q + (kk >> 2) * 8192 + koff), 16, 1024);
-                mma_bf16_ss(tZ, a, bw, id, kk > 0);
-                mma_bf16_ss(tO, a, bq, id, kk > 0);
-            }
-            mma_commit(&bars[2]);
-        }
-        {
-            const bool ok = mbar_wait_bounded(&bars[2], mma_phase, kSpin, err);
-            mma_phase ^= 1;
-            if (!__syncthreads_and(ok)) goto cleanup;
-        }
-        tc_fence_after();
-        // Z^T = U^T - S W<-^T  -> bf16 K-major operand in smem
-        {
-            float z[64];
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tZ + lane_base + cb * 16, z + cb * 16);
-            tmem_wait_ld();
-            const uint8_t *Ut = st + StSmem::U + (d >> 6) * 8192;
-#pragma unroll
-            for (int l = 0; l < 64; ++l) {
-                const float u = __bfloat162float(
-                    *reinterpret_cast<const __nv_bfloat16 *>(Ut + sw128_off(l, d & 63)));
-                z[l] = u - z[l];
-            }
-            uint8_t *rowp = sm + StSmem::ZT + d * 128;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<uint4 *>(rowp + ((j ^ (d & 7)) << 4)) = pack8(z + j * 8);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t idO = idesc_bf16(128, 64, 0, 0);
-            const uint32_t idS = idesc_bf16(128, 128, 0, 1);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t a = sdesc_sw128(smem_u32(sm + StSmem::ZT + kk * 32), 16, 1024);
-                const uint64_t ba = sdesc_sw128(smem_u32(st + StSmem::A + kk * 32), 16, 1024);
-                const uint64_t bk = sdesc_sw128(smem_u32(st + StSmem::K + kk * 2048), 8192, 1024);
-                mma_bf16_ss(tO, a, ba, idO, 1);
-                mma_bf16_ss(tS, a, bk, idS, 1);
-            }
-            mma_commit(&bars[2]);
-        }
-        {
-            const bool ok = mbar_wait_bounded(&bars[2], mma_phase, kSpin, err);
-            mma_phase ^= 1;
-            if (!__syncthreads_and(ok)) goto cleanup;
-        }
-        tc_fence_after();
-        // O^T (TMEM) -> out[t, h, d]
-        {
-            __nv_bfloat16 *og = out + ((size_t)tstart * geo.H + h) * D + d;
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                float o[16];
-                tmem_ld16(tO + lane_base + cb * 16, o);
+            {   // Z^T = U^T - S W<-^T -> bf16 K-major operand (this thread: 32 tokens)
+                float z[32];
+                tmem_ld16(tZ + lb + hf * 32, z);
+                tmem_ld16(tZ + lb + hf * 32 + 16, z + 16);
                 tmem_wait_ld();
+                const uint8_t *urow = st + StSmem::UT + d * 128;
+                uint8_t *zrow = sm + StSmem::ZT + d * 128;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int l = cb * 16 + i;
-                    if (l < len) og[(size_t)l * geo.H * D] = __float2bfloat16_rn(o[i]);
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = hf * 4 + jj;
+                    float u[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(urow + ((j ^ (d & 7)) << 4)), u);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) u[i] -= z[jj * 8 + i];
+                    *reinterpret_cast<uint4 *>(zrow + ((j ^ (d & 7)) << 4)) = pack8(u);
                 }
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(opsZ);
         }
-        __syncthreads();
-    }
-    if (S_final) {
+        if (ok && nch > 0) ok = mbar_wait_bounded(barS, (nch - 1) & 1, kSpin, err);
+        tc_fence_after();
+        if (ok && S_final) {
 #pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
-            float v[16];
-            tmem_ld16(tS + lane_base + cb * 16, v);
+            for (int cb = 0; cb < 4; ++cb) {
+                float v[16];
+                tmem_ld16(tS + lb + hf * 64 + cb * 16, v);
+                tmem_wait_ld();
+                float4 *dst = reinterpret_cast<float4 *>(S_final + soff + cb * 16);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+        }
+    } else if (warp < 12) {
+        // ===================== output =====================
+        const int qd = warp & 3;
+        const int d = qd * 32 + lane;
+        const int otid = tid - kChainThreads;
+        const uint32_t lb = (uint32_t)(qd * 32) << 16;
+        __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(sm + StSmem::OST);
+        for (int r = 0; r < nch && ok; ++r) {
+            ok = mbar_wait_bounded(&barO[r & 1], (r >> 1) & 1, kSpin, err);
+            if (!ok) break;
+            tc_fence_after();
+            float o[64];
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tO0 + (r & 1) * 64 + lb + cb * 16, o + cb * 16);
             tmem_wait_ld();
-            float4 *dst = reinterpret_cast<float4 *>(S_final + soff + cb * 16);
+            tc_fence_before();
+            mbar_arrive(&oFree[r & 1]);
+            const long ts = t0 + (long)r * C;
+            const int len = (int)min((long)C, t1 - ts);
+            if (len == C) {
+                if (otid == 0) bulk_wait_group_read<0>();  // staging buffer free again
+                named_sync(1, kOutThreads);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                for (int i = 0; i < 64; ++i) ost[i * D + d] = __float2bfloat16_rn(o[i]);
+                fence_proxy_async_smem();
+                named_sync(1, kOutThreads);
+                if (otid == 0) {
+                    tma_store_2d(&tm_out, ost, h * D, (int)ts);
+                    bulk_commit_group();
+                }
+            } else {
+                __nv_bfloat16 *og = out + ((size_t)ts * geo.H + h) * D + d;
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if (i < len) og[(size_t)i * geo.H * D] = __float2bfloat16_rn(o[i]);
+            }
+        }
+        if (otid == 0) bulk_wait_group<0>();
+    } else if (lane == 0) {
+        // ===================== producer: TMA + MMA =====================
+        auto issue = [&](int r) {
+            uint8_t *st = sm + (r & 1) * StSmem::STAGE;
+            uint64_t *bar = &full[r & 1];
+            const size_t sl = (size_t)(gc0 + r) * geo.H + h;
+            mbar_arrive_expect_tx(bar, StSmem::TX);
+            tma_load_2d(st + StSmem::WT, &tm_W, bar, 0, (int)(sl * D));
+            tma_load_2d(st + StSmem::UT, &tm_U, bar, 0, (int)(sl * D));
+            tma_load_2d(st + StSmem::Q, &tm_Q, bar, 0, (int)(sl * C));
+            tma_load_2d(st + StSmem::Q + 8192, &tm_Q, bar, 64, (int)(sl * C));
+            tma_load_2d(st + StSmem::K, &tm_K, bar, 0, (int)(sl * C));
+            tma_load_2d(st + StSmem::K + 8192, &tm_K, bar, 64, (int)(sl * C));
+            tma_load_2d(st + StSmem::A, &tm_A, bar, 0, (int)(sl * C));
+            bulk_load(sm + StSmem::DEC + (r & 1) * kDecBytes, ws.dec + sl * D, kDecBytes, bar);
+        };
+        if (nch > 0) {
+            prefetch_tmap(&tm_W);
+            prefetch_tmap(&tm_U);
+            prefetch_tmap(&tm_Q);
+            prefetch_tmap(&tm_K);
+            prefetch_tmap(&tm_A);
+            prefetch_tmap(&tm_out);
+            issue(0);
+            if (nch > 1) issue(1);
+        }
+        const uint32_t idZ = idesc_bf16(128, 64, 0, 1);
+        const uint32_t idO = idesc_bf16(128, 64, 0, 0);
+        const uint32_t idS = idesc_bf16(128, 128, 0, 1);
+        for (int r = 0; r < nch && ok; ++r) {
+            const uint8_t *st = sm + (r & 1) * StSmem::STAGE;
+            const uint32_t tO = tO0 + (r & 1) * 64;
+            ok = mbar_wait_bounded(opsS, r & 1, kSpin, err);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {  // Z^T = S W<-^T
+                const uint64_t a =
+                    sdesc_sw128(smem_u32(sm + StSmem::S + (kk >> 2) * 16384 + (kk & 3) * 32), 16, 1024);
+                const uint64_t bw = sdesc_sw128(smem_u32(st + StSmem::WT + kk * 2048), 16384, 1024);
+                mma_bf16_ss(tZ, a, bw, idZ, kk > 0);
+            }
+            mma_commit(barZ);
+            if (r >= 2) ok = mbar_wait_bounded(&oFree[r & 1], ((r - 2) >> 1) & 1, kSpin, err);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {  // O^T = S Q<-^T
+                const uint64_t a =
+                    sdesc_sw128(smem_u32(sm + StSmem::S + (kk >> 2) * 16384 + (kk & 3) * 32), 16, 1024);
+                const uint64_t bq =
+                    sdesc_sw128(smem_u32(st + StSmem::Q + (kk >> 2) * 8192 + (kk & 3) * 32), 16, 1024);
+                mma_bf16_ss(tO, a, bq, idO, kk > 0);
+            }
+            ok = mbar_wait_bounded(opsZ, r & 1, kSpin, err);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {  // S += Z^T K->
+                const uint64_t a = sdesc_sw128(smem_u32(sm + StSmem::ZT + kk * 32), 16, 1024);
+                const uint64_t bk = sdesc_sw128(smem_u32(st + StSmem::K + kk * 2048), 8192, 1024);
+                mma_bf16_ss(tS, a, bk, idS, 1);
+            }
+            mma_commit(barS);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {  // O^T += Z^T A^T
+                const uint64_t a = sdesc_sw128(smem_u32(sm + StSmem::ZT + kk * 32), 16, 1024);
+                const uint64_t ba = sdesc_sw128(smem_u32(st + StSmem::A + kk * 32), 16, 1024);
+                mma_bf16_ss(tO, a, ba, idO, 1);
+            }
+            mma_commit(&barO[r & 1]);
+            // this stage is free once chunk r's MMAs are done: prefetch chunk r+2
+            if (r + 2 < nch) {
+                ok = mbar_wait_bounded(&barO[r & 1], (r >> 1) & 1, kSpin, err);
+                if (!ok) break;
+                issue(r + 2);
+            }
         }
     }
-cleanup:
+    // every role ends here; the chain and output roles have waited for the
+    // last MMAs, so TMEM can be released
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 0) tmem_dealloc(tmem, kStTmemCols);
 }
 
 }  // namespace tc
@@ -723,23 +881,29 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map: inner extent `inner` elements, `rows` rows, row pitch
-// `pitch` bytes, box 64 x 64, 128-byte swizzle, zero fill out of bounds.
-bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t pitch) {
+// 2-D tensor map: inner extent `inner` elements, `rows` rows, row pitch
+// `pitch` bytes, box box0 x box1, zero fill out of bounds.
+bool make_map(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t inner,
+              uint64_t rows, uint64_t pitch, uint32_t box0, uint32_t box1,
+              CUtensorMapSwizzle swz) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {pitch};
-    cuuint32_t box[2] = {64, 64};
+    cuuint32_t box[2] = {box0, box1};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(m, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+constexpr CUtensorMapDataType kBF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+constexpr CUtensorMapDataType kF32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+constexpr CUtensorMapSwizzle kSW = CU_TENSOR_MAP_SWIZZLE_128B;
+constexpr CUtensorMapSwizzle kNoSW = CU_TENSOR_MAP_SWIZZLE_NONE;
 
-size_t wy_smem_bytes(bool ch) {
-    return 1024 + WySmem::end_tc(ch) + 4 * (64 * WySmem::NST + (ch ? 64 * D : 64) + 64) + 64;
+size_t wy_smem_bytes(bool ch) {  // + 1024 for the in-kernel alignment
+    return 1024 + WySmem::end_tc(ch) + 4 * (2 * 64 * WySmem::NST + (ch ? 64 * D : 64) + 64) + 64;
 }
 
 }  // namespace
@@ -776,22 +940,29 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
     geo.B = B; geo.T = T; geo.H = H; geo.n_seq = varlen ? n_seq : B;
     geo.nc = (T + C - 1) / C; geo.varlen = varlen; geo.T_total = B * T; geo.n_slots = L.n_slots;
 
-    const size_t tile_rows = (size_t)L.n_slots * H * C;
-    if (tile_rows >= (size_t)1 << 31) return cudaErrorInvalidValue;  // 32-bit TMA row coordinates
+    const size_t tiles = (size_t)L.n_slots * H;
+    if (tiles * D >= ((size_t)1 << 31)) return cudaErrorInvalidValue;  // 32-bit TMA rows
     const uint64_t tok_rows = (uint64_t)B * T;
-    CUtensorMap mq, mk, mv, mW, mU, mQ, mK, mA;
+    const uint64_t HD = (uint64_t)H * D;
+    CUtensorMap mq, mk, mv, mg, mW, mU, mQ, mK, mA, mo;
+    memset(&mg, 0, sizeof(mg));
     const bool have_tokens = tok_rows > 0;
     if (have_tokens) {
-        if (!make_map(&mq, q, (uint64_t)H * D, tok_rows, (uint64_t)H * D * 2) ||
-            !make_map(&mk, k, (uint64_t)H * D, tok_rows, (uint64_t)H * D * 2) ||
-            !make_map(&mv, v, (uint64_t)H * D, tok_rows, (uint64_t)H * D * 2) ||
-            !make_map(&mW, ws.W, D, tile_rows, D * 2) || !make_map(&mU, ws.U, D, tile_rows, D * 2) ||
-            !make_map(&mQ, ws.Q, D, tile_rows, D * 2) || !make_map(&mK, ws.K, D, tile_rows, D * 2) ||
-            !make_map(&mA, ws.A, C, tile_rows, C * 2))
+        if (!make_map(&mq, kBF, q, HD, tok_rows, HD * 2, 64, 64, kSW) ||
+            !make_map(&mk, kBF, k, HD, tok_rows, HD * 2, 64, 64, kSW) ||
+            !make_map(&mv, kBF, v, HD, tok_rows, HD * 2, 64, 64, kSW) ||
+            (gate == GDR_GATE_PER_KEY_CHANNEL &&
+             !make_map(&mg, kF32, g, HD, tok_rows, HD * 4, D, 64, kNoSW)) ||
+            !make_map(&mW, kBF, ws.W, C, tiles * D, C * 2, 64, 128, kSW) ||
+            !make_map(&mU, kBF, ws.U, C, tiles * D, C * 2, 64, 128, kSW) ||
+            !make_map(&mQ, kBF, ws.Q, D, tiles * C, D * 2, 64, 64, kSW) ||
+            !make_map(&mK, kBF, ws.K, D, tiles * C, D * 2, 64, 64, kSW) ||
+            !make_map(&mA, kBF, ws.A, C, tiles * C, C * 2, 64, 64, kSW) ||
+            !make_map(&mo, kBF, out, HD, tok_rows, HD * 2, D, 64, kNoSW))
             return cudaErrorInvalidValue;
     } else {
         memset(&mW, 0, sizeof(mW));
-        mU = mQ = mK = mA = mW;
+        mq = mk = mv = mU = mQ = mK = mA = mo = mW;
     }
     cudaError_t e;
     if (varlen) {
@@ -809,7 +980,7 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
             return e;
         dim3 grid((unsigned)L.n_slots, (unsigned)H);
         ProfToken tk = prof_begin(GDR_K_TC_WY, st);
-        kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, g, beta, cu, geo, ws, err);
+        kern<<<grid, kWyThreads, smem, st>>>(mq, mk, mv, mg, mU, mW, mA, g, beta, cu, geo, ws, err);
         prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -819,8 +990,8 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
                                       (int)smem)) != cudaSuccess)
             return e;
         ProfToken tk = prof_begin(GDR_K_TC_STATE, st);
-        state_kernel<<<(unsigned)(geo.n_seq * H), kThreads, smem, st>>>(
-            mW, mU, mQ, mK, mA, S0, (__nv_bfloat16 *)out, S_final, cu, geo, ws, err);
+        state_kernel<<<(unsigned)(geo.n_seq * H), kStThreads, smem, st>>>(
+            mW, mU, mQ, mK, mA, mo, S0, (__nv_bfloat16 *)out, S_final, cu, geo, ws, err);
         prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
