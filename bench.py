@@ -150,6 +150,14 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def aggregate(tokens_per_rank, ms_per_step, world):
+    """Whole-job throughput of a weak-scaling run: every rank processed
+    tokens_per_rank tokens per step; the job's step time is the slowest rank's.
+    Returns (tokens/s over all ranks, max ms per step)."""
+    ms = max_over_ranks(ms_per_step, world)
+    return tokens_per_rank * world / (ms * 1e-3), ms
+
+
 # ----------------------------------------------------------------- prefill
 class PrefillRun:
     def __init__(self, cfg, device, seed, path):
@@ -404,9 +412,8 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
     binding.profile_enable(False)
     prof = binding.profile_read()
     assert binding.device_status() == binding.GDR_OK
-    ms = max_over_ranks(sum(times) / len(times), world)
+    value, ms = aggregate(run.tokens(), sum(times) / len(times), world)
     tokens_all = run.tokens() * world
-    value = tokens_all / (ms * 1e-3)
     kernels = {k: {"launches": n, "avg_ms": (t / n if n else 0.0)} for k, (n, t) in prof.items()
                if n}
     launches = sum(n for n, _ in prof.values())
