@@ -145,6 +145,34 @@ gdr_status gdr_device_status(void *stream);
 gdr_status gdr_selftest_wait_timeout(unsigned int spin_limit, void *stream);
 
 /*
+ * gdr_fwd_noalloc -- the prefill for callers that cannot allocate device
+ * memory at call time (their memory manager owns the whole device heap and
+ * forbids further cudaMalloc, or an allocation's device synchronisation is not
+ * acceptable) and cannot pass a workspace of their own either.  The pages
+ * have no counterpart of this entry point; it exists only for such callers.
+ *
+ * Same arguments and results as gdr_fwd with path GDR_PATH_TENSORCORE, minus
+ * the workspace: the scratch comes from one fixed device array inside the
+ * library, gdr_fwd_noalloc_scratch_bytes() bytes (32 MiB) large, which every
+ * device that loads the library keeps until the process exits.  Calls whose
+ * scratch need (gdr_fwd_workspace_size with GDR_PATH_TENSORCORE) exceeds it,
+ * or whose shapes the tensor-core path does not take, return
+ * GDR_ERR_UNSUPPORTED; nothing is allocated, ever.
+ *
+ * The first call on a device looks up the array's device address (a CUDA
+ * runtime query, no allocation); make that first call outside any stream
+ * capture.  All calls on a device share the one array and nothing in it needs
+ * to start at zero, but two calls whose work overlaps on the GPU (different
+ * streams, no ordering between them) race on it: order them.
+ */
+gdr_status gdr_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const float *S0, void *out, float *S_final, int B,
+                           int T, int H, int d_k, int d_v, int chunk, const int32_t *cu_seqlens,
+                           int n_seq, gdr_dtype dtype, gdr_gate gate, void *stream);
+/* Size in bytes of the fixed scratch array used by gdr_fwd_noalloc. */
+size_t gdr_fwd_noalloc_scratch_bytes(void);
+
+/*
  * Per-kernel launch accounting and timing (a small built-in profiler).
  * Kernel ids: GDR_K_DECODE, GDR_K_FWD_SIMT, GDR_K_TC_PLAN, GDR_K_TC_WY,
  * GDR_K_TC_STATE.  Launches are always counted.  While timing is enabled,
