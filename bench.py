@@ -35,6 +35,29 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 SM_COUNT = 148
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture (summaries under profiles/), valid only for the kernel source
+# it was taken on: keyed by the first 16 hex digits of that file's sha256.
+NCU_TRAFFIC = {
+    "tc_wy": ("csrc/fwd_tc.cu", "738ff82dc9443843", 206.187264e6 + 253.290496e6),
+    "tc_state": ("csrc/fwd_tc.cu", "738ff82dc9443843", 308.476928e6 + 56.973312e6),
+    "decode": ("csrc/decode.cu", "8ab7b74f4e29cd3d", 543.248896e6 + 482.370048e6),
+}
+
+
+def ncu_traffic(kernel, workload):
+    """Measured traffic of `kernel` if its source is unchanged since the capture
+    (captures were taken on the gdn_prefill and decode workloads only)."""
+    import hashlib
+    ent = NCU_TRAFFIC.get(kernel)
+    if ent is None or workload not in ("gdn_prefill", "decode"):
+        return None
+    path = os.path.join(ROOT, "gated_delta_rule_90_b200", ent[0])
+    try:
+        digest = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return ent[2] if digest == ent[1] else None
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -425,7 +448,7 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
         B_ = decode_bytes(cfg)
         ach = B_ / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": ncu_traffic(dom, name),
                 "peak_source": peak_kind + " hbm_gbs", "algorithmic_bytes_per_launch": B_,
                 "frac_of_8TBps_spec": ach / 8000.0}
         conf["l2"] = "no flush: the 512 MiB state is larger than L2 and is streamed every step"
@@ -446,7 +469,7 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
             peak = peaks["bf16_tflops"]
             ach = flops / (dom_ms * 1e-3) / 1e12
             roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak,
-                    "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                    "unit": "TFLOP/s", "frac": ach / peak, "traffic": ncu_traffic(dom, name),
                     "peak_source": peak_kind + " bf16_tflops (burst)",
                     "algorithmic_flops_per_launch": flops}
         min_bytes = prefill_min_bytes(cfg, run.n_seq)
