@@ -181,9 +181,10 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     uint8_t *sm = align1024(smem_raw);
     uint8_t *sKQ = sm + WySmem::KQ, *sV = sm + WySmem::V, *sKL = sm + WySmem::KL;
     uint8_t *sT = sm + WySmem::TT, *sKH = sm + WySmem::KH, *sKC = sm + WySmem::KC;
-    float *sN = reinterpret_cast<float *>(sm + WySmem::end_tc(CH));   // [64][NST]
-    float *sX = sN + 64 * NST;                                          // [64][NST]
-    float *sG = sX + 64 * NST;                                          // CH ? [64][128] : [64]
+    float *sN = reinterpret_cast<float *>(sm + WySmem::end_tc(CH));   // N^T: [m][l], stride NST
+    float *sX = sN + 64 * NST;                                          // X: [row][col], stride NST
+    float *sXd = sX + 64 * NST;                                         // X_bb^T: [b][m][r] (4 x 16 x 16)
+    float *sG = sXd + 4 * 256;                                          // CH ? [64][128] : [64]
     float *sB = sG + (CH ? 64 * D : 64);                                // beta [64]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 64);            // [2]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
@@ -323,12 +324,13 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         const uint8_t *Bb = CH ? sKC : sKQ;
         const uint32_t bstride = CH ? 8192 : 16384;
         const uint32_t id = idesc_bf16(128, 64, 0, 0);
+        const uint64_t ad = sdesc_sw128(smem_u32(Ab), 16, 1024);
+        const uint64_t bd = sdesc_sw128(smem_u32(Bb), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint32_t koff = (kk & 3) * 32;
-            const uint64_t ad = sdesc_sw128(smem_u32(Ab + (kk >> 2) * 16384 + koff), 16, 1024);
-            const uint64_t bd = sdesc_sw128(smem_u32(Bb + (kk >> 2) * bstride + koff), 16, 1024);
-            mma_bf16_ss(tmem, ad, bd, id, kk > 0);
+            mma_bf16_ss(tmem, sdesc_add(ad, (kk >> 2) * 16384 + koff),
+                        sdesc_add(bd, (kk >> 2) * bstride + koff), id, kk > 0);
         }
         mma_commit(&bars[1]);
     }
@@ -352,7 +354,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             for (int i = 0; i < 32; ++i) {
                 const int m = m0 + i;
                 const float w = CH ? 1.f : __expf(Gl - sG[m]);
-                sN[l * NST + m] = (m < l) ? bl * gr[i] * w : 0.f;
+                sN[m * NST + l] = (m < l) ? bl * gr[i] * w : 0.f;  // stored transposed
             }
         } else {
 #pragma unroll
@@ -380,81 +382,113 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     // thread), then X_ij = -X_ii sum_{k=j}^{i-1} N_ik X_kj, one block
     // diagonal at a time (all fp32 in shared memory).
     {
+        // diagonal blocks: one column of X_bb = (I + N_bb)^{-1} per thread, kept
+        // row-major in X and transposed in Xd (for 4-row float4 reads)
         if (tid < C) {
             const int b = tid >> 4, j = tid & 15;
-            const float *Nb = sN + (16 * b) * NST + 16 * b;
             float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-                for (int m = 0; m < i; ++m) {
-                    if (m & 1) p1 = fmaf(Nb[i * NST + m], x[m], p1);
-                    else p0 = fmaf(Nb[i * NST + m], x[m], p0);
+                for (int m = 0; m < i; ++m) {  // N_bb[i][m] = N^T[16b+m][16b+i]
+                    const float nv = sN[(16 * b + m) * NST + 16 * b + i];
+                    if (m & 1) p1 = fmaf(nv, x[m], p1);
+                    else p0 = fmaf(nv, x[m], p0);
                 }
                 x[i] = ((i == j) ? 1.f : 0.f) - (p0 + p1);
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) sX[(16 * b + i) * NST + 16 * b + j] = x[i];
+            float4 *xd = reinterpret_cast<float4 *>(sXd + b * 256 + j * 16);  // X_bb^T[m = j][r]
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4)
+                xd[i4] = make_float4(x[4 * i4], x[4 * i4 + 1], x[4 * i4 + 2], x[4 * i4 + 3]);
         }
         __syncthreads();
-#pragma unroll 1
-        for (int dd = 1; dd < 4; ++dd) {
-            const int nout = (4 - dd) * 256;
-            // P_ij = sum_k N_ik X_kj, written into block (i, j) of X (not read in this pass)
+        // Thread tasks below are strips of 4 rows x 1 column of a 16 x 16 block
+        // (float4 reads of N^T and Xd give the 4 rows at once).
+        const int c = tid & 15, r0 = ((tid >> 4) & 3) * 4, blk = tid >> 6;
+        // level A: the two 32 x 32 diagonal blocks, X_10 and X_32:
+        //   X_i,i-1 = -X_ii (N_i,i-1 X_i-1,i-1)
+        {
+            const int j = blk * 2, i = j + 1;  // blk 0: (1,0), blk 1: (3,2)
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (tid < 128) {
 #pragma unroll
-            for (int kq = 0; kq < 3; ++kq) {
-                const int e = tid + kq * kWyThreads;
-                if (e < nout) {
-                    const int j = e >> 8, i = j + dd, r = (e >> 4) & 15, c = e & 15;
-                    float p0 = 0.f, p1 = 0.f;
-                    for (int kb = j; kb < i; ++kb) {
-                        const float4 *nr = reinterpret_cast<const float4 *>(sN + (16 * i + r) * NST + 16 * kb);
-                        const float *xc = sX + (16 * kb) * NST + 16 * j + c;
+                for (int m = 0; m < 16; ++m) {
+                    const float xv = sX[(16 * j + m) * NST + 16 * j + c];
+                    const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * j + m) * NST + 16 * i + r0);
+                    acc[0] = fmaf(nv.x, xv, acc[0]);
+                    acc[1] = fmaf(nv.y, xv, acc[1]);
+                    acc[2] = fmaf(nv.z, xv, acc[2]);
+                    acc[3] = fmaf(nv.w, xv, acc[3]);
+                }
 #pragma unroll
-                        for (int m4 = 0; m4 < 4; ++m4) {
-                            const float4 nv = nr[m4];
-                            p0 = fmaf(nv.x, xc[(4 * m4 + 0) * NST], p0);
-                            p1 = fmaf(nv.y, xc[(4 * m4 + 1) * NST], p1);
-                            p0 = fmaf(nv.z, xc[(4 * m4 + 2) * NST], p0);
-                            p1 = fmaf(nv.w, xc[(4 * m4 + 3) * NST], p1);
-                        }
-                    }
-                    sX[(16 * i + r) * NST + 16 * j + c] = p0 + p1;
+                for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * NST + 16 * j + c] = acc[t];
+            }
+            __syncthreads();
+            float res[4] = {0.f, 0.f, 0.f, 0.f};
+            if (tid < 128) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float pv = sX[(16 * i + m) * NST + 16 * j + c];
+                    const float4 xv = *reinterpret_cast<const float4 *>(sXd + i * 256 + m * 16 + r0);
+                    res[0] = fmaf(xv.x, pv, res[0]);
+                    res[1] = fmaf(xv.y, pv, res[1]);
+                    res[2] = fmaf(xv.z, pv, res[2]);
+                    res[3] = fmaf(xv.w, pv, res[3]);
                 }
             }
             __syncthreads();
-            float res[3];
+            if (tid < 128) {
 #pragma unroll
-            for (int kq = 0; kq < 3; ++kq) {
-                const int e = tid + kq * kWyThreads;
-                res[kq] = 0.f;
-                if (e < nout) {
-                    const int j = e >> 8, i = j + dd, r = (e >> 4) & 15, c = e & 15;
-                    const float4 *xr = reinterpret_cast<const float4 *>(sX + (16 * i + r) * NST + 16 * i);
-                    const float *pc = sX + (16 * i) * NST + 16 * j + c;
-                    float acc = 0.f;
+                for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * NST + 16 * j + c] = -res[t];
+            }
+            __syncthreads();
+        }
+        // level B: the lower-left 32 x 32 quadrant, blocks (i, j), i in {2,3}, j in {0,1}:
+        //   P_ij = N_i0 X_0j + N_i1 X_1j,  X_2j = -X_22 P_2j,  X_3j = -(X_32 P_2j + X_33 P_3j)
+        {
+            const int i = 2 + (blk >> 1), j = blk & 1;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int kb = j; kb < 2; ++kb) {
 #pragma unroll
-                    for (int m4 = 0; m4 < 4; ++m4) {
-                        const float4 xv = xr[m4];  // X_ii is lower triangular: zeros above
-                        acc = fmaf(xv.x, pc[(4 * m4 + 0) * NST], acc);
-                        acc = fmaf(xv.y, pc[(4 * m4 + 1) * NST], acc);
-                        acc = fmaf(xv.z, pc[(4 * m4 + 2) * NST], acc);
-                        acc = fmaf(xv.w, pc[(4 * m4 + 3) * NST], acc);
-                    }
-                    res[kq] = -acc;
+                for (int m = 0; m < 16; ++m) {
+                    const float xv = sX[(16 * kb + m) * NST + 16 * j + c];
+                    const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * kb + m) * NST + 16 * i + r0);
+                    acc[0] = fmaf(nv.x, xv, acc[0]);
+                    acc[1] = fmaf(nv.y, xv, acc[1]);
+                    acc[2] = fmaf(nv.z, xv, acc[2]);
+                    acc[3] = fmaf(nv.w, xv, acc[3]);
                 }
             }
-            if (dd == 3 && tid == 0) bulk_wait_group_read<0>();  // the A staging is read
+#pragma unroll
+            for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * NST + 16 * j + c] = acc[t];
+            __syncthreads();
+            float res[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {  // X_ii P_ij
+                const float pv = sX[(16 * i + m) * NST + 16 * j + c];
+                const float4 xv = *reinterpret_cast<const float4 *>(sXd + i * 256 + m * 16 + r0);
+                res[0] = fmaf(xv.x, pv, res[0]);
+                res[1] = fmaf(xv.y, pv, res[1]);
+                res[2] = fmaf(xv.z, pv, res[2]);
+                res[3] = fmaf(xv.w, pv, res[3]);
+            }
+            if (i == 3) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {  // + X_32 P_2j
+                    const float pv = sX[(32 + m) * NST + 16 * j + c];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        res[t] = fmaf(sX[(48 + r0 + t) * NST + 32 + m], pv, res[t]);
+                }
+            }
+            if (tid == 0) bulk_wait_group_read<0>();  // the A staging is read
             __syncthreads();
 #pragma unroll
-            for (int kq = 0; kq < 3; ++kq) {
-                const int e = tid + kq * kWyThreads;
-                if (e < nout) {
-                    const int j = e >> 8, i = j + dd, r = (e >> 4) & 15, c = e & 15;
-                    sX[(16 * i + r) * NST + 16 * j + c] = res[kq];
-                }
-            }
+            for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * NST + 16 * j + c] = -res[t];
             __syncthreads();
         }
         // T[i][j] = X[i][j] beta_j (lower triangle) -> bf16, K-major SW128 tile
@@ -476,13 +510,13 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     if (tid == 0) {
         tc_fence_after();
         const uint32_t id = idesc_bf16(128, 64, 1, 0);
+        const uint64_t bd = sdesc_sw128(smem_u32(sT), 16, 1024);
+        const uint64_t av = sdesc_sw128(smem_u32(sV), 8192, 1024);
+        const uint64_t ak = sdesc_sw128(smem_u32(sKL), 8192, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = sdesc_sw128(smem_u32(sT + kk * 32), 16, 1024);
-            const uint64_t av = sdesc_sw128(smem_u32(sV + kk * 2048), 8192, 1024);
-            const uint64_t ak = sdesc_sw128(smem_u32(sKL + kk * 2048), 8192, 1024);
-            mma_bf16_ss(tmem + 64, av, bd, id, kk > 0);
-            mma_bf16_ss(tmem + 128, ak, bd, id, kk > 0);
+            mma_bf16_ss(tmem + 64, sdesc_add(av, kk * 2048), sdesc_add(bd, kk * 32), id, kk > 0);
+            mma_bf16_ss(tmem + 128, sdesc_add(ak, kk * 2048), sdesc_add(bd, kk * 32), id, kk > 0);
         }
         mma_commit(&bars[1]);
     }
@@ -547,7 +581,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         bulk_commit_group();
     }
 cleanup:
-    if (tid == 0) bulk_wait_group<0>();
+    if (tid == 0) bulk_wait_group_read<0>();  // shared memory must outlive the stores' reads
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
@@ -664,15 +698,17 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     *reinterpret_cast<uint4 *>(rowp + ((j ^ (d & 7)) << 4)) = pack8(v + j * 8);
+                // the Z and O MMAs need only the bf16 copy: release it first
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(opsS);
+                // S <- S Diag(decay), needed by the S-update MMA (after opsZ)
 #pragma unroll
                 for (int i = 0; i < 64; ++i) v[i] *= dec[i];
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) tmem_st16(tS + lb + hf * 64 + cb * 16, v + cb * 16);
                 tmem_wait_st();
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(opsS);
             ok = mbar_wait_bounded(barZ, r & 1, kSpin, err);
             if (!ok) break;
             tc_fence_after();
@@ -748,7 +784,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
                     if (i < len) og[(size_t)i * geo.H * D] = __float2bfloat16_rn(o[i]);
             }
         }
-        if (otid == 0) bulk_wait_group<0>();
+        if (otid == 0) bulk_wait_group_read<0>();
     } else if (lane == 0) {
         // ===================== producer: TMA + MMA =====================
         auto issue = [&](int r) {
@@ -778,47 +814,43 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
         const uint32_t idZ = idesc_bf16(128, 64, 0, 1);
         const uint32_t idO = idesc_bf16(128, 64, 0, 0);
         const uint32_t idS = idesc_bf16(128, 128, 0, 1);
+        // operand descriptors, built once; k-steps only advance the start address
+        const uint64_t dS = sdesc_sw128(smem_u32(sm + StSmem::S), 16, 1024);
+        const uint64_t dZT = sdesc_sw128(smem_u32(sm + StSmem::ZT), 16, 1024);
+        const uint64_t dW0 = sdesc_sw128(smem_u32(sm + StSmem::WT), 16384, 1024);
+        const uint64_t dQ0 = sdesc_sw128(smem_u32(sm + StSmem::Q), 16, 1024);
+        const uint64_t dK0 = sdesc_sw128(smem_u32(sm + StSmem::K), 8192, 1024);
+        const uint64_t dA0 = sdesc_sw128(smem_u32(sm + StSmem::A), 16, 1024);
+        const uint32_t stage16 = StSmem::STAGE >> 4;  // stage stride in descriptor units
         for (int r = 0; r < nch && ok; ++r) {
-            const uint8_t *st = sm + (r & 1) * StSmem::STAGE;
             const uint32_t tO = tO0 + (r & 1) * 64;
+            const uint64_t so = (r & 1) ? stage16 : 0;
+            const uint64_t dw = dW0 + so, dq = dQ0 + so, dk = dK0 + so, da = dA0 + so;
             ok = mbar_wait_bounded(opsS, r & 1, kSpin, err);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {  // Z^T = S W<-^T
-                const uint64_t a =
-                    sdesc_sw128(smem_u32(sm + StSmem::S + (kk >> 2) * 16384 + (kk & 3) * 32), 16, 1024);
-                const uint64_t bw = sdesc_sw128(smem_u32(st + StSmem::WT + kk * 2048), 16384, 1024);
-                mma_bf16_ss(tZ, a, bw, idZ, kk > 0);
-            }
+            for (int kk = 0; kk < 8; ++kk)  // Z^T = S W<-^T
+                mma_bf16_ss(tZ, sdesc_add(dS, (kk >> 2) * 16384 + (kk & 3) * 32),
+                            sdesc_add(dw, kk * 2048), idZ, kk > 0);
             mma_commit(barZ);
             if (r >= 2) ok = mbar_wait_bounded(&oFree[r & 1], ((r - 2) >> 1) & 1, kSpin, err);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {  // O^T = S Q<-^T
-                const uint64_t a =
-                    sdesc_sw128(smem_u32(sm + StSmem::S + (kk >> 2) * 16384 + (kk & 3) * 32), 16, 1024);
-                const uint64_t bq =
-                    sdesc_sw128(smem_u32(st + StSmem::Q + (kk >> 2) * 8192 + (kk & 3) * 32), 16, 1024);
-                mma_bf16_ss(tO, a, bq, idO, kk > 0);
-            }
+            for (int kk = 0; kk < 8; ++kk)  // O^T = S Q<-^T
+                mma_bf16_ss(tO, sdesc_add(dS, (kk >> 2) * 16384 + (kk & 3) * 32),
+                            sdesc_add(dq, (kk >> 2) * 8192 + (kk & 3) * 32), idO, kk > 0);
             ok = mbar_wait_bounded(opsZ, r & 1, kSpin, err);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {  // S += Z^T K->
-                const uint64_t a = sdesc_sw128(smem_u32(sm + StSmem::ZT + kk * 32), 16, 1024);
-                const uint64_t bk = sdesc_sw128(smem_u32(st + StSmem::K + kk * 2048), 8192, 1024);
-                mma_bf16_ss(tS, a, bk, idS, 1);
-            }
+            for (int kk = 0; kk < 4; ++kk)  // S += Z^T K->
+                mma_bf16_ss(tS, sdesc_add(dZT, kk * 32), sdesc_add(dk, kk * 2048), idS, 1);
             mma_commit(barS);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {  // O^T += Z^T A^T
-                const uint64_t a = sdesc_sw128(smem_u32(sm + StSmem::ZT + kk * 32), 16, 1024);
-                const uint64_t ba = sdesc_sw128(smem_u32(st + StSmem::A + kk * 32), 16, 1024);
-                mma_bf16_ss(tO, a, ba, idO, 1);
-            }
+            for (int kk = 0; kk < 4; ++kk)  // O^T += Z^T A^T
+                mma_bf16_ss(tO, sdesc_add(dZT, kk * 32), sdesc_add(da, kk * 32), idO, 1);
             mma_commit(&barO[r & 1]);
             // this stage is free once chunk r's MMAs are done: prefetch chunk r+2
             if (r + 2 < nch) {
@@ -903,7 +935,7 @@ constexpr CUtensorMapSwizzle kSW = CU_TENSOR_MAP_SWIZZLE_128B;
 constexpr CUtensorMapSwizzle kNoSW = CU_TENSOR_MAP_SWIZZLE_NONE;
 
 size_t wy_smem_bytes(bool ch) {  // + 1024 for the in-kernel alignment
-    return 1024 + WySmem::end_tc(ch) + 4 * (2 * 64 * WySmem::NST + (ch ? 64 * D : 64) + 64) + 64;
+    return 1024 + WySmem::end_tc(ch) + 4 * (2 * 64 * WySmem::NST + 1024 + (ch ? 64 * D : 64) + 64) + 64;
 }
 
 }  // namespace
