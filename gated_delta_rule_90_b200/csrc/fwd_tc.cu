@@ -49,7 +49,6 @@ using namespace sm100;
 constexpr int C = 64;
 constexpr int D = 128;
 constexpr uint32_t kSpin = 1u << 24;  // poll limit of every mbarrier wait
-constexpr uint32_t kTmemCols = 256;
 
 constexpr uint32_t kTileBytes = C * D * 2;   // 16 KB: one [64][128] bf16 tile
 constexpr uint32_t kHalfBytes = C * 64 * 2;  // 8 KB: one [64][64] bf16 atom column
@@ -153,19 +152,30 @@ __global__ void plan_kernel(const int32_t *cu, int n_seq, int T_total, int *chun
 }
 
 // ------------------------------------------------------------------ WY kernel
-// 256 threads.  For accumulator epilogues, warp w serves TMEM lane quadrant
-// (w & 3) and column half (w >> 2).
+// 256 threads, 128 TMEM columns.  For accumulator epilogues, warp w serves TMEM
+// lane quadrant (w & 3) and column half (w >> 2).
 constexpr int kWyThreads = 256;
+constexpr uint32_t kWyTmemCols = 128;
 
+// Shared-memory plan (byte offsets from a 1024-aligned base).  Regions are
+// reused once their first contents are dead, so a scalar-gate CTA needs
+// 74 KB and three fit on an SM:
+//   KQ  [0, 32K)     raw K (rows 0-63) and Q (rows 64-127) in two 128-byte atom
+//                    columns.  Scalar gate: V replaces Q once Q is read; per-channel
+//                    gate: K^ and Q^ in place.  At the end: U^T / W^T staging.
+//   TT  [32K, 40K)   A staging for its TMA store, then T.
+//   NT  [40K, 56K)   N^T fp32 [64][64]; after the solve, K<- (bf16, 2 atoms).
+//                    Per-channel gate: NT and XR first hold the gate tile G.
+//   XR  [56K, 72.3K) X fp32 [64][65].
+//   per-channel gate only: V [73K, 89K) and K-check [89K, 105K).
 struct WySmem {
-    static constexpr uint32_t KQ = 0;                    // [K;Q] raw, 2 atoms x 128 rows; later U^T|W^T staging
-    static constexpr uint32_t V = KQ + 2 * 16384;        // 2 atoms x 64 rows
-    static constexpr uint32_t KL = V + 2 * 8192;         // K<- (MMA A operand, MN-major)
-    static constexpr uint32_t TT = KL + 2 * 8192;        // T (K-major B operand); A staging before
-    static constexpr uint32_t KH = TT + 8192;            // KDA: [K^;Q^] scaled Gram A
-    static constexpr uint32_t KC = KH + 2 * 16384;       // KDA: K-check, Gram B
-    static constexpr uint32_t end_tc(bool ch) { return ch ? KC + 2 * 8192 : KH; }
-    static constexpr int NST = 68;                       // fp32 row stride of N and X
+    static constexpr uint32_t KQ = 0, TT = 32768, NT = 40960, XR = 57344;
+    static constexpr int NTS = 64;                                   // N^T row stride (floats)
+    static constexpr int XST = 65;                                   // X row stride (floats)
+    static constexpr uint32_t XEND = XR + 64 * XST * 4;
+    static constexpr uint32_t VCH = 74752, KC = VCH + 16384;
+    static constexpr uint32_t small(bool ch) { return ch ? KC + 16384 : XEND; }
+    static constexpr uint32_t small_bytes(bool ch) { return (ch ? (2 * D + 64) : 128) * 4 + 64; }
 };
 
 template <bool CH>
@@ -176,16 +186,20 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           const __grid_constant__ CUtensorMap tm_Ast, const float *__restrict__ g,
           const float *__restrict__ beta, const int32_t *__restrict__ cu, Geo geo, Ws ws,
           unsigned int *err) {
-    constexpr int NST = WySmem::NST;
+    constexpr int NTS = WySmem::NTS, XST = WySmem::XST;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    uint8_t *sKQ = sm + WySmem::KQ, *sV = sm + WySmem::V, *sKL = sm + WySmem::KL;
-    uint8_t *sT = sm + WySmem::TT, *sKH = sm + WySmem::KH, *sKC = sm + WySmem::KC;
-    float *sN = reinterpret_cast<float *>(sm + WySmem::end_tc(CH));   // N^T: [m][l], stride NST
-    float *sX = sN + 64 * NST;                                          // X: [row][col], stride NST
-    float *sXd = sX + 64 * NST;                                         // X_bb^T: [b][m][r] (4 x 16 x 16)
-    float *sG = sXd + 4 * 256;                                          // CH ? [64][128] : [64]
-    float *sB = sG + (CH ? 64 * D : 64);                                // beta [64]
+    uint8_t *sKQ = sm + WySmem::KQ, *sT = sm + WySmem::TT;
+    uint8_t *sKL = sm + WySmem::NT;                                    // after the solve
+    uint8_t *sV = CH ? sm + WySmem::VCH : sKQ + 8192;                  // scalar gate: Q's place
+    uint8_t *sKC = sm + WySmem::KC;                                    // per-channel gate only
+    float *sN = reinterpret_cast<float *>(sm + WySmem::NT);            // N^T [m][l]
+    float *sX = reinterpret_cast<float *>(sm + WySmem::XR);            // X [row][col]
+    float *sGt = reinterpret_cast<float *>(sm + WySmem::NT);           // per-channel G [64][128]
+    float *sSm = reinterpret_cast<float *>(sm + WySmem::small(CH));
+    float *sG = sSm;                                                   // scalar: G [64]; channel: R row [128]
+    float *sGC = sSm + (CH ? D : 64);                                  // channel: G_C row [128]
+    float *sB = CH ? sGC + D : sSm + 64;                               // beta [64]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 64);            // [2]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
 
@@ -197,6 +211,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     int len;
     if (!locate_chunk(geo, cu, ws, gcid, tstart, len)) return;  // whole CTA, before any sync
     const size_t slot = (size_t)gcid * geo.H + h;
+    const int x0 = h * D, ytok = (int)tstart;
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
@@ -204,7 +219,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tslot, kTmemCols);
+        tmem_alloc(tslot, kWyTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -216,15 +231,16 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_arrive_expect_tx(&bars[0], 6 * kHalfBytes + (CH ? C * D * 4 : 0));
-        const int x0 = h * D, y = (int)tstart;
-        tma_load_2d(sKQ, &tm_k, &bars[0], x0, y);
-        tma_load_2d(sKQ + 16384, &tm_k, &bars[0], x0 + 64, y);
-        tma_load_2d(sKQ + 8192, &tm_q, &bars[0], x0, y);
-        tma_load_2d(sKQ + 16384 + 8192, &tm_q, &bars[0], x0 + 64, y);
-        tma_load_2d(sV, &tm_v, &bars[0], x0, y);
-        tma_load_2d(sV + 8192, &tm_v, &bars[0], x0 + 64, y);
-        if (CH) tma_load_2d(sG, &tm_g, &bars[0], x0, y);  // [64][128] fp32 per-channel gates
+        mbar_arrive_expect_tx(&bars[0], 4 * kHalfBytes + (CH ? 2 * kHalfBytes + C * D * 4 : 0));
+        tma_load_2d(sKQ, &tm_k, &bars[0], x0, ytok);
+        tma_load_2d(sKQ + 16384, &tm_k, &bars[0], x0 + 64, ytok);
+        tma_load_2d(sKQ + 8192, &tm_q, &bars[0], x0, ytok);
+        tma_load_2d(sKQ + 16384 + 8192, &tm_q, &bars[0], x0 + 64, ytok);
+        if (CH) {
+            tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
+            tma_load_2d(sV + 8192, &tm_v, &bars[0], x0 + 64, ytok);
+            tma_load_2d(sGt, &tm_g, &bars[0], x0, ytok);  // [64][128] fp32 per-channel gates
+        }
     }
     // gates and beta (zero beyond the sequence end), cumulative log-decay G
     if (!CH && tid < C) sG[tid] = (tid < len) ? g[(size_t)(tstart + tid) * geo.H + h] : 0.f;
@@ -255,63 +271,68 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         const int c = tid & 127, r0 = (tid >> 7) * 32;
         float acc = 0.f;
         for (int l = r0; l < r0 + 32; ++l) {
-            if (l < len) acc += sG[l * D + c];
-            sG[l * D + c] = acc;
+            if (l < len) acc += sGt[l * D + c];
+            sGt[l * D + c] = acc;
         }
         __syncthreads();
         if (r0) {
-            const float base = sG[31 * D + c];
-            for (int l = 32; l < 64; ++l) sG[l * D + c] += base;
+            const float base = sGt[31 * D + c];
+            for (int l = 32; l < 64; ++l) sGt[l * D + c] += base;
+        }
+        __syncthreads();
+        if (tid < D) {
+            sG[tid] = sGt[31 * D + tid];         // reference row R of the Gram factorisation
+            sGC[tid] = sGt[(C - 1) * D + tid];   // G_C
         }
     }
-    // zero the rows beyond the sequence end (whole 128-byte rows: swizzle-agnostic)
+    // zero K and Q rows beyond the sequence end (whole 128-byte rows)
     if (len < C) {
-        for (int e = tid; e < (C - len) * 8 * 6; e += kWyThreads) {
-            const int r = len + e / 48, part = e % 48, tile = part >> 3, ch16 = part & 7;
-            uint8_t *base = tile < 4 ? sKQ + (tile & 1) * 16384 + (tile >> 1) * 8192
-                                     : sV + (tile & 1) * 8192;
+        for (int e = tid; e < (C - len) * 8 * 4; e += kWyThreads) {
+            const int r = len + e / 32, part = e % 32, tile = part >> 3, ch16 = part & 7;
+            uint8_t *base = sKQ + (tile & 1) * 16384 + (tile >> 1) * 8192;
             *reinterpret_cast<uint4 *>(base + r * 128 + ch16 * 16) = make_uint4(0, 0, 0, 0);
         }
     }
     __syncthreads();
-    // decayed operands: K<- = e^G . k (all gates); KDA also the scaled Gram operands
-    for (int e = tid; e < C * 16; e += kWyThreads) {
-        const int l = e >> 4, a = (e >> 3) & 1, j = e & 7;
-        const int c0 = a * 64 + ((j ^ (l & 7)) << 3);
-        const uint32_t off = a * 16384 + l * 128 + j * 16;
-        float kv[8], w[8];
-        unpack8(*reinterpret_cast<const uint4 *>(sKQ + off), kv);
-        if (CH) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = __expf(sG[l * D + c0 + i]);
-        } else {
-            const float sc = __expf(sG[l]);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = sc;
-        }
-        float o[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = kv[i] * w[i];
-        *reinterpret_cast<uint4 *>(sKL + a * 8192 + l * 128 + j * 16) = pack8(o);
-        if (CH) {
-            float qv[8], e1[8], e2[8];
+    // From the raw K and Q: Q<- = e^G . q and K-> = e^(G_C - G) . k to the
+    // workspace; per-channel gate also K-check = k e^(R - G) and, in place,
+    // K^ = k e^(G - R), Q^ = q e^(G - R) (R = row 31 of G).
+    {
+        __nv_bfloat16 *Qg = ws.Q + slot * (C * D), *Kg = ws.K + slot * (C * D);
+        for (int e = tid; e < C * 16; e += kWyThreads) {
+            const int l = e >> 4, a = (e >> 3) & 1, j = e & 7;
+            const int c0 = a * 64 + ((j ^ (l & 7)) << 3);
+            const uint32_t off = a * 16384 + l * 128 + j * 16;
+            float kv[8], qv[8], wq[8], wk[8];
+            unpack8(*reinterpret_cast<const uint4 *>(sKQ + off), kv);
             unpack8(*reinterpret_cast<const uint4 *>(sKQ + off + 8192), qv);
+            if (CH) {
+                float kh[8], qh[8], kc[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float dlt = sG[l * D + c0 + i] - sG[31 * D + c0 + i];
-                e1[i] = __expf(dlt);
-                e2[i] = __expf(-dlt);
+                for (int i = 0; i < 8; ++i) {
+                    const float Gl = sGt[l * D + c0 + i], R = sG[c0 + i];
+                    wq[i] = qv[i] * __expf(Gl);
+                    wk[i] = kv[i] * __expf(sGC[c0 + i] - Gl);
+                    const float e1 = __expf(Gl - R), e2 = __expf(R - Gl);
+                    kh[i] = kv[i] * e1;
+                    qh[i] = qv[i] * e1;
+                    kc[i] = kv[i] * e2;
+                }
+                *reinterpret_cast<uint4 *>(sKQ + off) = pack8(kh);
+                *reinterpret_cast<uint4 *>(sKQ + off + 8192) = pack8(qh);
+                *reinterpret_cast<uint4 *>(sKC + a * 8192 + l * 128 + j * 16) = pack8(kc);
+            } else {
+                const float eq = __expf(sG[l]), ek = __expf(sG[C - 1] - sG[l]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    wq[i] = qv[i] * eq;
+                    wk[i] = kv[i] * ek;
+                }
             }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = kv[i] * e1[i];
-            *reinterpret_cast<uint4 *>(sKH + off) = pack8(o);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = qv[i] * e1[i];
-            *reinterpret_cast<uint4 *>(sKH + off + 8192) = pack8(o);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = kv[i] * e2[i];
-            *reinterpret_cast<uint4 *>(sKC + a * 8192 + l * 128 + j * 16) = pack8(o);
+            *reinterpret_cast<uint4 *>(Qg + l * D + c0) = pack8(wq);
+            *reinterpret_cast<uint4 *>(Kg + l * D + c0) = pack8(wk);
         }
+        if (tid < D) ws.dec[slot * D + tid] = __expf(CH ? sGC[tid] : sG[C - 1]);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -320,11 +341,10 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     // Gram: TMEM[0:64) = [K;Q] (128 x 128) * Kc^T (64 x 128)^T
     if (tid == 0) {
         tc_fence_after();
-        const uint8_t *Ab = CH ? sKH : sKQ;
         const uint8_t *Bb = CH ? sKC : sKQ;
         const uint32_t bstride = CH ? 8192 : 16384;
         const uint32_t id = idesc_bf16(128, 64, 0, 0);
-        const uint64_t ad = sdesc_sw128(smem_u32(Ab), 16, 1024);
+        const uint64_t ad = sdesc_sw128(smem_u32(sKQ), 16, 1024);
         const uint64_t bd = sdesc_sw128(smem_u32(Bb), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -339,9 +359,14 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         if (!__syncthreads_and(ok)) goto cleanup;
     }
     tc_fence_after();
+    if (!CH && tid == 0) {  // Q is read: V takes its place (lands during the solve)
+        mbar_arrive_expect_tx(&bars[0], 2 * kHalfBytes);
+        tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
+        tma_load_2d(sV + 16384, &tm_v, &bars[0], x0 + 64, ytok);
+    }
     {
-        // accumulator rows 0..63: K K^T -> N = diag(beta) tril_-1(. Gamma);
-        // rows 64..127: Q K^T -> A = tril_0(. Gamma), bf16, staged in the T tile
+        // accumulator rows 0..63: K K^T -> N = diag(beta) tril_-1(. Gamma), stored
+        // transposed; rows 64..127: Q K^T -> A = tril_0(. Gamma), bf16, staged in TT
         const int l = (qd & 1) * 32 + lane, m0 = hf * 32;
         float gr[32];
         tmem_ld16(tmem + lb + m0, gr);
@@ -354,7 +379,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             for (int i = 0; i < 32; ++i) {
                 const int m = m0 + i;
                 const float w = CH ? 1.f : __expf(Gl - sG[m]);
-                sN[m * NST + l] = (m < l) ? bl * gr[i] * w : 0.f;  // stored transposed
+                sN[m * NTS + l] = (m < l) ? bl * gr[i] * w : 0.f;
             }
         } else {
 #pragma unroll
@@ -372,6 +397,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         }
     }
     fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
     if (tid == 0) {  // A -> workspace
         tma_store_2d(&tm_Ast, sT, 0, (int)(slot * C));
@@ -379,11 +405,8 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     }
     // T = (I + N)^{-1} diag(beta), N = diag(beta) L strictly lower, by 16 x 16
     // blocks: X_ii = (I + N_ii)^{-1} by forward substitution (one column per
-    // thread), then X_ij = -X_ii sum_{k=j}^{i-1} N_ik X_kj, one block
-    // diagonal at a time (all fp32 in shared memory).
+    // thread); then X_10, X_32 and finally the lower-left 32 x 32 quadrant.
     {
-        // diagonal blocks: one column of X_bb = (I + N_bb)^{-1} per thread, kept
-        // row-major in X and transposed in Xd (for 4-row float4 reads)
         if (tid < C) {
             const int b = tid >> 4, j = tid & 15;
             float x[16];
@@ -392,71 +415,61 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 float p0 = 0.f, p1 = 0.f;
 #pragma unroll
                 for (int m = 0; m < i; ++m) {  // N_bb[i][m] = N^T[16b+m][16b+i]
-                    const float nv = sN[(16 * b + m) * NST + 16 * b + i];
+                    const float nv = sN[(16 * b + m) * NTS + 16 * b + i];
                     if (m & 1) p1 = fmaf(nv, x[m], p1);
                     else p0 = fmaf(nv, x[m], p0);
                 }
                 x[i] = ((i == j) ? 1.f : 0.f) - (p0 + p1);
             }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sX[(16 * b + i) * NST + 16 * b + j] = x[i];
-            float4 *xd = reinterpret_cast<float4 *>(sXd + b * 256 + j * 16);  // X_bb^T[m = j][r]
-#pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4)
-                xd[i4] = make_float4(x[4 * i4], x[4 * i4 + 1], x[4 * i4 + 2], x[4 * i4 + 3]);
+            for (int i = 0; i < 16; ++i) sX[(16 * b + i) * XST + 16 * b + j] = x[i];
         }
         __syncthreads();
-        // Thread tasks below are strips of 4 rows x 1 column of a 16 x 16 block
-        // (float4 reads of N^T and Xd give the 4 rows at once).
+        // tasks: strips of 4 rows x 1 column of a 16 x 16 block (float4 over N^T rows)
         const int c = tid & 15, r0 = ((tid >> 4) & 3) * 4, blk = tid >> 6;
-        // level A: the two 32 x 32 diagonal blocks, X_10 and X_32:
-        //   X_i,i-1 = -X_ii (N_i,i-1 X_i-1,i-1)
-        {
-            const int j = blk * 2, i = j + 1;  // blk 0: (1,0), blk 1: (3,2)
+        {   // level A: X_10 = -X_11 (N_10 X_00), X_32 = -X_33 (N_32 X_22)
+            const int j = blk * 2, i = j + 1;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             if (tid < 128) {
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
-                    const float xv = sX[(16 * j + m) * NST + 16 * j + c];
-                    const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * j + m) * NST + 16 * i + r0);
+                    const float xv = sX[(16 * j + m) * XST + 16 * j + c];
+                    const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * j + m) * NTS + 16 * i + r0);
                     acc[0] = fmaf(nv.x, xv, acc[0]);
                     acc[1] = fmaf(nv.y, xv, acc[1]);
                     acc[2] = fmaf(nv.z, xv, acc[2]);
                     acc[3] = fmaf(nv.w, xv, acc[3]);
                 }
 #pragma unroll
-                for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * NST + 16 * j + c] = acc[t];
+                for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = acc[t];
             }
             __syncthreads();
             float res[4] = {0.f, 0.f, 0.f, 0.f};
             if (tid < 128) {
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
-                    const float pv = sX[(16 * i + m) * NST + 16 * j + c];
-                    const float4 xv = *reinterpret_cast<const float4 *>(sXd + i * 256 + m * 16 + r0);
-                    res[0] = fmaf(xv.x, pv, res[0]);
-                    res[1] = fmaf(xv.y, pv, res[1]);
-                    res[2] = fmaf(xv.z, pv, res[2]);
-                    res[3] = fmaf(xv.w, pv, res[3]);
+                    const float pv = sX[(16 * i + m) * XST + 16 * j + c];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        res[t] = fmaf(sX[(16 * i + r0 + t) * XST + 16 * i + m], pv, res[t]);
                 }
             }
             __syncthreads();
             if (tid < 128) {
 #pragma unroll
-                for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * NST + 16 * j + c] = -res[t];
+                for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = -res[t];
             }
             __syncthreads();
         }
-        // level B: the lower-left 32 x 32 quadrant, blocks (i, j), i in {2,3}, j in {0,1}:
-        //   P_ij = N_i0 X_0j + N_i1 X_1j,  X_2j = -X_22 P_2j,  X_3j = -(X_32 P_2j + X_33 P_3j)
-        {
+        {   // level B: P_ij = N_i0 X_0j + N_i1 X_1j (i in {2,3}, j in {0,1});
+            // X_2j = -X_22 P_2j,  X_3j = -(X_32 P_2j + X_33 P_3j)
             const int i = 2 + (blk >> 1), j = blk & 1;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             for (int kb = j; kb < 2; ++kb) {
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
-                    const float xv = sX[(16 * kb + m) * NST + 16 * j + c];
-                    const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * kb + m) * NST + 16 * i + r0);
+                    const float xv = sX[(16 * kb + m) * XST + 16 * j + c];
+                    const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * kb + m) * NTS + 16 * i + r0);
                     acc[0] = fmaf(nv.x, xv, acc[0]);
                     acc[1] = fmaf(nv.y, xv, acc[1]);
                     acc[2] = fmaf(nv.z, xv, acc[2]);
@@ -464,31 +477,29 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 }
             }
 #pragma unroll
-            for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * NST + 16 * j + c] = acc[t];
-            __syncthreads();
+            for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = acc[t];
+            __syncthreads();  // N^T is dead from here on
             float res[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int m = 0; m < 16; ++m) {  // X_ii P_ij
-                const float pv = sX[(16 * i + m) * NST + 16 * j + c];
-                const float4 xv = *reinterpret_cast<const float4 *>(sXd + i * 256 + m * 16 + r0);
-                res[0] = fmaf(xv.x, pv, res[0]);
-                res[1] = fmaf(xv.y, pv, res[1]);
-                res[2] = fmaf(xv.z, pv, res[2]);
-                res[3] = fmaf(xv.w, pv, res[3]);
+                const float pv = sX[(16 * i + m) * XST + 16 * j + c];
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    res[t] = fmaf(sX[(16 * i + r0 + t) * XST + 16 * i + m], pv, res[t]);
             }
             if (i == 3) {
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {  // + X_32 P_2j
-                    const float pv = sX[(32 + m) * NST + 16 * j + c];
+                    const float pv = sX[(32 + m) * XST + 16 * j + c];
 #pragma unroll
                     for (int t = 0; t < 4; ++t)
-                        res[t] = fmaf(sX[(48 + r0 + t) * NST + 32 + m], pv, res[t]);
+                        res[t] = fmaf(sX[(48 + r0 + t) * XST + 32 + m], pv, res[t]);
                 }
             }
             if (tid == 0) bulk_wait_group_read<0>();  // the A staging is read
             __syncthreads();
 #pragma unroll
-            for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * NST + 16 * j + c] = -res[t];
+            for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = -res[t];
             __syncthreads();
         }
         // T[i][j] = X[i][j] beta_j (lower triangle) -> bf16, K-major SW128 tile
@@ -498,61 +509,46 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int j = j8 * 8 + u;
-                o[u] = (j <= i) ? sX[i * NST + j] * sB[j] : 0.f;
+                o[u] = (j <= i) ? sX[i * XST + j] * sB[j] : 0.f;
             }
             *reinterpret_cast<uint4 *>(sT + i * 128 + ((j8 ^ (i & 7)) << 4)) = pack8(o);
         }
+        // K<- into the dead N^T area: scalar gate e^G . k from raw K, per-channel
+        // gate K^ . e^R
+        for (int e = tid; e < C * 16; e += kWyThreads) {
+            const int l = e >> 4, a = (e >> 3) & 1, jj = e & 7;
+            const int c0 = a * 64 + ((jj ^ (l & 7)) << 3);
+            float kv[8], o[8];
+            unpack8(*reinterpret_cast<const uint4 *>(sKQ + a * 16384 + l * 128 + jj * 16), kv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = kv[i] * __expf(CH ? sG[c0 + i] : sG[l]);
+            *reinterpret_cast<uint4 *>(sKL + a * 8192 + l * 128 + jj * 16) = pack8(o);
+        }
+    }
+    if (!CH) {  // V has landed in Q's place
+        const bool okv = mbar_wait_bounded(&bars[0], 1, kSpin, err);
+        if (!__syncthreads_and(okv)) goto cleanup;
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    // U^T = V^T T^T -> TMEM[64:128), W<-^T = K<-^T T^T -> TMEM[128:192)
+    // U^T = V^T T^T -> TMEM[0:64), W<-^T = K<-^T T^T -> TMEM[64:128)
     if (tid == 0) {
         tc_fence_after();
         const uint32_t id = idesc_bf16(128, 64, 1, 0);
         const uint64_t bd = sdesc_sw128(smem_u32(sT), 16, 1024);
-        const uint64_t av = sdesc_sw128(smem_u32(sV), 8192, 1024);
+        const uint64_t av = sdesc_sw128(smem_u32(sV), CH ? 8192 : 16384, 1024);
         const uint64_t ak = sdesc_sw128(smem_u32(sKL), 8192, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16_ss(tmem + 64, sdesc_add(av, kk * 2048), sdesc_add(bd, kk * 32), id, kk > 0);
-            mma_bf16_ss(tmem + 128, sdesc_add(ak, kk * 2048), sdesc_add(bd, kk * 32), id, kk > 0);
+            mma_bf16_ss(tmem, sdesc_add(av, kk * 2048), sdesc_add(bd, kk * 32), id, kk > 0);
+            mma_bf16_ss(tmem + 64, sdesc_add(ak, kk * 2048), sdesc_add(bd, kk * 32), id, kk > 0);
         }
         mma_commit(&bars[1]);
     }
-    // meanwhile: Q<- and K-> to the workspace, and the chunk decay
-    {
-        __nv_bfloat16 *Qg = ws.Q + slot * (C * D), *Kg = ws.K + slot * (C * D);
-        for (int e = tid; e < C * 16; e += kWyThreads) {
-            const int l = e >> 4, a = (e >> 3) & 1, j = e & 7;
-            const int c0 = a * 64 + ((j ^ (l & 7)) << 3);
-            const uint32_t off = a * 16384 + l * 128 + j * 16;
-            float kv[8], qv[8], wq[8], wk[8];
-            unpack8(*reinterpret_cast<const uint4 *>(sKQ + off), kv);
-            unpack8(*reinterpret_cast<const uint4 *>(sKQ + off + 8192), qv);
-            if (CH) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float Gl = sG[l * D + c0 + i];
-                    wq[i] = qv[i] * __expf(Gl);
-                    wk[i] = kv[i] * __expf(sG[(C - 1) * D + c0 + i] - Gl);
-                }
-            } else {
-                const float eq = __expf(sG[l]), ek = __expf(sG[C - 1] - sG[l]);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    wq[i] = qv[i] * eq;
-                    wk[i] = kv[i] * ek;
-                }
-            }
-            *reinterpret_cast<uint4 *>(Qg + l * D + c0) = pack8(wq);
-            *reinterpret_cast<uint4 *>(Kg + l * D + c0) = pack8(wk);
-        }
-        if (tid < D) ws.dec[slot * D + tid] = __expf(CH ? sG[(C - 1) * D + tid] : sG[C - 1]);
-    }
     {
         const bool ok = mbar_wait_bounded(&bars[1], 1, kSpin, err);
-        if (!__syncthreads_and(ok)) goto cleanup;  // also: the raw K/Q tiles are no longer read
+        if (!__syncthreads_and(ok)) goto cleanup;  // V and K<- are no longer read
     }
     tc_fence_after();
     {
@@ -560,10 +556,10 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         // (128 x 64 bf16, 128-byte swizzle) -> TMA stores
         const int d = qd * 32 + lane;
         float u[32], w[32];
-        tmem_ld16(tmem + lb + 64 + hf * 32, u);
-        tmem_ld16(tmem + lb + 64 + hf * 32 + 16, u + 16);
-        tmem_ld16(tmem + lb + 128 + hf * 32, w);
-        tmem_ld16(tmem + lb + 128 + hf * 32 + 16, w + 16);
+        tmem_ld16(tmem + lb + hf * 32, u);
+        tmem_ld16(tmem + lb + hf * 32 + 16, u + 16);
+        tmem_ld16(tmem + lb + 64 + hf * 32, w);
+        tmem_ld16(tmem + lb + 64 + hf * 32 + 16, w + 16);
         tmem_wait_ld();
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -584,7 +580,7 @@ cleanup:
     if (tid == 0) bulk_wait_group_read<0>();  // shared memory must outlive the stores' reads
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 0) tmem_dealloc(tmem, kWyTmemCols);
 }
 
 // ------------------------------------------------------------------ state kernel
@@ -935,7 +931,7 @@ constexpr CUtensorMapSwizzle kSW = CU_TENSOR_MAP_SWIZZLE_128B;
 constexpr CUtensorMapSwizzle kNoSW = CU_TENSOR_MAP_SWIZZLE_NONE;
 
 size_t wy_smem_bytes(bool ch) {  // + 1024 for the in-kernel alignment
-    return 1024 + WySmem::end_tc(ch) + 4 * (2 * 64 * WySmem::NST + 1024 + (ch ? 64 * D : 64) + 64) + 64;
+    return 1024 + WySmem::small(ch) + WySmem::small_bytes(ch);
 }
 
 }  // namespace
