@@ -84,10 +84,13 @@ def prefill_flops_split(C, dk, dv):
 
 
 def prefill_min_bytes(cfg, n_seq):
-    """One read of q, k, v, g, beta, S0 and one write of out and S_final."""
+    """One read of q, k, v, g, beta, S0 and one write of out and S_final (k, v
+    and beta once per substep when a token has n_h > 1 substeps)."""
     e = 2 if cfg.dtype == "bf16" else 4
     th = cfg.B * cfg.T * cfg.H
-    per = (2 * cfg.d_k + cfg.d_v) * e + cfg.d_v * e + 4 + (4 * cfg.d_k if cfg.gate == "channel" else 4)
+    nh = cfg.n_h
+    per = ((cfg.d_k + nh * (cfg.d_k + cfg.d_v)) * e + cfg.d_v * e + 4 * nh
+           + (4 * cfg.d_k if cfg.gate == "channel" else 4))
     states = n_seq * cfg.H * cfg.d_k * cfg.d_v * 4 * ((1 if cfg.s0_var > 0 else 0) + 1)
     return th * per + states
 
@@ -186,7 +189,8 @@ class PrefillRun:
     def __init__(self, cfg, device, seed, path):
         self.cfg = cfg
         self.device = device
-        self.inp = inputs.prefill_inputs(cfg, seed=seed)
+        gen = inputs.product_inputs if cfg.n_h > 1 else inputs.prefill_inputs
+        self.inp = gen(cfg, seed=seed)
         inp = self.inp
         self.n_seq = inp.n_seq
         self.q, self.k, self.v = (dev_tensor(x, cfg.dtype, device) for x in (inp.q, inp.k, inp.v))
@@ -199,14 +203,22 @@ class PrefillRun:
                               device=device)
         gate = 1 if cfg.gate == "channel" else 0
         dt = 1 if cfg.dtype == "bf16" else 0
-        ws = binding.fwd_workspace_size(cfg.B, cfg.T, cfg.H, cfg.d_k, cfg.d_v, cfg.chunk,
-                                        self.n_seq, self.cu is not None, dt, gate, path)
+        if cfg.n_h > 1:
+            ws = binding.fwd_product_workspace_size(cfg.B, cfg.T, cfg.H, cfg.n_h, cfg.d_k,
+                                                    cfg.d_v, cfg.chunk, self.n_seq,
+                                                    self.cu is not None, dt, gate, path)
+        else:
+            ws = binding.fwd_workspace_size(cfg.B, cfg.T, cfg.H, cfg.d_k, cfg.d_v, cfg.chunk,
+                                            self.n_seq, self.cu is not None, dt, gate, path)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
 
+    def call(self, q, k, v, g, b, S0, cu, out=None, S_final=None):
+        fn = binding.gdr_fwd_product if self.cfg.n_h > 1 else binding.gdr_fwd
+        return fn(q, k, v, g, b, S0, chunk=self.cfg.chunk, cu_seqlens=cu, out=out,
+                  S_final=S_final, path=self.path, workspace=self.ws)
+
     def step(self):
-        binding.gdr_fwd(self.q, self.k, self.v, self.g, self.beta, self.S0, chunk=self.cfg.chunk,
-                        cu_seqlens=self.cu, out=self.out, S_final=self.SF, path=self.path,
-                        workspace=self.ws)
+        self.call(self.q, self.k, self.v, self.g, self.beta, self.S0, self.cu, self.out, self.SF)
 
     def tokens(self):
         return self.cfg.B * self.cfg.T
@@ -242,8 +254,7 @@ class PrefillRun:
             b = hb.to(dev, non_blocking=True)
             S0 = None if hS0 is None else hS0.to(dev, non_blocking=True)
             cu = None if hcu is None else hcu.to(dev, non_blocking=True)
-            out, SF = binding.gdr_fwd(q, k, v, g, b, S0, chunk=cfg.chunk, cu_seqlens=cu,
-                                      path=self.path, workspace=self.ws)
+            out, SF = self.call(q, k, v, g, b, S0, cu)
             hout.copy_(out, non_blocking=True)
             hSF.copy_(SF, non_blocking=True)
 
@@ -304,16 +315,21 @@ def oracle_prefill_sample(cfg, seed, budget_s):
     Returns (equivalent tokens/s, cores, description)."""
     import oracle  # CPU baseline leg only
 
-    inp = inputs.prefill_inputs(cfg, seed=seed)
-    cores = oracle.default_threads()
-    n_seq = inp.n_seq
+    product = cfg.n_h > 1
+    inp = (inputs.product_inputs if product else inputs.prefill_inputs)(cfg, seed=seed)
+    cores = 1 if product else oracle.default_threads()
 
     def run(h):
         sl = lambda x: None if x is None else np.ascontiguousarray(x[:, :, :h])
+        sl3 = lambda x: np.ascontiguousarray(x[:, :, :, :h])  # [B, T, n_h, H, ...]
         S0 = None if inp.S0 is None else np.ascontiguousarray(inp.S0[:, :h])
         t = time.perf_counter()
-        oracle.recurrence_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.g), sl(inp.beta), S0=S0,
-                              cu_seqlens=inp.cu_seqlens, threads=cores)
+        if product:
+            oracle.product_fwd(sl(inp.q), sl3(inp.k), sl3(inp.v), sl(inp.g), sl3(inp.beta), S0,
+                               inp.cu_seqlens)
+        else:
+            oracle.recurrence_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.g), sl(inp.beta),
+                                  S0=S0, cu_seqlens=inp.cu_seqlens, threads=cores)
         return time.perf_counter() - t
 
     t1 = run(1)
@@ -352,10 +368,26 @@ def workload_config(name):
         c = inputs.PREFILL[name]
         return c, {"workload": name, "B": c.B, "T": c.T, "H": c.H, "d_k": c.d_k, "d_v": c.d_v,
                    "chunk": c.chunk, "gate": c.gate, "dtype_io": c.dtype,
-                   **({"n_seq": c.n_seq} if c.n_seq else {})}
+                   **({"n_seq": c.n_seq} if c.n_seq else {}),
+                   **({"n_h": c.n_h} if c.n_h > 1 else {})}
     c = inputs.DECODE[name]
     return c, {"workload": name, "N": c.N, "H": c.H, "d_k": c.d_k, "d_v": c.d_v, "gate": c.gate,
                "dtype_io": c.dtype, "steps_per_sequence": c.steps}
+
+
+class L2Flush:
+    """Leaves L2 cold and clean between steps: writes one buffer larger than L2,
+    then reads a second one, so the dirty lines of the write are written back
+    before the next timed interval starts instead of inside it."""
+
+    def __init__(self, device):
+        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.acc = torch.empty((), dtype=torch.float32, device=device)
+
+    def zero_(self):
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.acc)
 
 
 def time_steps(run, steps, flush):
@@ -413,8 +445,7 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
     is_decode = isinstance(cfg, inputs.DecodeConfig)
     run = (DecodeRun(cfg, device, seed, steps + warmup) if is_decode
            else PrefillRun(cfg, device, seed, path))
-    flush = None if is_decode else torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32,
-                                               device=device)
+    flush = None if is_decode else L2Flush(device)
     for _ in range(warmup):
         if flush is not None:
             flush.zero_()
@@ -453,7 +484,7 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                 "frac_of_8TBps_spec": ach / 8000.0}
         conf["l2"] = "no flush: the 512 MiB state is larger than L2 and is streamed every step"
     else:
-        th = cfg.B * cfg.T * cfg.H
+        th = cfg.B * cfg.T * cfg.H * cfg.n_h  # virtual steps when a token has substeps
         f_all = prefill_flops_per_token_head(cfg.chunk, cfg.d_k, cfg.d_v)
         wy, st_ = prefill_flops_split(cfg.chunk, cfg.d_k, cfg.d_v)
         share = {"fwd_simt": f_all, "tc_wy": wy, "tc_state": st_}.get(dom, 0)
@@ -478,7 +509,8 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                         "hbm_gbs_min_bytes": min_bytes / (ms * 1e-3) / 1e9,
                         "hbm_frac": min_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                         "flops_per_step": f_all * th, "min_bytes_per_step": min_bytes}
-        conf["l2"] = (f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the "
+        conf["l2"] = (f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then a "
+                      f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer, outside the "
                       "per-step CUDA-event intervals)")
         conf["path"] = path
     res = {"value": value, "ms_per_step": ms, "wall_s_incl_flush": wall, "roofline": roof,
@@ -508,7 +540,7 @@ def main():
     ap.add_argument("--workload", default="gdn_prefill",
                     choices=list(inputs.PREFILL) + list(inputs.DECODE))
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
-    ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill",
+    ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill,gdp_prefill",
                     help="comma-separated workloads measured after the main one ('' for none)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -20,7 +20,7 @@ GDR_OK, GDR_ERR_INVALID, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT = ra
 GDR_F32, GDR_BF16 = 0, 1
 GDR_GATE_SCALAR, GDR_GATE_PER_KEY_CHANNEL = 0, 1
 PATHS = {"auto": 0, "simt": 1, "tc": 2}
-KERNELS = {"decode": 0, "fwd_simt": 1, "tc_plan": 2, "tc_wy": 3, "tc_state": 4}
+KERNELS = {"decode": 0, "fwd_simt": 1, "tc_plan": 2, "tc_wy": 3, "tc_state": 4, "gdp_remap": 5}
 
 _lib = None
 
@@ -52,6 +52,11 @@ def lib() -> ctypes.CDLL:
         L.gdr_device_status.argtypes = [vp]
         L.gdr_selftest_wait_timeout.restype = i
         L.gdr_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+        L.gdr_fwd_product_workspace_size.restype = sz
+        L.gdr_fwd_product_workspace_size.argtypes = [i] * 12
+        L.gdr_fwd_product.restype = i
+        L.gdr_fwd_product.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, i,
+                                      i, i, i, vp, sz, vp]
         L.gdr_profile_enable.restype = None
         L.gdr_profile_enable.argtypes = [i]
         L.gdr_profile_read.restype = i
@@ -94,6 +99,12 @@ def fwd_workspace_size(B, T, H, d_k, d_v, chunk, n_seq, varlen, dtype, gate, pat
                                             dtype, gate, PATHS[path]))
 
 
+def fwd_product_workspace_size(B, T, H, n_h, d_k, d_v, chunk, n_seq, varlen, dtype, gate,
+                               path="auto") -> int:
+    return int(lib().gdr_fwd_product_workspace_size(B, T, H, n_h, d_k, d_v, chunk, n_seq,
+                                                    int(bool(varlen)), dtype, gate, PATHS[path]))
+
+
 def gdr_fwd(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, out=None,
             S_final=None, want_final: bool = True, path: str = "auto", workspace=None,
             stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
@@ -118,6 +129,37 @@ def gdr_fwd(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, out=
                        gate, PATHS[path], _ptr(workspace), ws_avail, _stream(stream))
     if st != GDR_OK:
         raise GdrError(st, "gdr_fwd")
+    return out, S_final
+
+
+def gdr_fwd_product(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, out=None,
+                    S_final=None, want_final: bool = True, path: str = "auto", workspace=None,
+                    stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Gated DeltaProduct prefill: k [B,T,n_h,H,d_k], v [B,T,n_h,H,d_v],
+    beta [B,T,n_h,H]; returns (out [B,T,H,d_v], S_final)."""
+    B, T, H, d_k = q.shape
+    n_h = k.shape[2]
+    d_v = v.shape[-1]
+    dtype = _dtype_code(q)
+    gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
+    n_seq = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+    _need_contig(q, k, v, g, beta, S0, cu_seqlens)
+    if out is None:
+        out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
+    if S_final is None and want_final:
+        S_final = torch.empty((n_seq, H, d_v, d_k), dtype=torch.float32, device=q.device)
+    ws_bytes = int(lib().gdr_fwd_product_workspace_size(B, T, H, n_h, d_k, d_v, chunk, n_seq,
+                                                       int(cu_seqlens is not None), dtype, gate,
+                                                       PATHS[path]))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    ws_avail = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdr_fwd_product(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                               _ptr(out), _ptr(S_final), B, T, H, n_h, d_k, d_v, chunk,
+                               _ptr(cu_seqlens), n_seq, dtype, gate, PATHS[path],
+                               _ptr(workspace), ws_avail, _stream(stream))
+    if st != GDR_OK:
+        raise GdrError(st, "gdr_fwd_product")
     return out, S_final
 
 

@@ -14,6 +14,9 @@ decode          N=256 sequences, H=32, d=128, bf16 tokens, fp32 state
                 S ~ N(0, 0.1), 1000 steps
 varlen_prefill  16 packed sequences, sum T = 65536, lengths uniform in
                 [1024, 7168], H=16, d=128, bf16, scalar gate, S0 = 0
+gdp_prefill     Gated DeltaProduct, n_h = 2 substeps per token: B=4, H=16,
+                T=2048 (4096 virtual steps), d=128, bf16, scalar gate,
+                S0 ~ N(0, 0.01)
 ==============  ==========================================================
 
 N(0, x) is read as mean 0, variance x.  Draw order for prefill: q, k, v,
@@ -50,6 +53,7 @@ class PrefillConfig:
     len_lo: int = 0
     len_hi: int = 0
     seed_index: int = 0
+    n_h: int = 1          # Householder substeps per token (> 1: Gated DeltaProduct)
 
     @property
     def tokens(self) -> int:
@@ -86,6 +90,8 @@ PREFILL = {
                                  0.0, seed_index=2),
     "varlen_prefill": PrefillConfig("varlen_prefill", 1, 65536, 16, 128, 128, 64, "bf16", "scalar",
                                     0.1, 0.0, n_seq=16, len_lo=1024, len_hi=7168, seed_index=4),
+    "gdp_prefill": PrefillConfig("gdp_prefill", 4, 2048, 16, 128, 128, 64, "bf16", "scalar", 0.1,
+                                 0.01, seed_index=5, n_h=2),
 }
 DECODE = {
     "decode": DecodeConfig("decode", 256, 32, 128, 128, "bf16", "scalar", 0.1, 0.1, 1000),
@@ -163,6 +169,38 @@ def prefill_inputs(cfg: PrefillConfig, seed: Optional[int] = None,
     k = _l2_rows(rng.standard_normal((B, T, H, dk), dtype=f32))
     v = rng.standard_normal((B, T, H, dv), dtype=f32)
     beta = _sigmoid(rng.standard_normal((B, T, H), dtype=f32))
+    gshape = (B, T, H, dk) if cfg.gate == "channel" else (B, T, H)
+    g = (-_softplus(rng.standard_normal(gshape, dtype=f32)) * f32(cfg.gate_scale)).astype(f32)
+    n_seq = cfg.n_seq if cfg.n_seq > 0 else B
+    var = cfg.s0_var if s0_var is None else s0_var
+    S0 = None
+    if var > 0:
+        S0 = (rng.standard_normal((n_seq, H, dv, dk), dtype=f32) * f32(np.sqrt(var))).astype(f32)
+    cu = None
+    if cfg.n_seq > 0:
+        if B != 1:
+            raise ValueError("packed batches have B = 1")
+        lens = varlen_lengths(rng, cfg.n_seq, T, cfg.len_lo, cfg.len_hi)
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return PrefillInputs(cfg, round_to(q, cfg.dtype), round_to(k, cfg.dtype),
+                         round_to(v, cfg.dtype), g, beta, S0, cu)
+
+
+def product_inputs(cfg: PrefillConfig, seed: Optional[int] = None,
+                   s0_var: Optional[float] = None) -> PrefillInputs:
+    """Draw one Gated DeltaProduct batch: as :func:`prefill_inputs`, with k
+    ``[B, T, n_h, H, d_k]``, v ``[B, T, n_h, H, d_v]`` and beta
+    ``[B, T, n_h, H]`` (one key, value and step size per substep); q and g stay
+    one per token.  Same draw order, each substep's k normalised on its own."""
+    if seed is None:
+        seed = BASE_SEED + cfg.seed_index
+    rng = np.random.default_rng(seed)
+    B, T, H, dk, dv, nh = cfg.B, cfg.T, cfg.H, cfg.d_k, cfg.d_v, cfg.n_h
+    f32 = np.float32
+    q = _l2_rows(rng.standard_normal((B, T, H, dk), dtype=f32))
+    k = _l2_rows(rng.standard_normal((B, T, nh, H, dk), dtype=f32))
+    v = rng.standard_normal((B, T, nh, H, dv), dtype=f32)
+    beta = _sigmoid(rng.standard_normal((B, T, nh, H), dtype=f32))
     gshape = (B, T, H, dk) if cfg.gate == "channel" else (B, T, H)
     g = (-_softplus(rng.standard_normal(gshape, dtype=f32)) * f32(cfg.gate_scale)).astype(f32)
     n_seq = cfg.n_seq if cfg.n_seq > 0 else B

@@ -145,6 +145,36 @@ gdr_status gdr_device_status(void *stream);
 gdr_status gdr_selftest_wait_timeout(unsigned int spin_limit, void *stream);
 
 /*
+ * Gated DeltaProduct prefill ("Linear Attention, Visualized", section "Gated
+ * Delta Product (GDP)"): every token t applies n_h substeps
+ *     S <- S (I - beta_tj k_tj k_tj^T) + beta_tj v_tj k_tj^T,   j = 1..n_h,
+ * after the token's single decay D_t, and o_t = S q_t is read after the last
+ * substep.  Computed, as the page's section "GDP as GDN over a virtual
+ * sequence" shows, by the gated delta rule over the n_h T virtual steps with
+ * the decay on the first substep and the query on the last; the prefill kernels
+ * run unchanged.
+ *
+ *  q        [B, T, H, d_k]          dtype
+ *  k        [B, T, n_h, H, d_k]     dtype (substeps of a token adjacent)
+ *  v        [B, T, n_h, H, d_v]     dtype
+ *  g        [B, T, H] or [B, T, H, d_k]  fp32 log-decay, one per token
+ *  beta     [B, T, n_h, H]          fp32
+ *  S0, S_final, out, cu_seqlens (token offsets of real tokens), chunk, path:
+ *           as for gdr_fwd.
+ *  workspace: at least gdr_fwd_product_workspace_size(...) bytes (holds the
+ *           virtual queries and gates, the virtual outputs and the inner
+ *           prefill's workspace).  n_h = 1 is gdr_fwd.
+ */
+size_t gdr_fwd_product_workspace_size(int B, int T, int H, int n_h, int d_k, int d_v, int chunk,
+                                      int n_seq, int varlen, gdr_dtype dtype, gdr_gate gate,
+                                      gdr_path path);
+gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const float *S0, void *out, float *S_final, int B,
+                           int T, int H, int n_h, int d_k, int d_v, int chunk,
+                           const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype, gdr_gate gate,
+                           gdr_path path, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * gdr_fwd_noalloc -- the prefill for callers that cannot allocate device
  * memory at call time (their memory manager owns the whole device heap and
  * forbids further cudaMalloc, or an allocation's device synchronisation is not
@@ -175,7 +205,7 @@ size_t gdr_fwd_noalloc_scratch_bytes(void);
 /*
  * Per-kernel launch accounting and timing (a small built-in profiler).
  * Kernel ids: GDR_K_DECODE, GDR_K_FWD_SIMT, GDR_K_TC_PLAN, GDR_K_TC_WY,
- * GDR_K_TC_STATE.  Launches are always counted.  While timing is enabled,
+ * GDR_K_TC_STATE, GDR_K_GDP_REMAP (the Gated DeltaProduct expand/gather).  Launches are always counted.  While timing is enabled,
  * every launch is bracketed by two CUDA events recorded on the launch's own
  * stream.  gdr_profile_read waits for the recorded events, returns the
  * launches and the summed device time (ms) of kernel `id` since the last read
@@ -183,7 +213,7 @@ size_t gdr_fwd_noalloc_scratch_bytes(void);
  * from other host threads.
  */
 enum { GDR_K_DECODE = 0, GDR_K_FWD_SIMT = 1, GDR_K_TC_PLAN = 2, GDR_K_TC_WY = 3,
-       GDR_K_TC_STATE = 4, GDR_K_COUNT = 5 };
+       GDR_K_TC_STATE = 4, GDR_K_GDP_REMAP = 5, GDR_K_COUNT = 6 };
 void gdr_profile_enable(int on);
 gdr_status gdr_profile_read(int id, long long *launches, double *total_ms);
 

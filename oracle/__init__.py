@@ -12,6 +12,9 @@ Two independent fp64 CPU implementations live here:
   the Arithmetic of Forgetting", section "The gated delta rule"; "Linear
   Attention, Visualized", sections "DeltaNet / Recurrent form", "Gated DeltaNet
   (GDN)" and "Kimi Delta Attention (KDA)".
+* :func:`product_fwd` -- Gated DeltaProduct, token by token with n_h
+  Householder substeps per token ("Linear Attention, Visualized", section
+  "Gated Delta Product (GDP)"), written from that definition.
 * :func:`oracle.chunked.chunked_fwd` -- the chunkwise WY/UT algorithm written
   from "Linear Attention, Visualized", sections "Gated DeltaNet (GDN) /
   Complete per-chunk algorithm" and "Kimi Delta Attention (KDA) / Complete
@@ -59,6 +62,10 @@ def _load():
                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ip, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int]
+            lib.oracle_gdp_fwd.restype = ctypes.c_int
+            lib.oracle_gdp_fwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ip, ctypes.c_int, ctypes.c_int]
             lib.oracle_gdr_decode_step.restype = ctypes.c_int
             lib.oracle_gdr_decode_step.argtypes = [dp, dp, dp, dp, dp, dp, dp,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -131,3 +138,28 @@ def recurrence_decode_step(q, k, v, g, beta, S):
     if rc != 0:
         raise ValueError("oracle_gdr_decode_step rejected its arguments")
     return out, S_new
+
+
+def product_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None):
+    """Gated DeltaProduct, fp64.  q ``[B,T,H,d_k]``; k ``[B,T,n_h,H,d_k]``;
+    v ``[B,T,n_h,H,d_v]``; g ``[B,T,H]`` or ``[B,T,H,d_k]``; beta
+    ``[B,T,n_h,H]``.  Returns ``(O [B,T,H,d_v], S_final [N,H,d_v,d_k])``."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    nh = k.shape[2]
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        n_seq = len(cu) - 1
+        cu_p = cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    else:
+        cu, n_seq, cu_p = None, B, None
+    S0a = None if S0 is None else _f64(S0)
+    out = np.zeros((B, T, H, dv))
+    S_final = np.zeros((n_seq, H, dv, dk))
+    rc = _load().oracle_gdp_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0a),
+                                _ptr(out), _ptr(S_final), B, T, H, nh, dk, dv, cu_p, n_seq,
+                                1 if g.ndim == 4 else 0)
+    if rc != 0:
+        raise ValueError("oracle_gdp_fwd rejected its arguments")
+    return out, S_final

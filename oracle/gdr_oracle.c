@@ -200,3 +200,69 @@ int oracle_gdr_decode_step(const double *q, const double *k, const double *v, co
     free(p);
     return 0;
 }
+
+/*
+ * Gated DeltaProduct ("Linear Attention, Visualized", section "Gated Delta
+ * Product (GDP)"): per token t, decay once (S' = S D_t), then n_h substeps
+ *     p = S k_tj;  u = beta_tj (v_tj - p);  S = S + u k_tj^T      (j = 1..n_h)
+ * and read o_t = S q_t after the last substep.  Written from that definition,
+ * not from the virtual-sequence mapping, so the mapping can be checked
+ * against it.
+ *   q [B,T,H,dk]; k [B,T,nh,H,dk]; v [B,T,nh,H,dv]; g [B,T,H] or [B,T,H,dk];
+ *   beta [B,T,nh,H]; S0/S_final [n_seq,H,dv,dk]; out [B,T,H,dv].
+ * Single-threaded over (sequence, head).
+ */
+int oracle_gdp_fwd(const double *q, const double *k, const double *v, const double *g,
+                   const double *beta, const double *S0, double *out, double *S_final, int B,
+                   int T, int H, int nh, int dk, int dv, const int *cu_seqlens, int n_seq,
+                   int per_channel) {
+    if (!q || !k || !v || !g || !beta || !out || nh < 1) return 1;
+    if (B <= 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return 1;
+    if (cu_seqlens) {
+        if (B != 1 || n_seq <= 0 || cu_seqlens[0] != 0 || cu_seqlens[n_seq] != T) return 1;
+        for (int i = 0; i < n_seq; ++i)
+            if (cu_seqlens[i + 1] < cu_seqlens[i]) return 1;
+    } else {
+        n_seq = B;
+    }
+    double *S = (double *)malloc(sizeof(double) * (size_t)dv * dk);
+    double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+    for (int s = 0; s < n_seq; ++s) {
+        long t0 = cu_seqlens ? cu_seqlens[s] : (long)s * T;
+        long t1 = cu_seqlens ? cu_seqlens[s + 1] : t0 + T;
+        for (int h = 0; h < H; ++h) {
+            const size_t soff = ((size_t)s * H + h) * (size_t)dv * dk;
+            if (S0) memcpy(S, S0 + soff, sizeof(double) * (size_t)dv * dk);
+            else memset(S, 0, sizeof(double) * (size_t)dv * dk);
+            for (long t = t0; t < t1; ++t) {
+                const size_t tok = (size_t)t * H + h;
+                for (int j = 0; j < dk; ++j) {
+                    const double a = per_channel ? exp(g[tok * dk + j]) : exp(g[tok]);
+                    for (int i = 0; i < dv; ++i) S[(size_t)i * dk + j] *= a;
+                }
+                for (int jj = 0; jj < nh; ++jj) {
+                    const size_t sub = ((size_t)t * nh + jj) * H + h;
+                    const double *kt = k + sub * dk, *vt = v + sub * dv;
+                    const double bt = beta[sub];
+                    for (int i = 0; i < dv; ++i) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * kt[j];
+                        u[i] = bt * (vt[i] - acc);
+                    }
+                    for (int i = 0; i < dv; ++i)
+                        for (int j = 0; j < dk; ++j) S[(size_t)i * dk + j] += u[i] * kt[j];
+                }
+                const double *qt = q + tok * dk;
+                for (int i = 0; i < dv; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * qt[j];
+                    out[tok * dv + i] = acc;
+                }
+            }
+            if (S_final) memcpy(S_final + soff, S, sizeof(double) * (size_t)dv * dk);
+        }
+    }
+    free(S);
+    free(u);
+    return 0;
+}

@@ -95,3 +95,35 @@ def test_workspace_size_is_zero_for_simt_and_rejected_args():
 
 def test_selftest_rejects_bad_limit():
     assert binding.lib().gdr_selftest_wait_timeout(0, None) == binding.GDR_ERR_INVALID
+
+
+def product(**kw):
+    a = dict(q=P, k=P, v=P, g=P, beta=P, S0=None, out=P, SF=P, B=2, T=64, H=2, nh=2, dk=128,
+             dv=128, chunk=64, cu=None, n_seq=2, dtype=1, gate=0, path=0, ws=P, ws_bytes=16)
+    a.update(kw)
+    return binding.lib().gdr_fwd_product(
+        a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["out"], a["SF"], a["B"], a["T"],
+        a["H"], a["nh"], a["dk"], a["dv"], a["chunk"], a["cu"], a["n_seq"], a["dtype"], a["gate"],
+        a["path"], a["ws"], a["ws_bytes"], None)
+
+
+@nogpu
+@pytest.mark.parametrize("kw,expect", [
+    (dict(nh=0), 1), (dict(dk=72), 2), (dict(dv=136), 2), (dict(q=ctypes.c_void_p(0x10004)), 1),
+    (dict(cu=P, B=2), 1), (dict(dtype=7), 1), (dict(ws=None, ws_bytes=0), 1), (dict(ws_bytes=16), 1),
+    (dict(k=None), 1),
+])
+def test_product_rejects_on_host(kw, expect):
+    assert product(**kw) == expect
+
+
+def test_product_workspace_holds_the_virtual_sequence():
+    """The product workspace covers q~, g~ and o~ for n_h T virtual steps plus
+    the gated delta rule's own workspace for them."""
+    lib = binding.lib()
+    B, T, H, nh, d = 2, 300, 4, 3, 128
+    inner = binding.fwd_workspace_size(B, T * nh, H, d, d, 64, B, False, 1, 0, "auto")
+    ws = binding.fwd_product_workspace_size(B, T, H, nh, d, d, 64, B, False, 1, 0, "auto")
+    assert inner > 0 and ws >= inner + 2 * B * T * nh * H * d * 2 + B * T * nh * H * 4
+    assert binding.fwd_product_workspace_size(B, T, H, 0, d, d, 64, B, False, 1, 0, "auto") == 0
+    assert lib.gdr_fwd_product_workspace_size is not None
