@@ -82,6 +82,12 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
         f[2 * i + 1] = x.y;
     }
 }
+__device__ __forceinline__ void ld8(const float *p, float *f) {  // 32-byte aligned
+    const float4 x = reinterpret_cast<const float4 *>(p)[0], y = reinterpret_cast<const float4 *>(p)[1];
+    f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+    f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
+}
+
 __device__ __forceinline__ uint4 pack8(const float *f) {
     uint4 u;
     __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
@@ -156,6 +162,10 @@ __global__ void plan_kernel(const int32_t *cu, int n_seq, int T_total, int *chun
 // lane quadrant (w & 3) and column half (w >> 2).
 constexpr int kWyThreads = 256;
 constexpr uint32_t kWyTmemCols = 128;
+// Issues every TMA load and the A store: a thread outside warps 0-1, which
+// load the gates and run the diagonal-block solve, so that a slow TMA issue
+// never holds up that work.
+constexpr int kWyTmaThread = 128;
 
 // Shared-memory plan (byte offsets from a 1024-aligned base).  Regions are
 // reused once their first contents are dead, so a scalar-gate CTA needs
@@ -175,7 +185,12 @@ struct WySmem {
     static constexpr uint32_t XEND = XR + 64 * XST * 4;
     static constexpr uint32_t VCH = 74752, KC = VCH + 16384;
     static constexpr uint32_t small(bool ch) { return ch ? KC + 16384 : XEND; }
-    static constexpr uint32_t small_bytes(bool ch) { return (ch ? (2 * D + 64) : 128) * 4 + 64; }
+    // scalar gate: G and beta per row; per-channel gate: R, G_C, beta, e^R and
+    // e^(G_C - R) per channel; then two mbarriers and the TMEM slot.  The
+    // scalar gate's Gram factors e^(G - R), e^(R - G) and their flag live in XR,
+    // which is dead until the solve.
+    static constexpr int small_floats(bool ch) { return ch ? 2 * D + 64 + 2 * D : 128; }
+    static constexpr uint32_t small_bytes(bool ch) { return small_floats(ch) * 4 + 64; }
 };
 
 template <bool CH>
@@ -200,7 +215,11 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     float *sG = sSm;                                                   // scalar: G [64]; channel: R row [128]
     float *sGC = sSm + (CH ? D : 64);                                  // channel: G_C row [128]
     float *sB = CH ? sGC + D : sSm + 64;                               // beta [64]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 64);            // [2]
+    // exponential tables, so that no element-wise exp is needed below
+    float *eR = sB + 64, *eCR = sB + 64 + D;                           // channel: per channel
+    float *eA = sX, *eB = sX + 64;                                     // scalar: per row (XR)
+    int *sFact = reinterpret_cast<int *>(sX + 128);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 64 + (CH ? 2 * D : 0));  // [2]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -227,7 +246,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    if (tid == 0) {
+    if (tid == kWyTmaThread) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
@@ -260,6 +279,20 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         b += __shfl_sync(0xffffffffu, a, 31);
         sG[lane] = a;
         sG[lane + 32] = b;
+        // Gamma[l][m] = e^(G_l - G_m) factorised around the middle row R = G_31 as
+        // e^(G_l - R) e^(R - G_m) -- exact up to rounding while every |G_l - R|
+        // stays far from the fp32 exp range; otherwise the Gram epilogue takes
+        // the exp of each difference (flag 0)
+        const float R = __shfl_sync(0xffffffffu, a, 31);
+        float spread = fmaxf(fabsf(a - R), fabsf(b - R));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, off));
+        eA[lane] = __expf(a - R);
+        eA[lane + 32] = __expf(b - R);
+        eB[lane] = __expf(R - a);
+        eB[lane + 32] = __expf(R - b);
+        if (lane == 0) *sFact = spread < 60.f;
     }
     {
         const bool ok_ld = mbar_wait_bounded(&bars[0], 0, kSpin, err);
@@ -269,20 +302,28 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         // per-channel scan, rows past the sequence end count as g = 0: thread
         // (c, half) scans 32 rows, the upper half then adds the lower half's total
         const int c = tid & 127, r0 = (tid >> 7) * 32;
-        float acc = 0.f;
-        for (int l = r0; l < r0 + 32; ++l) {
-            if (l < len) acc += sGt[l * D + c];
-            sGt[l * D + c] = acc;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = (r0 + i < len) ? sGt[(r0 + i) * D + c] : 0.f;
+#pragma unroll
+        for (int i = 1; i < 32; ++i) v[i] += v[i - 1];
+        if (!r0) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sGt[i * D + c] = v[i];
         }
         __syncthreads();
         if (r0) {
             const float base = sGt[31 * D + c];
-            for (int l = 32; l < 64; ++l) sGt[l * D + c] += base;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sGt[(32 + i) * D + c] = v[i] + base;
         }
         __syncthreads();
         if (tid < D) {
-            sG[tid] = sGt[31 * D + tid];         // reference row R of the Gram factorisation
-            sGC[tid] = sGt[(C - 1) * D + tid];   // G_C
+            const float R = sGt[31 * D + tid], GC = sGt[(C - 1) * D + tid];
+            sG[tid] = R;    // reference row R of the Gram factorisation
+            sGC[tid] = GC;  // G_C
+            eR[tid] = __expf(R);
+            eCR[tid] = __expf(GC - R);
         }
     }
     // zero K and Q rows beyond the sequence end (whole 128-byte rows)
@@ -298,22 +339,32 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     // workspace; per-channel gate also K-check = k e^(R - G) and, in place,
     // K^ = k e^(G - R), Q^ = q e^(G - R) (R = row 31 of G).
     {
+        // thread: channels c0..c0+7 (8-channel group cg) of rows l0, l0+16, ...;
+        // the group's per-channel factors stay in registers
         __nv_bfloat16 *Qg = ws.Q + slot * (C * D), *Kg = ws.K + slot * (C * D);
-        for (int e = tid; e < C * 16; e += kWyThreads) {
-            const int l = e >> 4, a = (e >> 3) & 1, j = e & 7;
-            const int c0 = a * 64 + ((j ^ (l & 7)) << 3);
+        const int cg = tid & 15, c0 = cg * 8, a = cg >> 3, l0 = tid >> 4;
+        float R8[8], eR8[8], eCR8[8];
+        if (CH) {
+            ld8(sG + c0, R8);
+            ld8(eR + c0, eR8);
+            ld8(eCR + c0, eCR8);
+        }
+#pragma unroll
+        for (int k = 0; k < C / 16; ++k) {
+            const int l = l0 + 16 * k, j = (cg & 7) ^ (l & 7);  // physical 16-byte chunk
             const uint32_t off = a * 16384 + l * 128 + j * 16;
             float kv[8], qv[8], wq[8], wk[8];
             unpack8(*reinterpret_cast<const uint4 *>(sKQ + off), kv);
             unpack8(*reinterpret_cast<const uint4 *>(sKQ + off + 8192), qv);
             if (CH) {
-                float kh[8], qh[8], kc[8];
+                float kh[8], qh[8], kc[8], G8[8];
+                ld8(sGt + l * D + c0, G8);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float Gl = sGt[l * D + c0 + i], R = sG[c0 + i];
-                    wq[i] = qv[i] * __expf(Gl);
-                    wk[i] = kv[i] * __expf(sGC[c0 + i] - Gl);
-                    const float e1 = __expf(Gl - R), e2 = __expf(R - Gl);
+                    // e^G = e^(G - R) e^R and e^(G_C - G) = e^(R - G) e^(G_C - R)
+                    const float e1 = __expf(G8[i] - R8[i]), e2 = __expf(R8[i] - G8[i]);
+                    wq[i] = qv[i] * (e1 * eR8[i]);
+                    wk[i] = kv[i] * (e2 * eCR8[i]);
                     kh[i] = kv[i] * e1;
                     qh[i] = qv[i] * e1;
                     kc[i] = kv[i] * e2;
@@ -332,7 +383,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             *reinterpret_cast<uint4 *>(Qg + l * D + c0) = pack8(wq);
             *reinterpret_cast<uint4 *>(Kg + l * D + c0) = pack8(wk);
         }
-        if (tid < D) ws.dec[slot * D + tid] = __expf(CH ? sGC[tid] : sG[C - 1]);
+        if (tid < D) ws.dec[slot * D + tid] = CH ? eCR[tid] * eR[tid] : __expf(sG[C - 1]);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -359,11 +410,6 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         if (!__syncthreads_and(ok)) goto cleanup;
     }
     tc_fence_after();
-    if (!CH && tid == 0) {  // Q is read: V takes its place (lands during the solve)
-        mbar_arrive_expect_tx(&bars[0], 2 * kHalfBytes);
-        tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
-        tma_load_2d(sV + 16384, &tm_v, &bars[0], x0 + 64, ytok);
-    }
     {
         // accumulator rows 0..63: K K^T -> N = diag(beta) tril_-1(. Gamma), stored
         // transposed; rows 64..127: Q K^T -> A = tril_0(. Gamma), bf16, staged in TT
@@ -372,36 +418,50 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         tmem_ld16(tmem + lb + m0, gr);
         tmem_ld16(tmem + lb + m0 + 16, gr + 16);
         tmem_wait_ld();
-        const float Gl = CH ? 0.f : sG[l];
-        if (qd < 2) {
-            const float bl = sB[l];
+        // gam(m) = Gamma[l][m] (scalar gate; the per-channel gate is inside the operands)
+        auto epilogue = [&](auto gam) {
+            if (qd < 2) {
+                const float bl = sB[l];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int m = m0 + i;
-                const float w = CH ? 1.f : __expf(Gl - sG[m]);
-                sN[m * NTS + l] = (m < l) ? bl * gr[i] * w : 0.f;
-            }
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                float o[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int m = m0 + jj * 8 + i;
-                    const float w = CH ? 1.f : __expf(Gl - sG[m]);
-                    o[i] = (m <= l) ? gr[jj * 8 + i] * w : 0.f;
+                for (int i = 0; i < 32; ++i) {
+                    const int m = m0 + i;
+                    sN[m * NTS + l] = (m < l) ? bl * gr[i] * gam(m) : 0.f;
                 }
-                const int j = hf * 4 + jj;
-                *reinterpret_cast<uint4 *>(sT + l * 128 + ((j ^ (l & 7)) << 4)) = pack8(o);
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    float o[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int m = m0 + jj * 8 + i;
+                        o[i] = (m <= l) ? gr[jj * 8 + i] * gam(m) : 0.f;
+                    }
+                    const int j = hf * 4 + jj;
+                    *reinterpret_cast<uint4 *>(sT + l * 128 + ((j ^ (l & 7)) << 4)) = pack8(o);
+                }
             }
+        };
+        if (CH) {
+            epilogue([](int) { return 1.f; });
+        } else if (*sFact) {
+            const float eAl = eA[l];
+            epilogue([&](int m) { return eAl * eB[m]; });
+        } else {
+            const float Gl = sG[l];
+            epilogue([&](int m) { return __expf(Gl - sG[m]); });
         }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {  // A -> workspace
+    if (tid == kWyTmaThread) {  // A -> workspace
         tma_store_2d(&tm_Ast, sT, 0, (int)(slot * C));
         bulk_commit_group();
+        if (!CH) {  // Q is read: V takes its place (lands during the solve)
+            mbar_arrive_expect_tx(&bars[0], 2 * kHalfBytes);
+            tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
+            tma_load_2d(sV + 16384, &tm_v, &bars[0], x0 + 64, ytok);
+        }
     }
     // T = (I + N)^{-1} diag(beta), N = diag(beta) L strictly lower, by 16 x 16
     // blocks: X_ii = (I + N_ii)^{-1} by forward substitution (one column per
@@ -496,7 +556,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                         res[t] = fmaf(sX[(48 + r0 + t) * XST + 32 + m], pv, res[t]);
                 }
             }
-            if (tid == 0) bulk_wait_group_read<0>();  // the A staging is read
+            if (tid == kWyTmaThread) bulk_wait_group_read<0>();  // the A staging is read
             __syncthreads();
 #pragma unroll
             for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = -res[t];
@@ -515,14 +575,20 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         }
         // K<- into the dead N^T area: scalar gate e^G . k from raw K, per-channel
         // gate K^ . e^R
-        for (int e = tid; e < C * 16; e += kWyThreads) {
-            const int l = e >> 4, a = (e >> 3) & 1, jj = e & 7;
-            const int c0 = a * 64 + ((jj ^ (l & 7)) << 3);
-            float kv[8], o[8];
-            unpack8(*reinterpret_cast<const uint4 *>(sKQ + a * 16384 + l * 128 + jj * 16), kv);
+        {
+            const int cg = tid & 15, c0 = cg * 8, a = cg >> 3, l0 = tid >> 4;
+            float eR8[8];
+            if (CH) ld8(eR + c0, eR8);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = kv[i] * __expf(CH ? sG[c0 + i] : sG[l]);
-            *reinterpret_cast<uint4 *>(sKL + a * 8192 + l * 128 + jj * 16) = pack8(o);
+            for (int k = 0; k < C / 16; ++k) {
+                const int l = l0 + 16 * k, jj = (cg & 7) ^ (l & 7);
+                float kv[8], o[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sKQ + a * 16384 + l * 128 + jj * 16), kv);
+                const float el = CH ? 0.f : __expf(sG[l]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[i] = kv[i] * (CH ? eR8[i] : el);
+                *reinterpret_cast<uint4 *>(sKL + a * 8192 + l * 128 + jj * 16) = pack8(o);
+            }
         }
     }
     if (!CH) {  // V has landed in Q's place
@@ -577,7 +643,8 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         bulk_commit_group();
     }
 cleanup:
-    if (tid == 0) bulk_wait_group_read<0>();  // shared memory must outlive the stores' reads
+    // shared memory must outlive the stores' reads
+    if (tid == 0 || tid == kWyTmaThread) bulk_wait_group_read<0>();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kWyTmemCols);

@@ -249,6 +249,16 @@ def test_tc_small_against_oracle(cuda_device, gate, T):
     check(inputs.prefill_inputs(cfg, seed=301), cuda_device, path="tc")
 
 
+@pytest.mark.parametrize("gate_scale", [1.5, 4.0])
+def test_tc_strong_scalar_gates(cuda_device, gate_scale):
+    """Scalar log-decays far larger than the workloads': with scale 1.5 the
+    Gram weights come from the factorised exponentials with wide exponent
+    ranges; with scale 4 the spread inside a chunk passes the factorisation's
+    limit and the kernel takes the exp of every difference."""
+    cfg = small_cfg(B=2, T=300, H=2, gate_scale=gate_scale)
+    check(inputs.prefill_inputs(cfg, seed=305), cuda_device, path="tc")
+
+
 def test_tc_varlen_with_empty_and_unit_sequences(cuda_device):
     cfg = inputs.PREFILL["varlen_prefill"].replace(T=600, H=2, n_seq=0, s0_var=0.01)
     inp = inputs.prefill_inputs(cfg, seed=302)
