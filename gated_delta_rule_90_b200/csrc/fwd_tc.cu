@@ -14,6 +14,7 @@
 //                  (I + diag(beta) L) T = diag(beta) by column forward
 //                  substitution in fp32 (shared memory);
 //                  U^T = V^T T^T and W<-^T = K<-^T T^T on the tensor cores;
+//                  (W<- is stored back in token-major order)
 //                writes W<-, U, A, Q<- = e^G . q, K-> = e^(G_C - G) . k and the
 //                chunk decay e^(G_C) to the workspace (bf16 tiles, fp32 decay).
 //  state_kernel  one CTA per (sequence, head), chunks in order (the boundary
@@ -63,7 +64,8 @@ struct Ws {
     int *chunk_start;  // [n_seq + 1] (varlen)
     int *order;        // [n_seq] longest first (varlen)
     float *dec;        // [slots*H][128]
-    __nv_bfloat16 *W, *U;          // transposed: [slots*H][128 (d)][64 (token)]
+    __nv_bfloat16 *W;              // [slots*H][64 (token)][128 (d)]
+    __nv_bfloat16 *U;              // transposed: [slots*H][128 (d)][64 (token)]
     __nv_bfloat16 *Q, *K;          // [slots*H][64 (token)][128 (d)]
     __nv_bfloat16 *A;              // [slots*H][64][64]
 };
@@ -197,7 +199,7 @@ template <bool CH>
 __global__ void __launch_bounds__(kWyThreads)
 wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-          const __grid_constant__ CUtensorMap tm_Ust, const __grid_constant__ CUtensorMap tm_Wst,
+          const __grid_constant__ CUtensorMap tm_Ust,
           const __grid_constant__ CUtensorMap tm_Ast, const float *__restrict__ g,
           const float *__restrict__ beta, const int32_t *__restrict__ cu, Geo geo, Ws ws,
           unsigned int *err) {
@@ -618,8 +620,8 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     }
     tc_fence_after();
     {
-        // U^T, W<-^T rows (feature d, 32 tokens each) -> staging in the K/Q area
-        // (128 x 64 bf16, 128-byte swizzle) -> TMA stores
+        // U^T as [d][token] (this thread: row d, 32 tokens) -> staging in the
+        // K/Q area (128-byte swizzle) -> TMA store; W<- (this thread: column d)
         const int d = qd * 32 + lane;
         float u[32], w[32];
         tmem_ld16(tmem + lb + hf * 32, u);
@@ -632,14 +634,17 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             const int j = hf * 4 + jj;
             const uint32_t off = d * 128 + ((j ^ (d & 7)) << 4);
             *reinterpret_cast<uint4 *>(sKQ + off) = pack8(u + jj * 8);
-            *reinterpret_cast<uint4 *>(sKQ + 16384 + off) = pack8(w + jj * 8);
         }
+        // W<- goes straight to the workspace in token-major order: per token,
+        // a warp writes 32 consecutive features (64 contiguous bytes)
+        __nv_bfloat16 *wg = ws.W + slot * (C * D) + d;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) wg[(hf * 32 + i) * D] = __float2bfloat16_rn(w[i]);
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
         tma_store_2d(&tm_Ust, sKQ, 0, (int)(slot * D));
-        tma_store_2d(&tm_Wst, sKQ + 16384, 0, (int)(slot * D));
         bulk_commit_group();
     }
 cleanup:
@@ -656,29 +661,41 @@ cleanup:
 //               lane quadrant (w & 3) -- state rows d = 32 (w & 3) + lane -- and
 //               column half (w >> 2) of the accumulators it touches.
 //   warps 8-11  output: O^T (TMEM) -> shared staging -> TMA store.
-//   warp 12     producer: TMA loads of the next chunks and every tcgen05.mma.
+//   warp 12     MMA issue: every tcgen05.mma, in chunk order, never waiting on
+//               a load slot, so it answers the chain's hand-offs at once.
+//   warp 13     TMA: loads chunk r + 2 into a stage once chunk r's MMAs are done.
 // The roles hand over through mbarriers only; the chain never waits on the
-// output path.  TMEM columns: S [0,128), Z^T [128,192), O^T x2 [192,320).
+// output path.  TMEM columns: S [0,128); two buffers [Z^T | O^T] at [128,256)
+// and [256,384), filled by one N = 128 MMA per k-step; and the bf16 A
+// operands of the MMAs -- S [384,448) and Z^T [448,480), two elements per
+// column -- so the MMAs read only B from shared memory.
 struct StSmem {
-    // per stage: W<-^T (128 x 64, MN-major B), Q<- (64 x 128, K-major B),
+    // per stage: [W<-; Q<-] stacked along N (128 x 128, K-major B: each 64-column
+    // atom holds W<- rows then Q<- rows),
     // K-> (64 x 128, MN-major B), U^T (128 x 64), A (64 x 64, K-major B)
-    static constexpr uint32_t WT = 0, Q = 16384, K = 32768, UT = 49152, A = 65536;
+    static constexpr uint32_t WQ = 0, K = 32768, UT = 49152, A = 65536;
     static constexpr uint32_t STAGE = 73728;
     static constexpr uint32_t DEC = 2 * STAGE;      // decay [2][128] fp32
-    static constexpr uint32_t S = DEC + 1024;       // bf16 S, K-major A operand (2 atoms)
-    static constexpr uint32_t ZT = S + 32768;       // bf16 Z^T, K-major A operand
-    static constexpr uint32_t OST = ZT + 16384;     // O staging for the TMA store [64][128]
+    static constexpr uint32_t OST = DEC + 1024;     // O staging for the TMA store [64][128]
     static constexpr uint32_t BARS = OST + 16384;
     static constexpr uint32_t TOTAL = BARS + 256;
     static constexpr uint32_t TX = 4 * kTileBytes + kHalfBytes + kDecBytes;
 };
 constexpr int kChainThreads = 256, kOutThreads = 128;
-constexpr int kStThreads = kChainThreads + kOutThreads + 32;
+constexpr int kStThreads = kChainThreads + kOutThreads + 64;
 constexpr uint32_t kStTmemCols = 512;
 
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+__device__ __forceinline__ void named_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Chain -> MMA-warp hand-offs on hardware named barriers (the chain warps
+// arrive, the MMA warp syncs).  Both sides pass each barrier exactly twice per
+// chunk on every path, error paths included, so neither can be left waiting.
+constexpr int kBarOpsS = 2, kBarOpsZ = 3;
+constexpr int kOpsThreads = 256 + 32;
 
 __global__ void __launch_bounds__(kStThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ CUtensorMap tm_U,
@@ -690,12 +707,10 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + StSmem::BARS);  // [2] TMA stage loaded
-    uint64_t *opsS = full + 2;   // chain: S operand + decayed S ready    (count 256)
-    uint64_t *opsZ = full + 3;   // chain: Z^T operand ready               (count 256)
     uint64_t *barZ = full + 4;   // mma: Z^T accumulated
     uint64_t *barS = full + 5;   // mma: S update accumulated
     uint64_t *barO = full + 6;   // [2] mma: O^T buffer complete
-    uint64_t *oFree = full + 8;  // [2] output warps: O^T buffer read (count 128)
+    uint64_t *oFree = full + 8;  // [2] output warps: O^T buffer read (one arrival per warp)
     uint32_t *tslot = reinterpret_cast<uint32_t *>(full + 10);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int unit = blockIdx.x;
@@ -709,14 +724,12 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
-        mbar_init(opsS, kChainThreads);
-        mbar_init(opsZ, kChainThreads);
         mbar_init(barZ, 1);
         mbar_init(barS, 1);
         mbar_init(&barO[0], 1);
         mbar_init(&barO[1], 1);
-        mbar_init(&oFree[0], kOutThreads);
-        mbar_init(&oFree[1], kOutThreads);
+        mbar_init(&oFree[0], kOutThreads / 32);
+        mbar_init(&oFree[1], kOutThreads / 32);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -727,7 +740,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t tS = tmem, tZ = tmem + 128, tO0 = tmem + 192;
+    const uint32_t tS = tmem, tZO0 = tmem + 128, tS16 = tmem + 384, tZ16 = tmem + 448;
     bool ok = true;
 
     if (warp < 8) {
@@ -744,44 +757,51 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             tmem_st16(tS + lb + hf * 64 + cb * 16, v);
         }
         tmem_wait_st();
-        for (int r = 0; r < nch && ok; ++r) {
+        for (int r = 0; r < nch; ++r) {
             const uint8_t *st = sm + (r & 1) * StSmem::STAGE;
-            ok = mbar_wait_bounded(&full[r & 1], (r >> 1) & 1, kSpin, err);
-            if (r > 0) ok = ok && mbar_wait_bounded(barS, (r - 1) & 1, kSpin, err);
-            if (!ok) break;
-            tc_fence_after();
-            {   // S (fp32) -> bf16 operand; S <- S Diag(decay) in TMEM
-                const float *dec = reinterpret_cast<const float *>(sm + StSmem::DEC) +
-                                   (r & 1) * D + hf * 64;
-                float v[64];
+            if (ok) ok = mbar_wait_bounded(&full[r & 1], (r >> 1) & 1, kSpin, err);
+            if (ok && r > 0) ok = mbar_wait_bounded(barS, (r - 1) & 1, kSpin, err);
+            float v[64];
+            if (ok) {  // S (fp32) -> bf16 operand in TMEM
+                tc_fence_after();
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) tmem_ld16(tS + lb + hf * 64 + cb * 16, v + cb * 16);
                 tmem_wait_ld();
-                uint8_t *rowp = sm + StSmem::S + hf * 16384 + d * 128;
+                float p[32];  // bf16 pairs
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<uint4 *>(rowp + ((j ^ (d & 7)) << 4)) = pack8(v + j * 8);
-                // the Z and O MMAs need only the bf16 copy: release it first
-                fence_proxy_async_smem();
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 w = pack8(v + j * 8);
+                    p[4 * j] = __uint_as_float(w.x);
+                    p[4 * j + 1] = __uint_as_float(w.y);
+                    p[4 * j + 2] = __uint_as_float(w.z);
+                    p[4 * j + 3] = __uint_as_float(w.w);
+                }
+                tmem_st16(tS16 + lb + hf * 32, p);
+                tmem_st16(tS16 + lb + hf * 32 + 16, p + 16);
+                tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(opsS);
-                // S <- S Diag(decay), needed by the S-update MMA (after opsZ)
+            }
+            // the Z and O MMAs need only the bf16 copy: release it first
+            named_arrive(kBarOpsS, kOpsThreads);
+            if (ok) {  // S <- S Diag(decay), needed by the S-update MMA (after opsZ)
+                const float *dec = reinterpret_cast<const float *>(sm + StSmem::DEC) +
+                                   (r & 1) * D + hf * 64;
 #pragma unroll
                 for (int i = 0; i < 64; ++i) v[i] *= dec[i];
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) tmem_st16(tS + lb + hf * 64 + cb * 16, v + cb * 16);
                 tmem_wait_st();
             }
-            ok = mbar_wait_bounded(barZ, r & 1, kSpin, err);
-            if (!ok) break;
-            tc_fence_after();
-            {   // Z^T = U^T - S W<-^T -> bf16 K-major operand (this thread: 32 tokens)
+            if (ok) ok = mbar_wait_bounded(barZ, r & 1, kSpin, err);
+            if (ok) {  // Z^T = U^T - S W<-^T -> bf16 A operand in TMEM (this thread: 32 tokens)
+                tc_fence_after();
                 float z[32];
+                const uint32_t tZ = tZO0 + (r & 1) * 128;
                 tmem_ld16(tZ + lb + hf * 32, z);
                 tmem_ld16(tZ + lb + hf * 32 + 16, z + 16);
                 tmem_wait_ld();
                 const uint8_t *urow = st + StSmem::UT + d * 128;
-                uint8_t *zrow = sm + StSmem::ZT + d * 128;
+                float p[16];
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                     const int j = hf * 4 + jj;
@@ -789,12 +809,17 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
                     unpack8(*reinterpret_cast<const uint4 *>(urow + ((j ^ (d & 7)) << 4)), u);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) u[i] -= z[jj * 8 + i];
-                    *reinterpret_cast<uint4 *>(zrow + ((j ^ (d & 7)) << 4)) = pack8(u);
+                    const uint4 w = pack8(u);
+                    p[4 * jj] = __uint_as_float(w.x);
+                    p[4 * jj + 1] = __uint_as_float(w.y);
+                    p[4 * jj + 2] = __uint_as_float(w.z);
+                    p[4 * jj + 3] = __uint_as_float(w.w);
                 }
+                tmem_st16(tZ16 + lb + hf * 16, p);
+                tmem_wait_st();
+                tc_fence_before();
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(opsZ);
+            named_arrive(kBarOpsZ, kOpsThreads);
         }
         if (ok && nch > 0) ok = mbar_wait_bounded(barS, (nch - 1) & 1, kSpin, err);
         tc_fence_after();
@@ -823,10 +848,12 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             tc_fence_after();
             float o[64];
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tO0 + (r & 1) * 64 + lb + cb * 16, o + cb * 16);
+            for (int cb = 0; cb < 4; ++cb)
+                tmem_ld16(tZO0 + (r & 1) * 128 + 64 + lb + cb * 16, o + cb * 16);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&oFree[r & 1]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&oFree[r & 1]);
             const long ts = t0 + (long)r * C;
             const int len = (int)min((long)C, t1 - ts);
             if (len == C) {
@@ -848,22 +875,24 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             }
         }
         if (otid == 0) bulk_wait_group_read<0>();
-    } else if (lane == 0) {
-        // ===================== producer: TMA + MMA =====================
+    } else if (warp == 13 && lane == 0) {
+        // ===================== TMA loads =====================
         auto issue = [&](int r) {
             uint8_t *st = sm + (r & 1) * StSmem::STAGE;
             uint64_t *bar = &full[r & 1];
             const size_t sl = (size_t)(gc0 + r) * geo.H + h;
             mbar_arrive_expect_tx(bar, StSmem::TX);
-            tma_load_2d(st + StSmem::WT, &tm_W, bar, 0, (int)(sl * D));
+            tma_load_2d(st + StSmem::WQ, &tm_W, bar, 0, (int)(sl * C));
+            tma_load_2d(st + StSmem::WQ + 16384, &tm_W, bar, 64, (int)(sl * C));
             tma_load_2d(st + StSmem::UT, &tm_U, bar, 0, (int)(sl * D));
-            tma_load_2d(st + StSmem::Q, &tm_Q, bar, 0, (int)(sl * C));
-            tma_load_2d(st + StSmem::Q + 8192, &tm_Q, bar, 64, (int)(sl * C));
+            tma_load_2d(st + StSmem::WQ + 8192, &tm_Q, bar, 0, (int)(sl * C));
+            tma_load_2d(st + StSmem::WQ + 16384 + 8192, &tm_Q, bar, 64, (int)(sl * C));
             tma_load_2d(st + StSmem::K, &tm_K, bar, 0, (int)(sl * C));
             tma_load_2d(st + StSmem::K + 8192, &tm_K, bar, 64, (int)(sl * C));
             tma_load_2d(st + StSmem::A, &tm_A, bar, 0, (int)(sl * C));
             bulk_load(sm + StSmem::DEC + (r & 1) * kDecBytes, ws.dec + sl * D, kDecBytes, bar);
         };
+        int issued = 0;
         if (nch > 0) {
             prefetch_tmap(&tm_W);
             prefetch_tmap(&tm_U);
@@ -872,54 +901,62 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             prefetch_tmap(&tm_A);
             prefetch_tmap(&tm_out);
             issue(0);
-            if (nch > 1) issue(1);
+            issued = 1;
+            if (nch > 1) {
+                issue(1);
+                issued = 2;
+            }
         }
-        const uint32_t idZ = idesc_bf16(128, 64, 0, 1);
+        // stage r & 1 is free once chunk r - 2's MMAs (the last is O2) are done
+        for (int r = 2; r < nch && ok; ++r) {
+            ok = mbar_wait_bounded(&barO[r & 1], ((r - 2) >> 1) & 1, kSpin, err);
+            if (!ok) break;
+            issue(r);
+            issued = r + 1;
+        }
+        // let every load this thread issued land before the CTA can exit
+        for (int i = issued - 2; i < issued; ++i)
+            if (i >= 0) mbar_wait_bounded(&full[i & 1], (i >> 1) & 1, kSpin, err);
+    } else if (warp == 12) {
+        // ===================== MMA issue (lane 0; the warp syncs) =====================
+        const uint32_t idZO = idesc_bf16(128, 128, 0, 0);
         const uint32_t idO = idesc_bf16(128, 64, 0, 0);
         const uint32_t idS = idesc_bf16(128, 128, 0, 1);
         // operand descriptors, built once; k-steps only advance the start address
-        const uint64_t dS = sdesc_sw128(smem_u32(sm + StSmem::S), 16, 1024);
-        const uint64_t dZT = sdesc_sw128(smem_u32(sm + StSmem::ZT), 16, 1024);
-        const uint64_t dW0 = sdesc_sw128(smem_u32(sm + StSmem::WT), 16384, 1024);
-        const uint64_t dQ0 = sdesc_sw128(smem_u32(sm + StSmem::Q), 16, 1024);
+        const uint64_t dWQ0 = sdesc_sw128(smem_u32(sm + StSmem::WQ), 16, 1024);
         const uint64_t dK0 = sdesc_sw128(smem_u32(sm + StSmem::K), 8192, 1024);
         const uint64_t dA0 = sdesc_sw128(smem_u32(sm + StSmem::A), 16, 1024);
         const uint32_t stage16 = StSmem::STAGE >> 4;  // stage stride in descriptor units
-        for (int r = 0; r < nch && ok; ++r) {
-            const uint32_t tO = tO0 + (r & 1) * 64;
+        for (int r = 0; r < nch; ++r) {
+            const uint32_t tZr = tZO0 + (r & 1) * 128, tO = tZr + 64;
             const uint64_t so = (r & 1) ? stage16 : 0;
-            const uint64_t dw = dW0 + so, dq = dQ0 + so, dk = dK0 + so, da = dA0 + so;
-            ok = mbar_wait_bounded(opsS, r & 1, kSpin, err);
-            if (!ok) break;
-            tc_fence_after();
+            const uint64_t dwq = dWQ0 + so, dk = dK0 + so, da = dA0 + so;
+            // this buffer's O half must have been read out (chunk r - 2)
+            if (ok && lane == 0 && r >= 2)
+                ok = mbar_wait_bounded(&oFree[r & 1], ((r - 2) >> 1) & 1, kSpin, err);
+            __syncwarp();
+            // the chain has written S(r) in bf16 (and so has seen chunk r's stage land)
+            named_sync(kBarOpsS, kOpsThreads);
+            if (ok && lane == 0) {
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // Z^T = S W<-^T
-                mma_bf16_ss(tZ, sdesc_add(dS, (kk >> 2) * 16384 + (kk & 3) * 32),
-                            sdesc_add(dw, kk * 2048), idZ, kk > 0);
-            mma_commit(barZ);
-            if (r >= 2) ok = mbar_wait_bounded(&oFree[r & 1], ((r - 2) >> 1) & 1, kSpin, err);
-            if (!ok) break;
-            tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk)  // [Z^T | O^T] = S [W<-; Q<-]^T
+                    mma_bf16_ts(tZr, tS16 + kk * 8,
+                                sdesc_add(dwq, (kk >> 2) * 16384 + (kk & 3) * 32), idZO, kk > 0);
+                mma_commit(barZ);
+            }
+            __syncwarp();
+            named_sync(kBarOpsZ, kOpsThreads);
+            if (ok && lane == 0) {
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // O^T = S Q<-^T
-                mma_bf16_ss(tO, sdesc_add(dS, (kk >> 2) * 16384 + (kk & 3) * 32),
-                            sdesc_add(dq, (kk >> 2) * 8192 + (kk & 3) * 32), idO, kk > 0);
-            ok = mbar_wait_bounded(opsZ, r & 1, kSpin, err);
-            if (!ok) break;
-            tc_fence_after();
+                for (int kk = 0; kk < 4; ++kk)  // S += Z^T K->
+                    mma_bf16_ts(tS, tZ16 + kk * 8, sdesc_add(dk, kk * 2048), idS, 1);
+                mma_commit(barS);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)  // S += Z^T K->
-                mma_bf16_ss(tS, sdesc_add(dZT, kk * 32), sdesc_add(dk, kk * 2048), idS, 1);
-            mma_commit(barS);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)  // O^T += Z^T A^T
-                mma_bf16_ss(tO, sdesc_add(dZT, kk * 32), sdesc_add(da, kk * 32), idO, 1);
-            mma_commit(&barO[r & 1]);
-            // this stage is free once chunk r's MMAs are done: prefetch chunk r+2
-            if (r + 2 < nch) {
-                ok = mbar_wait_bounded(&barO[r & 1], (r >> 1) & 1, kSpin, err);
-                if (!ok) break;
-                issue(r + 2);
+                for (int kk = 0; kk < 4; ++kk)  // O^T += Z^T A^T
+                    mma_bf16_ts(tO, tZ16 + kk * 8, sdesc_add(da, kk * 32), idO, 1);
+                mma_commit(&barO[r & 1]);
             }
         }
     }
@@ -1048,7 +1085,7 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
             !make_map(&mv, kBF, v, HD, tok_rows, HD * 2, 64, 64, kSW) ||
             (gate == GDR_GATE_PER_KEY_CHANNEL &&
              !make_map(&mg, kF32, g, HD, tok_rows, HD * 4, D, 64, kNoSW)) ||
-            !make_map(&mW, kBF, ws.W, C, tiles * D, C * 2, 64, 128, kSW) ||
+            !make_map(&mW, kBF, ws.W, D, tiles * C, D * 2, 64, 64, kSW) ||
             !make_map(&mU, kBF, ws.U, C, tiles * D, C * 2, 64, 128, kSW) ||
             !make_map(&mQ, kBF, ws.Q, D, tiles * C, D * 2, 64, 64, kSW) ||
             !make_map(&mK, kBF, ws.K, D, tiles * C, D * 2, 64, 64, kSW) ||
@@ -1075,7 +1112,7 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
             return e;
         dim3 grid((unsigned)L.n_slots, (unsigned)H);
         ProfToken tk = prof_begin(GDR_K_TC_WY, st);
-        kern<<<grid, kWyThreads, smem, st>>>(mq, mk, mv, mg, mU, mW, mA, g, beta, cu, geo, ws, err);
+        kern<<<grid, kWyThreads, smem, st>>>(mq, mk, mv, mg, mU, mA, g, beta, cu, geo, ws, err);
         prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
