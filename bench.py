@@ -36,28 +36,36 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 SM_COUNT = 148
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu capture (summaries under profiles/), valid only for the kernel source
-# it was taken on: keyed by the first 16 hex digits of that file's sha256.
+# one ncu capture (summaries under profiles/), valid only for the kernel sources
+# it was taken on: keyed by (kernel, workload), with the first 16 hex digits of
+# the sha256 of those sources in order.
+_TC_SRC = ('csrc/fwd_tc.cu', 'csrc/sm100.cuh', 'csrc/common.cuh')
+_DEC_SRC = ('csrc/decode.cu', 'csrc/common.cuh')
 NCU_TRAFFIC = {
-    "tc_wy": ("csrc/fwd_tc.cu", "738ff82dc9443843", 206.187264e6 + 253.290496e6),
-    "tc_state": ("csrc/fwd_tc.cu", "738ff82dc9443843", 308.476928e6 + 56.973312e6),
-    "decode": ("csrc/decode.cu", "8ab7b74f4e29cd3d", 543.248896e6 + 482.370048e6),
+    ("tc_wy", "gdn_prefill"): (_TC_SRC, "53402063a98e7810", 206.236928e6 + 254.719488e6),
+    ("tc_state", "gdn_prefill"): (_TC_SRC, "53402063a98e7810", 308.370432e6 + 57.609728e6),
+    ("tc_wy", "kda_prefill"): (_TC_SRC, "53402063a98e7810", 680.951040e6 + 565.304576e6),
+    ("decode", "decode"): (_DEC_SRC, "9fc20c5d1e64ce78", 543.248896e6 + 482.370048e6),
 }
 
 
 def ncu_traffic(kernel, workload):
-    """Measured traffic of `kernel` if its source is unchanged since the capture
-    (captures were taken on the gdn_prefill and decode workloads only)."""
+    """Measured traffic of `kernel` on `workload` if its sources are unchanged
+    since the capture, else None."""
     import hashlib
-    ent = NCU_TRAFFIC.get(kernel)
-    if ent is None or workload not in ("gdn_prefill", "decode"):
+    ent = NCU_TRAFFIC.get((kernel, workload))
+    if ent is None:
         return None
-    path = os.path.join(ROOT, "gated_delta_rule_90_b200", ent[0])
+    h = hashlib.sha256()
     try:
-        digest = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+        for f in ent[0]:
+            with open(os.path.join(ROOT, "gated_delta_rule_90_b200", f), "rb") as fh:
+                h.update(fh.read())
     except OSError:
         return None
-    return ent[2] if digest == ent[1] else None
+    return ent[2] if h.hexdigest()[:16] == ent[1] else None
+
+
 L2_FLUSH_BYTES = 256 << 20
 
 
