@@ -17,6 +17,9 @@ varlen_prefill  16 packed sequences, sum T = 65536, lengths uniform in
 gdp_prefill     Gated DeltaProduct, n_h = 2 substeps per token: B=4, H=16,
                 T=2048 (4096 virtual steps), d=128, bf16, scalar gate,
                 S0 ~ N(0, 0.01)
+gdn2_prefill    Gated DeltaNet-2 (erase gate b per key channel, write gate w
+                per value channel, b, w = sigmoid(N(0, 1))): B=2, H=16,
+                T=4096, d=128, bf16, per-channel decay, S0 = 0
 ==============  ==========================================================
 
 N(0, x) is read as mean 0, variance x.  Draw order for prefill: q, k, v,
@@ -92,6 +95,8 @@ PREFILL = {
                                     0.1, 0.0, n_seq=16, len_lo=1024, len_hi=7168, seed_index=4),
     "gdp_prefill": PrefillConfig("gdp_prefill", 4, 2048, 16, 128, 128, 64, "bf16", "scalar", 0.1,
                                  0.01, seed_index=5, n_h=2),
+    "gdn2_prefill": PrefillConfig("gdn2_prefill", 2, 4096, 16, 128, 128, 64, "bf16", "channel", 0.05,
+                                  0.0, seed_index=6),
 }
 DECODE = {
     "decode": DecodeConfig("decode", 256, 32, 128, 128, "bf16", "scalar", 0.1, 0.1, 1000),
@@ -216,6 +221,56 @@ def product_inputs(cfg: PrefillConfig, seed: Optional[int] = None,
         cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     return PrefillInputs(cfg, round_to(q, cfg.dtype), round_to(k, cfg.dtype),
                          round_to(v, cfg.dtype), g, beta, S0, cu)
+
+
+@dataclasses.dataclass
+class Gdn2Inputs:
+    cfg: PrefillConfig
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    g: np.ndarray
+    b: np.ndarray          # erase gate [B, T, H, d_k]
+    w: np.ndarray          # write gate [B, T, H, d_v]
+    S0: Optional[np.ndarray]
+    cu_seqlens: Optional[np.ndarray]
+
+    @property
+    def n_seq(self) -> int:
+        return self.cfg.B if self.cu_seqlens is None else len(self.cu_seqlens) - 1
+
+
+def gdn2_inputs(cfg: PrefillConfig, seed: Optional[int] = None,
+                s0_var: Optional[float] = None) -> Gdn2Inputs:
+    """Draw one Gated DeltaNet-2 batch: as :func:`prefill_inputs`, with the
+    scalar beta replaced by an erase gate b (per key channel) and a write gate
+    w (per value channel), each sigmoid(N(0, 1)).  Draw order: q, k, v, b
+    logits, w logits, gate noise, S0, lengths."""
+    if seed is None:
+        seed = BASE_SEED + cfg.seed_index
+    rng = np.random.default_rng(seed)
+    B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.d_k, cfg.d_v
+    f32 = np.float32
+    q = _l2_rows(rng.standard_normal((B, T, H, dk), dtype=f32))
+    k = _l2_rows(rng.standard_normal((B, T, H, dk), dtype=f32))
+    v = rng.standard_normal((B, T, H, dv), dtype=f32)
+    b = _sigmoid(rng.standard_normal((B, T, H, dk), dtype=f32))
+    w = _sigmoid(rng.standard_normal((B, T, H, dv), dtype=f32))
+    gshape = (B, T, H, dk) if cfg.gate == "channel" else (B, T, H)
+    g = (-_softplus(rng.standard_normal(gshape, dtype=f32)) * f32(cfg.gate_scale)).astype(f32)
+    n_seq = cfg.n_seq if cfg.n_seq > 0 else B
+    var = cfg.s0_var if s0_var is None else s0_var
+    S0 = None
+    if var > 0:
+        S0 = (rng.standard_normal((n_seq, H, dv, dk), dtype=f32) * f32(np.sqrt(var))).astype(f32)
+    cu = None
+    if cfg.n_seq > 0:
+        if B != 1:
+            raise ValueError("packed batches have B = 1")
+        lens = varlen_lengths(rng, cfg.n_seq, T, cfg.len_lo, cfg.len_hi)
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return Gdn2Inputs(cfg, round_to(q, cfg.dtype), round_to(k, cfg.dtype), round_to(v, cfg.dtype),
+                      g, b, w, S0, cu)
 
 
 @dataclasses.dataclass

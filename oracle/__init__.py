@@ -15,6 +15,11 @@ Two independent fp64 CPU implementations live here:
 * :func:`product_fwd` -- Gated DeltaProduct, token by token with n_h
   Householder substeps per token ("Linear Attention, Visualized", section
   "Gated Delta Product (GDP)"), written from that definition.
+* :func:`gdn2_fwd` -- Gated DeltaNet-2 (decoupled erase and write gates),
+  token by token ("Gated DeltaNet-2, and the gate that was doing two jobs",
+  section "What decoupling actually means here"), and
+  :func:`oracle.chunked.gdn2_chunked_fwd`, its chunkwise form from the same
+  section, used only to pin it.
 * :func:`oracle.chunked.chunked_fwd` -- the chunkwise WY/UT algorithm written
   from "Linear Attention, Visualized", sections "Gated DeltaNet (GDN) /
   Complete per-chunk algorithm" and "Kimi Delta Attention (KDA) / Complete
@@ -66,6 +71,9 @@ def _load():
             lib.oracle_gdp_fwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ip, ctypes.c_int, ctypes.c_int]
+            lib.oracle_gdn2_fwd.restype = ctypes.c_int
+            lib.oracle_gdn2_fwd.argtypes = [dp] * 9 + [ctypes.c_int] * 5 + [ip, ctypes.c_int,
+                                                                             ctypes.c_int]
             lib.oracle_gdr_decode_step.restype = ctypes.c_int
             lib.oracle_gdr_decode_step.argtypes = [dp, dp, dp, dp, dp, dp, dp,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -162,4 +170,28 @@ def product_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None):
                                 1 if g.ndim == 4 else 0)
     if rc != 0:
         raise ValueError("oracle_gdp_fwd rejected its arguments")
+    return out, S_final
+
+
+def gdn2_fwd(q, k, v, g, b, w, S0=None, cu_seqlens=None):
+    """Gated DeltaNet-2, fp64.  q, k ``[B,T,H,d_k]``; v ``[B,T,H,d_v]``; g
+    ``[B,T,H]`` or ``[B,T,H,d_k]``; erase gate b ``[B,T,H,d_k]``; write gate w
+    ``[B,T,H,d_v]``.  Returns ``(O [B,T,H,d_v], S_final [N,H,d_v,d_k])``."""
+    q, k, v, g, b, w = (_f64(x) for x in (q, k, v, g, b, w))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        n_seq = len(cu) - 1
+        cu_p = cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    else:
+        cu, n_seq, cu_p = None, B, None
+    S0a = None if S0 is None else _f64(S0)
+    out = np.zeros((B, T, H, dv))
+    S_final = np.zeros((n_seq, H, dv, dk))
+    rc = _load().oracle_gdn2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0a),
+                                 _ptr(out), _ptr(S_final), B, T, H, dk, dv, cu_p, n_seq,
+                                 1 if g.ndim == 4 else 0)
+    if rc != 0:
+        raise ValueError("oracle_gdn2_fwd rejected its arguments")
     return out, S_final

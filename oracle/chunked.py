@@ -97,3 +97,47 @@ def chunked_fwd(q, k, v, g, beta, chunk, S0=None, cu_seqlens=None):
                 out[b, c0:c1, h] = O
             S_final[s, h] = S.T
     return out, S_final
+
+
+def gdn2_chunked_fwd(q, k, v, g, b, w, S0=None, C=64):
+    """Chunkwise Gated DeltaNet-2 in fp64 -- pins :func:`oracle.gdn2_fwd`.
+
+    "Gated DeltaNet-2, and the gate that was doing two jobs", section "What
+    decoupling actually means here", in its row convention (S is d_k x d_v,
+    o = S^T q).  Inside a chunk the decay is normalised out: with Gamma_t the
+    product of the chunk's decays up to t, the keys are scaled by the inverse
+    decay (k~ = Gamma_t^-1 k) and the erase vectors by the decay
+    (e~ = Gamma_t e), which leaves an undecayed recurrence
+    S~_t = (I - k~_t e~_t^T) S~_{t-1} + k~_t z_t^T.  Then T = tril(E~ K~^T, -1),
+    A = (I + T)^-1, and the one solve serves both right-hand sides, Y = A E~
+    and U = A Z, with the chunk's correction rows U - Y S0.
+    Shapes as :func:`oracle.gdn2_fwd` for one batch row set (B sequences of
+    length T); returns the column-convention state.
+    """
+    q, k, v, g, b, w = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, b, w))
+    Bn, T, H, dk = q.shape
+    dv = v.shape[-1]
+    out = np.zeros((Bn, T, H, dv))
+    Sf = np.zeros((Bn, H, dv, dk))
+    for s in range(Bn):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else np.array(S0[s, h], dtype=np.float64).T.copy()
+            for c0 in range(0, T, C):
+                c1 = min(T, c0 + C)
+                Kc, Qc, Vc = k[s, c0:c1, h], q[s, c0:c1, h], v[s, c0:c1, h]
+                E = b[s, c0:c1, h] * Kc
+                Z = w[s, c0:c1, h] * Vc
+                a = np.exp(g[s, c0:c1, h])
+                if a.ndim == 1:
+                    a = np.repeat(a[:, None], dk, axis=1)
+                Gam = np.cumprod(a, axis=0)            # Gamma_t, one row per token
+                Kt, Et, Qt = Kc / Gam, E * Gam, Qc * Gam
+                n = c1 - c0
+                Tm = np.tril(Et @ Kt.T, -1)
+                A = np.linalg.solve(np.eye(n) + Tm, np.eye(n))
+                Y, U = A @ Et, A @ Z
+                Ucorr = U - Y @ S                      # rows u_t^T
+                out[s, c0:c1, h] = Qt @ S + np.tril(Qt @ Kt.T) @ Ucorr
+                S = Gam[-1][:, None] * (S + Kt.T @ Ucorr)
+            Sf[s, h] = S.T
+    return out, Sf

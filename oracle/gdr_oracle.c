@@ -266,3 +266,70 @@ int oracle_gdp_fwd(const double *q, const double *k, const double *v, const doub
     free(u);
     return 0;
 }
+
+/*
+ * Gated DeltaNet-2 ("Gated DeltaNet-2, and the gate that was doing two jobs",
+ * section "What decoupling actually means here"): the scalar step size splits
+ * into an erase gate b_t (per key channel) and a write gate w_t (per value
+ * channel), e_t = b_t . k_t, z_t = w_t . v_t, and in the page's row convention
+ *     S_t = (I - k_t e_t^T) D_t S_{t-1} + k_t z_t^T,   o_t = S_t^T q_t.
+ * Transposed to the column convention used here (S is d_v x d_k):
+ *     S' = S D_t;  p = S' e_t;  u = z_t - p;  S = S' + u k_t^T;  o_t = S q_t.
+ *   q, k [B,T,H,dk]; v, out [B,T,H,dv]; g [B,T,H] or [B,T,H,dk];
+ *   b [B,T,H,dk]; w [B,T,H,dv]; S0/S_final [n_seq,H,dv,dk].
+ * Single-threaded over (sequence, head).
+ */
+int oracle_gdn2_fwd(const double *q, const double *k, const double *v, const double *g,
+                    const double *b, const double *w, const double *S0, double *out,
+                    double *S_final, int B, int T, int H, int dk, int dv, const int *cu_seqlens,
+                    int n_seq, int per_channel) {
+    if (!q || !k || !v || !g || !b || !w || !out) return 1;
+    if (B <= 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return 1;
+    if (cu_seqlens) {
+        if (B != 1 || n_seq <= 0 || cu_seqlens[0] != 0 || cu_seqlens[n_seq] != T) return 1;
+        for (int i = 0; i < n_seq; ++i)
+            if (cu_seqlens[i + 1] < cu_seqlens[i]) return 1;
+    } else {
+        n_seq = B;
+    }
+    double *S = (double *)malloc(sizeof(double) * (size_t)dv * dk);
+    double *e = (double *)malloc(sizeof(double) * (size_t)dk);
+    double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+    for (int s = 0; s < n_seq; ++s) {
+        long t0 = cu_seqlens ? cu_seqlens[s] : (long)s * T;
+        long t1 = cu_seqlens ? cu_seqlens[s + 1] : t0 + T;
+        for (int h = 0; h < H; ++h) {
+            const size_t soff = ((size_t)s * H + h) * (size_t)dv * dk;
+            if (S0) memcpy(S, S0 + soff, sizeof(double) * (size_t)dv * dk);
+            else memset(S, 0, sizeof(double) * (size_t)dv * dk);
+            for (long t = t0; t < t1; ++t) {
+                const size_t tok = (size_t)t * H + h;
+                const double *kt = k + tok * dk, *vt = v + tok * dv, *qt = q + tok * dk;
+                for (int j = 0; j < dk; ++j) {
+                    const double a = per_channel ? exp(g[tok * dk + j]) : exp(g[tok]);
+                    for (int i = 0; i < dv; ++i) S[(size_t)i * dk + j] *= a;
+                    e[j] = b[tok * dk + j] * kt[j];
+                }
+                for (int i = 0; i < dv; ++i) {
+                    double p = 0.0;
+                    for (int j = 0; j < dk; ++j) p += S[(size_t)i * dk + j] * e[j];
+                    u[i] = w[tok * dv + i] * vt[i] - p;
+                }
+                for (int i = 0; i < dv; ++i) {
+                    double acc = 0.0;
+                    double *row = S + (size_t)i * dk;
+                    for (int j = 0; j < dk; ++j) {
+                        row[j] += u[i] * kt[j];
+                        acc += row[j] * qt[j];
+                    }
+                    out[tok * dv + i] = acc;
+                }
+            }
+            if (S_final) memcpy(S_final + soff, S, sizeof(double) * (size_t)dv * dk);
+        }
+    }
+    free(S);
+    free(e);
+    free(u);
+    return 0;
+}
