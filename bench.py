@@ -97,7 +97,8 @@ def prefill_min_bytes(cfg, n_seq):
     e = 2 if cfg.dtype == "bf16" else 4
     th = cfg.B * cfg.T * cfg.H
     nh = cfg.n_h
-    per = ((cfg.d_k + nh * (cfg.d_k + cfg.d_v)) * e + cfg.d_v * e + 4 * nh
+    gates = 4 * (cfg.d_k + cfg.d_v) if cfg.variant == "gdn2" else 4 * nh  # b, w or beta
+    per = ((cfg.d_k + nh * (cfg.d_k + cfg.d_v)) * e + cfg.d_v * e + gates
            + (4 * cfg.d_k if cfg.gate == "channel" else 4))
     states = n_seq * cfg.H * cfg.d_k * cfg.d_v * 4 * ((1 if cfg.s0_var > 0 else 0) + 1)
     return th * per + states
@@ -197,12 +198,17 @@ class PrefillRun:
     def __init__(self, cfg, device, seed, path):
         self.cfg = cfg
         self.device = device
-        gen = inputs.product_inputs if cfg.n_h > 1 else inputs.prefill_inputs
+        self.gdn2 = cfg.variant == "gdn2"
+        gen = (inputs.gdn2_inputs if self.gdn2 else
+               inputs.product_inputs if cfg.n_h > 1 else inputs.prefill_inputs)
         self.inp = gen(cfg, seed=seed)
         inp = self.inp
         self.n_seq = inp.n_seq
         self.q, self.k, self.v = (dev_tensor(x, cfg.dtype, device) for x in (inp.q, inp.k, inp.v))
-        self.g, self.beta = dev_tensor(inp.g, "f32", device), dev_tensor(inp.beta, "f32", device)
+        self.g = dev_tensor(inp.g, "f32", device)
+        # Gated DeltaNet-2 passes its (erase, write) gates where the others pass beta
+        self.beta = ((dev_tensor(inp.b, "f32", device), dev_tensor(inp.w, "f32", device))
+                     if self.gdn2 else dev_tensor(inp.beta, "f32", device))
         self.S0 = dev_tensor(inp.S0, "f32", device)
         self.cu = None if inp.cu_seqlens is None else torch.from_numpy(inp.cu_seqlens).to(device)
         self.path = path
@@ -211,7 +217,9 @@ class PrefillRun:
                               device=device)
         gate = 1 if cfg.gate == "channel" else 0
         dt = 1 if cfg.dtype == "bf16" else 0
-        if cfg.n_h > 1:
+        if self.gdn2:
+            ws = 0  # CUDA-core path, no workspace
+        elif cfg.n_h > 1:
             ws = binding.fwd_product_workspace_size(cfg.B, cfg.T, cfg.H, cfg.n_h, cfg.d_k,
                                                     cfg.d_v, cfg.chunk, self.n_seq,
                                                     self.cu is not None, dt, gate, path)
@@ -221,6 +229,9 @@ class PrefillRun:
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
 
     def call(self, q, k, v, g, b, S0, cu, out=None, S_final=None):
+        if self.gdn2:
+            return binding.gdr_fwd_gdn2(q, k, v, g, b[0], b[1], S0, chunk=self.cfg.chunk,
+                                        cu_seqlens=cu, out=out, S_final=S_final)
         fn = binding.gdr_fwd_product if self.cfg.n_h > 1 else binding.gdr_fwd
         return fn(q, k, v, g, b, S0, chunk=self.cfg.chunk, cu_seqlens=cu, out=out,
                   S_final=S_final, path=self.path, workspace=self.ws)
@@ -245,11 +256,13 @@ class PrefillRun:
             return t.pin_memory()
 
         hq, hk, hv = (host(x, cfg.dtype) for x in (inp.q, inp.k, inp.v))
-        hg, hb, hS0 = host(inp.g, "f32"), host(inp.beta, "f32"), host(inp.S0, "f32")
+        hg, hS0 = host(inp.g, "f32"), host(inp.S0, "f32")
+        hb = (host(inp.b, "f32"), host(inp.w, "f32")) if self.gdn2 else host(inp.beta, "f32")
         hcu = None if inp.cu_seqlens is None else torch.from_numpy(inp.cu_seqlens).pin_memory()
         hout = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
         hSF = torch.empty(self.SF.shape, dtype=torch.float32).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hS0, hcu)
+        hbs = hb if isinstance(hb, tuple) else (hb,)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, *hbs, hS0, hcu)
                   if t is not None)
         d2h = hout.numel() * hout.element_size() + hSF.numel() * hSF.element_size()
         st = torch.cuda.current_stream()
@@ -259,7 +272,8 @@ class PrefillRun:
             k = hk.to(dev, non_blocking=True)
             v = hv.to(dev, non_blocking=True)
             g = hg.to(dev, non_blocking=True)
-            b = hb.to(dev, non_blocking=True)
+            b = (tuple(x.to(dev, non_blocking=True) for x in hb) if isinstance(hb, tuple)
+                 else hb.to(dev, non_blocking=True))
             S0 = None if hS0 is None else hS0.to(dev, non_blocking=True)
             cu = None if hcu is None else hcu.to(dev, non_blocking=True)
             out, SF = self.call(q, k, v, g, b, S0, cu)
@@ -323,16 +337,20 @@ def oracle_prefill_sample(cfg, seed, budget_s):
     Returns (equivalent tokens/s, cores, description)."""
     import oracle  # CPU baseline leg only
 
-    product = cfg.n_h > 1
-    inp = (inputs.product_inputs if product else inputs.prefill_inputs)(cfg, seed=seed)
-    cores = 1 if product else oracle.default_threads()
+    product, gdn2 = cfg.n_h > 1, cfg.variant == "gdn2"
+    gen = inputs.gdn2_inputs if gdn2 else inputs.product_inputs if product else inputs.prefill_inputs
+    inp = gen(cfg, seed=seed)
+    cores = 1 if (product or gdn2) else oracle.default_threads()
 
     def run(h):
         sl = lambda x: None if x is None else np.ascontiguousarray(x[:, :, :h])
         sl3 = lambda x: np.ascontiguousarray(x[:, :, :, :h])  # [B, T, n_h, H, ...]
         S0 = None if inp.S0 is None else np.ascontiguousarray(inp.S0[:, :h])
         t = time.perf_counter()
-        if product:
+        if gdn2:
+            oracle.gdn2_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.g), sl(inp.b), sl(inp.w), S0,
+                            inp.cu_seqlens)
+        elif product:
             oracle.product_fwd(sl(inp.q), sl3(inp.k), sl3(inp.v), sl(inp.g), sl3(inp.beta), S0,
                                inp.cu_seqlens)
         else:
@@ -377,7 +395,8 @@ def workload_config(name):
         return c, {"workload": name, "B": c.B, "T": c.T, "H": c.H, "d_k": c.d_k, "d_v": c.d_v,
                    "chunk": c.chunk, "gate": c.gate, "dtype_io": c.dtype,
                    **({"n_seq": c.n_seq} if c.n_seq else {}),
-                   **({"n_h": c.n_h} if c.n_h > 1 else {})}
+                   **({"n_h": c.n_h} if c.n_h > 1 else {}),
+                   **({"variant": c.variant} if c.variant else {})}
     c = inputs.DECODE[name]
     return c, {"workload": name, "N": c.N, "H": c.H, "d_k": c.d_k, "d_v": c.d_v, "gate": c.gate,
                "dtype_io": c.dtype, "steps_per_sequence": c.steps}
@@ -495,9 +514,9 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
         th = cfg.B * cfg.T * cfg.H * cfg.n_h  # virtual steps when a token has substeps
         f_all = prefill_flops_per_token_head(cfg.chunk, cfg.d_k, cfg.d_v)
         wy, st_ = prefill_flops_split(cfg.chunk, cfg.d_k, cfg.d_v)
-        share = {"fwd_simt": f_all, "tc_wy": wy, "tc_state": st_}.get(dom, 0)
+        share = {"fwd_simt": f_all, "gdn2_simt": f_all, "tc_wy": wy, "tc_state": st_}.get(dom, 0)
         flops = share * th
-        if dom == "fwd_simt":
+        if dom in ("fwd_simt", "gdn2_simt"):
             peak = SM_COUNT * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
             ach = flops / (dom_ms * 1e-3) / 1e12
             roof = {"bound": "alu", "kernel": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
@@ -548,7 +567,7 @@ def main():
     ap.add_argument("--workload", default="gdn_prefill",
                     choices=list(inputs.PREFILL) + list(inputs.DECODE))
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
-    ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill,gdp_prefill",
+    ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill,gdp_prefill,gdn2_prefill",
                     help="comma-separated workloads measured after the main one ('' for none)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

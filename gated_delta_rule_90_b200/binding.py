@@ -20,7 +20,8 @@ GDR_OK, GDR_ERR_INVALID, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT = ra
 GDR_F32, GDR_BF16 = 0, 1
 GDR_GATE_SCALAR, GDR_GATE_PER_KEY_CHANNEL = 0, 1
 PATHS = {"auto": 0, "simt": 1, "tc": 2}
-KERNELS = {"decode": 0, "fwd_simt": 1, "tc_plan": 2, "tc_wy": 3, "tc_state": 4, "gdp_remap": 5}
+KERNELS = {"decode": 0, "fwd_simt": 1, "tc_plan": 2, "tc_wy": 3, "tc_state": 4, "gdp_remap": 5,
+           "gdn2_simt": 6, "gdn2_decode": 7}
 
 _lib = None
 
@@ -57,6 +58,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_fwd_product.restype = i
         L.gdr_fwd_product.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, i,
                                       i, i, i, vp, sz, vp]
+        L.gdr_fwd_gdn2.restype = i
+        L.gdr_fwd_gdn2.argtypes = [vp] * 9 + [i] * 6 + [vp, i, i, i, vp]
+        L.gdr_decode_step_gdn2.restype = i
+        L.gdr_decode_step_gdn2.argtypes = [vp] * 8 + [i] * 6 + [vp]
         L.gdr_profile_enable.restype = None
         L.gdr_profile_enable.argtypes = [i]
         L.gdr_profile_read.restype = i
@@ -161,6 +166,45 @@ def gdr_fwd_product(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=No
     if st != GDR_OK:
         raise GdrError(st, "gdr_fwd_product")
     return out, S_final
+
+
+def gdr_fwd_gdn2(q, k, v, g, b, w, S0=None, *, chunk: int = 64, cu_seqlens=None, out=None,
+                 S_final=None, want_final: bool = True,
+                 stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Gated DeltaNet-2 prefill: erase gate b [B,T,H,d_k], write gate w
+    [B,T,H,d_v] (fp32); returns (out [B,T,H,d_v], S_final)."""
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    dtype = _dtype_code(q)
+    gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
+    n_seq = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+    _need_contig(q, k, v, g, b, w, S0, cu_seqlens)
+    if out is None:
+        out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
+    if S_final is None and want_final:
+        S_final = torch.empty((n_seq, H, d_v, d_k), dtype=torch.float32, device=q.device)
+    st = lib().gdr_fwd_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
+                            _ptr(out), _ptr(S_final), B, T, H, d_k, d_v, chunk, _ptr(cu_seqlens),
+                            n_seq, dtype, gate, _stream(stream))
+    if st != GDR_OK:
+        raise GdrError(st, "gdr_fwd_gdn2")
+    return out, S_final
+
+
+def gdr_decode_step_gdn2(q, k, v, g, b, w, S, *, out=None, stream=None) -> torch.Tensor:
+    """Gated DeltaNet-2 decode of one token per sequence, updating ``S`` in place."""
+    N, H, d_k = q.shape
+    d_v = v.shape[-1]
+    dtype = _dtype_code(q)
+    gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 3 else GDR_GATE_SCALAR
+    _need_contig(q, k, v, g, b, w, S)
+    if out is None:
+        out = torch.empty((N, H, d_v), dtype=q.dtype, device=q.device)
+    st = lib().gdr_decode_step_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S),
+                                    _ptr(out), N, H, d_k, d_v, dtype, gate, _stream(stream))
+    if st != GDR_OK:
+        raise GdrError(st, "gdr_decode_step_gdn2")
+    return out
 
 
 def gdr_decode_step(q, k, v, g, beta, S, *, out=None, stream=None) -> torch.Tensor:

@@ -11,6 +11,11 @@
 // So one warp owns a row at a time (32 lanes x d_k/32 floats, 128-bit loads),
 // reduces the two dot products with shuffles and writes the row back: the
 // state is read once and written once, which is the whole HBM cost of a step.
+//
+// With DEC (Gated DeltaNet-2, "Gated DeltaNet-2, and the gate that was doing
+// two jobs", section "What decoupling actually means here") the erase vector
+// e = b . k reads the row and the write gate scales the value:
+//     p_i = s_i . e,  u_i = w_i v_i - p_i,  s_i <- s_i + u_i k.
 #include "common.cuh"
 
 namespace gdr {
@@ -35,21 +40,23 @@ struct VecF<2> {
 constexpr int kDecodeThreads = 128;  // 4 warps, each owns d_v/4 rows of one head
 constexpr int kRowsInFlight = 8;     // rows a warp loads before using any
 
-template <typename Tin, int DK, bool CHANNEL>
+template <typename Tin, int DK, bool CHANNEL, bool DEC>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                    const float *__restrict__ g, const float *__restrict__ beta,
+                   const float *__restrict__ eg, const float *__restrict__ wg,
                    float *__restrict__ S, Tin *__restrict__ out, int dv) {
     constexpr int VEC = DK / 32;
     using V = VecF<VEC>;
     const size_t head = blockIdx.x;  // flattened (sequence, head)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    float kk[VEC], qq[VEC], aa[VEC];
+    float kk[VEC], qq[VEC], aa[VEC], ee[VEC];  // ee: the reading direction
 #pragma unroll
     for (int j = 0; j < VEC; ++j) {
         kk[j] = ld_in(k, head * DK + lane * VEC + j);
         qq[j] = ld_in(q, head * DK + lane * VEC + j);
+        ee[j] = DEC ? kk[j] * eg[head * DK + lane * VEC + j] : kk[j];
     }
     if (CHANNEL) {
 #pragma unroll
@@ -64,7 +71,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
     for (int j = 0; j < VEC; ++j) kq = fmaf(kk[j], qq[j], kq);
 #pragma unroll
     for (int off = 16; off; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-    const float b = beta[head];
+    const float b = DEC ? 1.f : beta[head];
 
     const int rpw = dv >> 2;  // rows per warp (dv is a multiple of 32)
     const int row0 = warp * rpw;
@@ -81,6 +88,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
             const int row = row0 + r0 + j;
             raw[j] = __ldcs(reinterpret_cast<const typename V::T *>(Sh + (size_t)row * DK) + lane);
             vi[j] = ld_in(vh, row);
+            if (DEC) vi[j] *= wg[head * (size_t)dv + row];
         }
 #pragma unroll
         for (int j = 0; j < kRowsInFlight; ++j) {
@@ -90,7 +98,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
                 s[e] *= aa[e];
-                p = fmaf(s[e], kk[e], p);
+                p = fmaf(s[e], ee[e], p);
                 r = fmaf(s[e], qq[e], r);
             }
 #pragma unroll
@@ -117,13 +125,14 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
 
 using namespace gdr;
 
-template <typename Tin, int DK, bool CH>
+template <typename Tin, int DK, bool CH, bool DEC = false>
 static cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, float *S, void *out, int N, int H, int dv,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, const float *eg = nullptr,
+                                 const float *wg = nullptr) {
     const unsigned int blocks = (unsigned int)((size_t)N * H);
-    decode_step_kernel<Tin, DK, CH><<<blocks, kDecodeThreads, 0, st>>>(
-        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, S, (Tin *)out, dv);
+    decode_step_kernel<Tin, DK, CH, DEC><<<blocks, kDecodeThreads, 0, st>>>(
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, eg, wg, S, (Tin *)out, dv);
     return cudaGetLastError();
 }
 
@@ -142,5 +151,24 @@ cudaError_t decode_dispatch(const void *q, const void *k, const void *v, const f
     if (dk == 128) GDR_DEC(float, 128);
     GDR_DEC(float, 64);
 #undef GDR_DEC
+}
+// Gated DeltaNet-2 step: erase gate eg [N, H, d_k], write gate wg [N, H, d_v].
+cudaError_t decode_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
+                                 const float *eg, const float *wg, float *S, void *out, int N,
+                                 int H, int dk, int dv, gdr_dtype dtype, gdr_gate gate,
+                                 cudaStream_t st) {
+    const bool ch = gate == GDR_GATE_PER_KEY_CHANNEL;
+#define GDR_DEC2(T, DK)                                                                          \
+    return ch ? launch_decode<T, DK, true, true>(q, k, v, g, nullptr, S, out, N, H, dv, st, eg,  \
+                                                 wg)                                             \
+              : launch_decode<T, DK, false, true>(q, k, v, g, nullptr, S, out, N, H, dv, st, eg, \
+                                                  wg)
+    if (dtype == GDR_BF16) {
+        if (dk == 128) GDR_DEC2(__nv_bfloat16, 128);
+        GDR_DEC2(__nv_bfloat16, 64);
+    }
+    if (dk == 128) GDR_DEC2(float, 128);
+    GDR_DEC2(float, 64);
+#undef GDR_DEC2
 }
 }  // namespace gdr_host

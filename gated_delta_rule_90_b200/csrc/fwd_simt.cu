@@ -20,6 +20,15 @@
 // of products.  A chunk that runs past the end of its sequence treats the
 // missing tokens as k = q = v = 0, beta = 0, g = 0, which leaves every valid
 // row unchanged (the pages assume the chunk size divides the length).
+//
+// With DEC (Gated DeltaNet-2, "Gated DeltaNet-2, and the gate that was doing
+// two jobs", section "What decoupling actually means here") beta splits into an
+// erase gate b (per key channel) and a write gate w (per value channel):
+// e = b . k, z = w . v.  The same chunk algorithm then reads
+//   L[l,m]  = sum_c e_lc k_mc exp(G_lc - G_mc)   (m < l),  (I + L) T = I,
+//   Z       = T (w . V - E<- S^T),   E<- = exp(G) . E,
+// and O, S as above: the erase vector replaces beta k on the reading side, the
+// key stays the writing direction.
 #include "common.cuh"
 
 namespace gdr {
@@ -33,14 +42,14 @@ struct SimtSmem {
     int kst;  // padded row stride of the [C][d_k] buffers
 };
 
-__host__ __device__ inline SimtSmem simt_layout(int C, int dk, bool channel) {
+__host__ __device__ inline SimtSmem simt_layout(int C, int dk, bool channel, bool dec) {
     SimtSmem L;
     L.kst = dk + 1;
     int o = 0;
     L.Kc = o; o += C * L.kst;
     L.Qc = o; o += C * L.kst;
     L.Gc = o; o += channel ? C * L.kst : C;
-    L.Kx = o; o += channel ? C * L.kst : 0;
+    L.Kx = o; o += (channel || dec) ? C * L.kst : 0;  // K<- / E<-, then K->
     L.bt = o; o += C;
     L.Nm = o; o += C * C;
     L.Am = o; o += C * C;
@@ -52,14 +61,15 @@ __host__ __device__ inline SimtSmem simt_layout(int C, int dk, bool channel) {
     return L;
 }
 
-template <typename Tin, bool CH>
+template <typename Tin, bool CH, bool DEC>
 __global__ void __launch_bounds__(kSimtThreads)
 fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                 const float *__restrict__ g, const float *__restrict__ beta,
+                const float *__restrict__ eg, const float *__restrict__ wg,
                 const float *__restrict__ S0, Tin *__restrict__ out, float *__restrict__ S_final,
                 int T, int H, int dk, int dv, int C, const int32_t *__restrict__ cu, int T_total) {
     extern __shared__ float sm[];
-    const SimtSmem L = simt_layout(C, dk, CH);
+    const SimtSmem L = simt_layout(C, dk, CH, DEC);
     float *Kc = sm + L.Kc, *Qc = sm + L.Qc, *Gc = sm + L.Gc, *Kx = sm + L.Kx, *bt = sm + L.bt;
     float *Nm = sm + L.Nm, *Am = sm + L.Am, *Tm = sm + L.Tm, *Pm = sm + L.Pm, *Zm = sm + L.Zm;
     float *Ss = sm + L.Ss;
@@ -93,10 +103,11 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             Kc[l * kst + c] = kv;
             Qc[l * kst + c] = qv;
             if (CH) Gc[l * kst + c] = (l < len) ? g[((size_t)(c0 + l) * H + h) * dk + c] : 0.f;
+            if (DEC) Kx[l * kst + c] = (l < len) ? kv * eg[((size_t)(c0 + l) * H + h) * dk + c] : 0.f;
         }
         for (int l = tid; l < C; l += kSimtThreads) {
             const size_t off = (size_t)(c0 + l) * H + h;
-            bt[l] = (l < len) ? beta[off] : 0.f;
+            bt[l] = (l < len) ? (DEC ? 1.f : beta[off]) : 0.f;
             if (!CH) Gc[l] = (l < len) ? g[off] : 0.f;
         }
         __syncthreads();
@@ -122,7 +133,8 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             const int l = p / C, m = p % C;
             float lv = 0.f, av = 0.f;
             if (m <= l) {
-                const float *kl = Kc + l * kst, *km = Kc + m * kst, *ql = Qc + l * kst;
+                // reading side: the key (beta applied below) or the erase vector
+                const float *kl = (DEC ? Kx : Kc) + l * kst, *km = Kc + m * kst, *ql = Qc + l * kst;
                 if (CH) {
                     const float *gl = Gc + l * kst, *gm = Gc + m * kst;
                     for (int c = 0; c < dk; ++c) {
@@ -152,12 +164,14 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                 Tm[i * C + j] = (i < j) ? 0.f : acc;
             }
         }
-        // decayed copies: Q<- in place; K<- into Kx (per channel) -- A and L are done
+        // decayed copies: Q<- in place; K<- into Kx (per channel), or E<- in
+        // place in Kx (erase vectors) -- A and L are done
         for (int e = tid; e < C * dk; e += kSimtThreads) {
             const int l = e / dk, c = e % dk;
             const float w = expf(CH ? Gc[l * kst + c] : Gc[l]);
             Qc[l * kst + c] *= w;
-            if (CH) Kx[l * kst + c] = Kc[l * kst + c] * w;
+            if (DEC) Kx[l * kst + c] *= w;
+            else if (CH) Kx[l * kst + c] = Kc[l * kst + c] * w;
         }
         __syncthreads();
         // ---- P = V - K<- S^T  (C x nr) ----
@@ -165,11 +179,12 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             const int l = e / kSimtRows, r = e % kSimtRows;
             float acc = 0.f;
             if (r < nr && l < len) {
-                const float *kl = CH ? Kx + l * kst : Kc + l * kst;
+                const float *kl = (CH || DEC) ? Kx + l * kst : Kc + l * kst;
                 const float *sr = Ss + r * kst;
                 for (int c = 0; c < dk; ++c) acc = fmaf(kl[c], sr[c], acc);
-                if (!CH) acc *= expf(Gc[l]);
-                acc = ld_in(v, ((size_t)(c0 + l) * H + h) * dv + r0 + r) - acc;
+                if (!CH && !DEC) acc *= expf(Gc[l]);
+                const size_t vo = ((size_t)(c0 + l) * H + h) * dv + r0 + r;
+                acc = (DEC ? ld_in(v, vo) * wg[vo] : ld_in(v, vo)) - acc;
             }
             Pm[e] = acc;
         }
@@ -232,24 +247,45 @@ using namespace gdr;
 
 namespace gdr_host {
 
-size_t simt_smem_bytes(int C, int dk, bool channel) {
-    return sizeof(float) * (size_t)simt_layout(C, dk, channel).total;
+size_t simt_smem_bytes(int C, int dk, bool channel, bool dec) {
+    return sizeof(float) * (size_t)simt_layout(C, dk, channel, dec).total;
 }
 
-template <typename Tin, bool CH>
+template <typename Tin, bool CH, bool DEC = false>
 static cudaError_t launch_simt(const void *q, const void *k, const void *v, const float *g,
                                const float *beta, const float *S0, void *out, float *S_final,
                                int T, int H, int dk, int dv, int C, const int32_t *cu, int n_seq,
-                               int T_total, cudaStream_t st) {
-    const size_t smem = simt_smem_bytes(C, dk, CH);
-    cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<Tin, CH>,
+                               int T_total, cudaStream_t st, const float *eg = nullptr,
+                               const float *wg = nullptr) {
+    const size_t smem = simt_smem_bytes(C, dk, CH, DEC);
+    cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<Tin, CH, DEC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(n_seq * H), (unsigned)((dv + kSimtRows - 1) / kSimtRows));
-    fwd_simt_kernel<Tin, CH><<<grid, kSimtThreads, smem, st>>>(
-        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, S0, (Tin *)out, S_final, T, H,
-        dk, dv, C, cu, T_total);
+    fwd_simt_kernel<Tin, CH, DEC><<<grid, kSimtThreads, smem, st>>>(
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, eg, wg, S0, (Tin *)out, S_final,
+        T, H, dk, dv, C, cu, T_total);
     return cudaGetLastError();
+}
+
+// Gated DeltaNet-2: erase gate eg [.., d_k], write gate wg [.., d_v] instead of beta.
+cudaError_t fwd_simt_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
+                                   const float *eg, const float *wg, const float *S0, void *out,
+                                   float *S_final, int T, int H, int dk, int dv, int C,
+                                   const int32_t *cu, int n_seq, int T_total, gdr_dtype dtype,
+                                   gdr_gate gate, cudaStream_t st) {
+    const bool ch = gate == GDR_GATE_PER_KEY_CHANNEL;
+    if (dtype == GDR_BF16)
+        return ch ? launch_simt<__nv_bfloat16, true, true>(q, k, v, g, nullptr, S0, out, S_final,
+                                                           T, H, dk, dv, C, cu, n_seq, T_total,
+                                                           st, eg, wg)
+                  : launch_simt<__nv_bfloat16, false, true>(q, k, v, g, nullptr, S0, out, S_final,
+                                                            T, H, dk, dv, C, cu, n_seq, T_total,
+                                                            st, eg, wg);
+    return ch ? launch_simt<float, true, true>(q, k, v, g, nullptr, S0, out, S_final, T, H, dk,
+                                               dv, C, cu, n_seq, T_total, st, eg, wg)
+              : launch_simt<float, false, true>(q, k, v, g, nullptr, S0, out, S_final, T, H, dk,
+                                                dv, C, cu, n_seq, T_total, st, eg, wg);
 }
 
 cudaError_t fwd_simt_dispatch(const void *q, const void *k, const void *v, const float *g,

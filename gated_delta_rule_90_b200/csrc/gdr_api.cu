@@ -18,7 +18,16 @@ cudaError_t fwd_simt_dispatch(const void *q, const void *k, const void *v, const
                               const float *beta, const float *S0, void *out, float *S_final,
                               int T, int H, int dk, int dv, int C, const int32_t *cu, int n_seq,
                               int T_total, gdr_dtype dtype, gdr_gate gate, cudaStream_t st);
-size_t simt_smem_bytes(int C, int dk, bool channel);
+size_t simt_smem_bytes(int C, int dk, bool channel, bool dec);
+cudaError_t fwd_simt_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
+                                   const float *eg, const float *wg, const float *S0, void *out,
+                                   float *S_final, int T, int H, int dk, int dv, int C,
+                                   const int32_t *cu, int n_seq, int T_total, gdr_dtype dtype,
+                                   gdr_gate gate, cudaStream_t st);
+cudaError_t decode_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
+                                 const float *eg, const float *wg, float *S, void *out, int N,
+                                 int H, int dk, int dv, gdr_dtype dtype, gdr_gate gate,
+                                 cudaStream_t st);
 // tensor-core path (fwd_tc.cu)
 bool tc_applies(int dk, int dv, int chunk, gdr_dtype dtype);
 size_t tc_workspace_bytes(int B, int T, int H, int n_seq, int varlen, gdr_gate gate);
@@ -189,8 +198,8 @@ gdr_status gdr_fwd(const void *q, const void *k, const void *v, const float *g, 
                                       nseq, gate, workspace, workspace_bytes,
                                       gdr_host::device_error_word(), s);
     } else {
-        if ((size_t)gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL) >
-            227u * 1024u)
+        if ((size_t)gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL,
+                                              false) > 227u * 1024u)
             return GDR_ERR_UNSUPPORTED;
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FWD_SIMT, s);
         e = gdr_host::fwd_simt_dispatch(q, k, v, g, beta, S0, out, S_final, T, H, d_k, d_v, chunk,
@@ -214,6 +223,52 @@ gdr_status gdr_decode_step(const void *q, const void *k, const void *v, const fl
     gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_DECODE, (cudaStream_t)stream);
     cudaError_t e = gdr_host::decode_dispatch(q, k, v, g, beta, S_inout, out, N, H, d_k, d_v,
                                               dtype, gate, (cudaStream_t)stream);
+    gdr_host::prof_end(tk, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+gdr_status gdr_fwd_gdn2(const void *q, const void *k, const void *v, const float *g,
+                        const float *b, const float *w, const float *S0, void *out,
+                        float *S_final, int B, int T, int H, int d_k, int d_v, int chunk,
+                        const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype, gdr_gate gate,
+                        void *stream) {
+    if ((long long)B * T > 0 && (!q || !k || !v || !g || !b || !w || !out)) return GDR_ERR_INVALID;
+    if (!valid_enum(dtype, gate)) return GDR_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(b) ||
+        !aligned16(w) || !aligned16(S0) || !aligned16(out) || !aligned16(S_final) ||
+        !aligned16(cu_seqlens))
+        return GDR_ERR_INVALID;
+    const bool varlen = cu_seqlens != nullptr;
+    gdr_status st = check_fwd_shapes(B, T, H, d_k, d_v, chunk, n_seq, varlen);
+    if (st != GDR_OK) return st;
+    if (!simt_shape_ok(d_k, d_v, chunk)) return GDR_ERR_UNSUPPORTED;
+    if (gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL, true) >
+        227u * 1024u)
+        return GDR_ERR_UNSUPPORTED;
+    cudaStream_t s = (cudaStream_t)stream;
+    gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_GDN2_SIMT, s);
+    cudaError_t e = gdr_host::fwd_simt_gdn2_dispatch(q, k, v, g, b, w, S0, out, S_final, T, H,
+                                                     d_k, d_v, chunk, cu_seqlens,
+                                                     varlen ? n_seq : B, B * T, dtype, gate, s);
+    gdr_host::prof_end(tk, s);
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, const float *g,
+                                const float *b, const float *w, float *S_inout, void *out, int N,
+                                int H, int d_k, int d_v, gdr_dtype dtype, gdr_gate gate,
+                                void *stream) {
+    if (!q || !k || !v || !g || !b || !w || !S_inout || !out) return GDR_ERR_INVALID;
+    if (!valid_enum(dtype, gate)) return GDR_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(b) ||
+        !aligned16(w) || !aligned16(S_inout) || !aligned16(out))
+        return GDR_ERR_INVALID;
+    if (N < 1 || H < 1 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID;
+    if ((double)N * H > 2.0e9) return GDR_ERR_INVALID;
+    if (!(d_k == 64 || d_k == 128) || d_v % 32 != 0 || d_v > 256) return GDR_ERR_UNSUPPORTED;
+    gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_GDN2_DECODE, (cudaStream_t)stream);
+    cudaError_t e = gdr_host::decode_gdn2_dispatch(q, k, v, g, b, w, S_inout, out, N, H, d_k, d_v,
+                                                   dtype, gate, (cudaStream_t)stream);
     gdr_host::prof_end(tk, (cudaStream_t)stream);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }

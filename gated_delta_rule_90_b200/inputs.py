@@ -57,6 +57,7 @@ class PrefillConfig:
     len_hi: int = 0
     seed_index: int = 0
     n_h: int = 1          # Householder substeps per token (> 1: Gated DeltaProduct)
+    variant: str = ""     # "gdn2": Gated DeltaNet-2 (erase and write gates instead of beta)
 
     @property
     def tokens(self) -> int:
@@ -96,7 +97,7 @@ PREFILL = {
     "gdp_prefill": PrefillConfig("gdp_prefill", 4, 2048, 16, 128, 128, 64, "bf16", "scalar", 0.1,
                                  0.01, seed_index=5, n_h=2),
     "gdn2_prefill": PrefillConfig("gdn2_prefill", 2, 4096, 16, 128, 128, 64, "bf16", "channel", 0.05,
-                                  0.0, seed_index=6),
+                                  0.0, seed_index=6, variant="gdn2"),
 }
 DECODE = {
     "decode": DecodeConfig("decode", 256, 32, 128, 128, "bf16", "scalar", 0.1, 0.1, 1000),

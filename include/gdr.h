@@ -175,6 +175,37 @@ gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const fl
                            gdr_path path, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Gated DeltaNet-2 ("Gated DeltaNet-2, and the gate that was doing two jobs",
+ * section "What decoupling actually means here"): the scalar step size splits
+ * into an erase gate b_t (one value per key channel) and a write gate w_t (one
+ * per value channel), e_t = b_t . k_t, z_t = w_t . v_t, and in the page's row
+ * convention S_t = (I - k_t e_t^T) D_t S_{t-1} + k_t z_t^T.  In this library's
+ * column convention (S is d_v x d_k):
+ *     S' = S D_t;  u = z_t - S' e_t;  S <- S' + u k_t^T;  o_t = S q_t.
+ * b = w = beta (broadcast) is gdr_fwd / gdr_decode_step.
+ *
+ * gdr_fwd_gdn2: the chunkwise prefill (that section's WY form: one triangular
+ * solve serves both right-hand sides) on the CUDA cores (fp32 arithmetic).
+ *  q, k     [B, T, H, d_k]   dtype;  v, out [B, T, H, d_v] dtype
+ *  g        [B, T, H] or [B, T, H, d_k]  fp32 log-decay
+ *  b        [B, T, H, d_k]   fp32 erase gate;  w [B, T, H, d_v] fp32 write gate
+ *  S0, S_final, cu_seqlens, n_seq, chunk: as for gdr_fwd (chunk 16, 32 or 64;
+ *  d_k, d_v multiples of 16 up to 128, else GDR_ERR_UNSUPPORTED).  No workspace.
+ * gdr_decode_step_gdn2: one token per sequence in place on S_inout, with
+ *  b [N, H, d_k] and w [N, H, d_v]; otherwise as gdr_decode_step.
+ * Pointers are caller-owned device memory, 16-byte aligned; errors as gdr_fwd.
+ */
+gdr_status gdr_fwd_gdn2(const void *q, const void *k, const void *v, const float *g,
+                        const float *b, const float *w, const float *S0, void *out,
+                        float *S_final, int B, int T, int H, int d_k, int d_v, int chunk,
+                        const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype, gdr_gate gate,
+                        void *stream);
+gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, const float *g,
+                                const float *b, const float *w, float *S_inout, void *out, int N,
+                                int H, int d_k, int d_v, gdr_dtype dtype, gdr_gate gate,
+                                void *stream);
+
+/*
  * gdr_fwd_noalloc -- the prefill for callers that cannot allocate device
  * memory at call time (their memory manager owns the whole device heap and
  * forbids further cudaMalloc, or an allocation's device synchronisation is not
@@ -205,7 +236,9 @@ size_t gdr_fwd_noalloc_scratch_bytes(void);
 /*
  * Per-kernel launch accounting and timing (a small built-in profiler).
  * Kernel ids: GDR_K_DECODE, GDR_K_FWD_SIMT, GDR_K_TC_PLAN, GDR_K_TC_WY,
- * GDR_K_TC_STATE, GDR_K_GDP_REMAP (the Gated DeltaProduct expand/gather).  Launches are always counted.  While timing is enabled,
+ * GDR_K_TC_STATE, GDR_K_GDP_REMAP (the Gated DeltaProduct expand/gather),
+ * GDR_K_GDN2_SIMT and GDR_K_GDN2_DECODE (Gated DeltaNet-2).  Launches are
+ * always counted.  While timing is enabled,
  * every launch is bracketed by two CUDA events recorded on the launch's own
  * stream.  gdr_profile_read waits for the recorded events, returns the
  * launches and the summed device time (ms) of kernel `id` since the last read
@@ -213,7 +246,8 @@ size_t gdr_fwd_noalloc_scratch_bytes(void);
  * from other host threads.
  */
 enum { GDR_K_DECODE = 0, GDR_K_FWD_SIMT = 1, GDR_K_TC_PLAN = 2, GDR_K_TC_WY = 3,
-       GDR_K_TC_STATE = 4, GDR_K_GDP_REMAP = 5, GDR_K_COUNT = 6 };
+       GDR_K_TC_STATE = 4, GDR_K_GDP_REMAP = 5, GDR_K_GDN2_SIMT = 6, GDR_K_GDN2_DECODE = 7,
+       GDR_K_COUNT = 8 };
 void gdr_profile_enable(int on);
 gdr_status gdr_profile_read(int id, long long *launches, double *total_ms);
 

@@ -127,3 +127,29 @@ def test_product_workspace_holds_the_virtual_sequence():
     assert inner > 0 and ws >= inner + 2 * B * T * nh * H * d * 2 + B * T * nh * H * 4
     assert binding.fwd_product_workspace_size(B, T, H, 0, d, d, 64, B, False, 1, 0, "auto") == 0
     assert lib.gdr_fwd_product_workspace_size is not None
+
+
+@nogpu
+@pytest.mark.parametrize("kw,expect", [
+    (dict(b=None), 1), (dict(dk=72), 2), (dict(chunk=128), 2), (dict(chunk=48), 1),
+    (dict(w=ctypes.c_void_p(0x10008)), 1), (dict(cu=P, B=2), 1), (dict(gate=3), 1),
+])
+def test_gdn2_fwd_rejects_on_host(kw, expect):
+    a = dict(q=P, k=P, v=P, g=P, b=P, w=P, S0=None, out=P, SF=P, B=2, T=64, H=2, dk=64, dv=64,
+             chunk=64, cu=None, n_seq=2, dtype=0, gate=1)
+    a.update(kw)
+    st = binding.lib().gdr_fwd_gdn2(a["q"], a["k"], a["v"], a["g"], a["b"], a["w"], a["S0"],
+                                    a["out"], a["SF"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                                    a["chunk"], a["cu"], a["n_seq"], a["dtype"], a["gate"], None)
+    assert st == expect
+
+
+@nogpu
+@pytest.mark.parametrize("kw,expect", [(dict(w=None), 1), (dict(dk=96), 2), (dict(N=0), 1)])
+def test_gdn2_decode_rejects_on_host(kw, expect):
+    a = dict(q=P, k=P, v=P, g=P, b=P, w=P, S=P, out=P, N=2, H=2, dk=128, dv=128, dtype=1, gate=1)
+    a.update(kw)
+    st = binding.lib().gdr_decode_step_gdn2(a["q"], a["k"], a["v"], a["g"], a["b"], a["w"],
+                                            a["S"], a["out"], a["N"], a["H"], a["dk"], a["dv"],
+                                            a["dtype"], a["gate"], None)
+    assert st == expect
