@@ -218,7 +218,8 @@ class PrefillRun:
         gate = 1 if cfg.gate == "channel" else 0
         dt = 1 if cfg.dtype == "bf16" else 0
         if self.gdn2:
-            ws = 0  # CUDA-core path, no workspace
+            ws = binding.fwd_gdn2_workspace_size(cfg.B, cfg.T, cfg.H, cfg.d_k, cfg.d_v, cfg.chunk,
+                                                 self.n_seq, self.cu is not None, dt, gate, path)
         elif cfg.n_h > 1:
             ws = binding.fwd_product_workspace_size(cfg.B, cfg.T, cfg.H, cfg.n_h, cfg.d_k,
                                                     cfg.d_v, cfg.chunk, self.n_seq,
@@ -231,7 +232,8 @@ class PrefillRun:
     def call(self, q, k, v, g, b, S0, cu, out=None, S_final=None):
         if self.gdn2:
             return binding.gdr_fwd_gdn2(q, k, v, g, b[0], b[1], S0, chunk=self.cfg.chunk,
-                                        cu_seqlens=cu, out=out, S_final=S_final)
+                                        cu_seqlens=cu, out=out, S_final=S_final, path=self.path,
+                                        workspace=self.ws)
         fn = binding.gdr_fwd_product if self.cfg.n_h > 1 else binding.gdr_fwd
         return fn(q, k, v, g, b, S0, chunk=self.cfg.chunk, cu_seqlens=cu, out=out,
                   S_final=S_final, path=self.path, workspace=self.ws)

@@ -59,7 +59,9 @@ def lib() -> ctypes.CDLL:
         L.gdr_fwd_product.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, i,
                                       i, i, i, vp, sz, vp]
         L.gdr_fwd_gdn2.restype = i
-        L.gdr_fwd_gdn2.argtypes = [vp] * 9 + [i] * 6 + [vp, i, i, i, vp]
+        L.gdr_fwd_gdn2.argtypes = [vp] * 9 + [i] * 6 + [vp, i, i, i, i, vp, sz, vp]
+        L.gdr_fwd_gdn2_workspace_size.restype = sz
+        L.gdr_fwd_gdn2_workspace_size.argtypes = [i] * 11
         L.gdr_decode_step_gdn2.restype = i
         L.gdr_decode_step_gdn2.argtypes = [vp] * 8 + [i] * 6 + [vp]
         L.gdr_profile_enable.restype = None
@@ -168,8 +170,14 @@ def gdr_fwd_product(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=No
     return out, S_final
 
 
+def fwd_gdn2_workspace_size(B, T, H, d_k, d_v, chunk, n_seq, varlen, dtype, gate,
+                            path="auto") -> int:
+    return int(lib().gdr_fwd_gdn2_workspace_size(B, T, H, d_k, d_v, chunk, n_seq,
+                                                 int(bool(varlen)), dtype, gate, PATHS[path]))
+
+
 def gdr_fwd_gdn2(q, k, v, g, b, w, S0=None, *, chunk: int = 64, cu_seqlens=None, out=None,
-                 S_final=None, want_final: bool = True,
+                 S_final=None, want_final: bool = True, path: str = "auto", workspace=None,
                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Gated DeltaNet-2 prefill: erase gate b [B,T,H,d_k], write gate w
     [B,T,H,d_v] (fp32); returns (out [B,T,H,d_v], S_final)."""
@@ -183,9 +191,15 @@ def gdr_fwd_gdn2(q, k, v, g, b, w, S0=None, *, chunk: int = 64, cu_seqlens=None,
         out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
     if S_final is None and want_final:
         S_final = torch.empty((n_seq, H, d_v, d_k), dtype=torch.float32, device=q.device)
+    ws_bytes = fwd_gdn2_workspace_size(B, T, H, d_k, d_v, chunk, n_seq, cu_seqlens is not None,
+                                       dtype, gate, path)
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    ws_avail = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().gdr_fwd_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
                             _ptr(out), _ptr(S_final), B, T, H, d_k, d_v, chunk, _ptr(cu_seqlens),
-                            n_seq, dtype, gate, _stream(stream))
+                            n_seq, dtype, gate, PATHS[path], _ptr(workspace), ws_avail,
+                            _stream(stream))
     if st != GDR_OK:
         raise GdrError(st, "gdr_fwd_gdn2")
     return out, S_final

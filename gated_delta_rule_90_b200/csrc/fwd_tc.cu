@@ -195,13 +195,19 @@ struct WySmem {
     static constexpr uint32_t small_bytes(bool ch) { return small_floats(ch) * 4 + 64; }
 };
 
-template <bool CH>
+// DEC (per-channel decay only): Gated DeltaNet-2's erase gate b and write gate
+// w replace beta ("Gated DeltaNet-2, and the gate that was doing two jobs",
+// section "What decoupling actually means here"): the Gram's reading rows are
+// e = b . k (so L = tril_-1(E K^T . Gamma) and W<- = T E<-), T solves
+// (I + L) T = I, and U = T (w . V).  The writing direction stays k (K->, A).
+template <bool CH, bool DEC = false>
 __global__ void __launch_bounds__(kWyThreads)
 wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
           const __grid_constant__ CUtensorMap tm_Ust,
           const __grid_constant__ CUtensorMap tm_Ast, const float *__restrict__ g,
-          const float *__restrict__ beta, const int32_t *__restrict__ cu, Geo geo, Ws ws,
+          const float *__restrict__ beta, const float *__restrict__ eg,
+          const float *__restrict__ wg, const int32_t *__restrict__ cu, Geo geo, Ws ws,
           unsigned int *err) {
     constexpr int NTS = WySmem::NTS, XST = WySmem::XST;
     extern __shared__ uint8_t smem_raw[];
@@ -265,7 +271,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     }
     // gates and beta (zero beyond the sequence end), cumulative log-decay G
     if (!CH && tid < C) sG[tid] = (tid < len) ? g[(size_t)(tstart + tid) * geo.H + h] : 0.f;
-    if (tid < C) sB[tid] = (tid < len) ? beta[(size_t)(tstart + tid) * geo.H + h] : 0.f;
+    if (tid < C) sB[tid] = (tid < len) ? (DEC ? 1.f : beta[(size_t)(tstart + tid) * geo.H + h]) : 0.f;
     __syncthreads();
     if (!CH && warp == 0) {
         float a = sG[lane], b = sG[lane + 32];
@@ -359,15 +365,31 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             unpack8(*reinterpret_cast<const uint4 *>(sKQ + off), kv);
             unpack8(*reinterpret_cast<const uint4 *>(sKQ + off + 8192), qv);
             if (CH) {
-                float kh[8], qh[8], kc[8], G8[8];
+                float kh[8], qh[8], kc[8], G8[8], b8[8];
                 ld8(sGt + l * D + c0, G8);
+                if (DEC) {  // erase gate of this row (reading side); write gate into V
+                    const size_t gro = ((size_t)(tstart + l) * geo.H + h) * D + c0;
+                    float w8[8], vv[8];
+                    if (l < len) {
+                        ld8(eg + gro, b8);
+                        ld8(wg + gro, w8);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) b8[i] = w8[i] = 0.f;
+                    }
+                    uint4 *vp = reinterpret_cast<uint4 *>(sV + a * 8192 + l * 128 + j * 16);
+                    unpack8(*vp, vv);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) vv[i] *= w8[i];
+                    *vp = pack8(vv);
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     // e^G = e^(G - R) e^R and e^(G_C - G) = e^(R - G) e^(G_C - R)
                     const float e1 = __expf(G8[i] - R8[i]), e2 = __expf(R8[i] - G8[i]);
                     wq[i] = qv[i] * (e1 * eR8[i]);
                     wk[i] = kv[i] * (e2 * eCR8[i]);
-                    kh[i] = kv[i] * e1;
+                    kh[i] = (DEC ? kv[i] * b8[i] : kv[i]) * e1;
                     qh[i] = qv[i] * e1;
                     kc[i] = kv[i] * e2;
                 }
@@ -1050,11 +1072,11 @@ size_t tc_workspace_bytes(int B, int T, int H, int n_seq, int varlen, gdr_gate) 
     return ws_layout(B, T, H, n_seq, varlen).total;
 }
 
-cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const float *g,
-                            const float *beta, const float *S0, void *out, float *S_final, int B,
-                            int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
-                            void *workspace, size_t ws_bytes, unsigned int *err,
-                            cudaStream_t st) {
+static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *eg, const float *wg,
+                               const float *S0, void *out, float *S_final, int B, int T, int H,
+                               const int32_t *cu, int n_seq, gdr_gate gate, void *workspace,
+                               size_t ws_bytes, unsigned int *err, cudaStream_t st) {
     const int varlen = cu != nullptr;
     const WsLayout L = ws_layout(B, T, H, n_seq, varlen);
     if (ws_bytes < L.total || !err) return cudaErrorInvalidValue;
@@ -1106,13 +1128,16 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
     const bool ch = gate == GDR_GATE_PER_KEY_CHANNEL;
     if (have_tokens && L.n_slots > 0) {
         const size_t smem = wy_smem_bytes(ch);
-        auto kern = ch ? wy_kernel<true> : wy_kernel<false>;
+        const bool dec = eg != nullptr;
+        if (dec && !ch) return cudaErrorInvalidValue;  // decoupled gates need the per-channel decay
+        auto kern = dec ? wy_kernel<true, true> : ch ? wy_kernel<true> : wy_kernel<false>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem)) != cudaSuccess)
             return e;
         dim3 grid((unsigned)L.n_slots, (unsigned)H);
         ProfToken tk = prof_begin(GDR_K_TC_WY, st);
-        kern<<<grid, kWyThreads, smem, st>>>(mq, mk, mv, mg, mU, mA, g, beta, cu, geo, ws, err);
+        kern<<<grid, kWyThreads, smem, st>>>(mq, mk, mv, mg, mU, mA, g, beta, eg, wg, cu, geo, ws,
+                                             err);
         prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -1128,6 +1153,26 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const float *S0, void *out, float *S_final, int B,
+                            int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
+                            void *workspace, size_t ws_bytes, unsigned int *err,
+                            cudaStream_t st) {
+    return tc_dispatch(q, k, v, g, beta, nullptr, nullptr, S0, out, S_final, B, T, H, cu, n_seq,
+                       gate, workspace, ws_bytes, err, st);
+}
+
+// Gated DeltaNet-2 (per-channel decay): erase gate eg [.., d_k], write gate wg [.., d_v].
+cudaError_t fwd_tc_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
+                                 const float *eg, const float *wg, const float *S0, void *out,
+                                 float *S_final, int B, int T, int H, const int32_t *cu, int n_seq,
+                                 void *workspace, size_t ws_bytes, unsigned int *err,
+                                 cudaStream_t st) {
+    if (!eg || !wg) return cudaErrorInvalidValue;
+    return tc_dispatch(q, k, v, g, nullptr, eg, wg, S0, out, S_final, B, T, H, cu, n_seq,
+                       GDR_GATE_PER_KEY_CHANNEL, workspace, ws_bytes, err, st);
 }
 
 }  // namespace gdr_host

@@ -24,6 +24,11 @@ cudaError_t fwd_simt_gdn2_dispatch(const void *q, const void *k, const void *v, 
                                    float *S_final, int T, int H, int dk, int dv, int C,
                                    const int32_t *cu, int n_seq, int T_total, gdr_dtype dtype,
                                    gdr_gate gate, cudaStream_t st);
+cudaError_t fwd_tc_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
+                                 const float *eg, const float *wg, const float *S0, void *out,
+                                 float *S_final, int B, int T, int H, const int32_t *cu, int n_seq,
+                                 void *workspace, size_t ws_bytes, unsigned int *err,
+                                 cudaStream_t st);
 cudaError_t decode_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
                                  const float *eg, const float *wg, float *S, void *out, int N,
                                  int H, int dk, int dv, gdr_dtype dtype, gdr_gate gate,
@@ -134,6 +139,23 @@ gdr_status resolve_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_path pat
     return GDR_OK;
 }
 
+// Gated DeltaNet-2 takes the tensor-core path only with the per-channel decay.
+gdr_status resolve_gdn2_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate gate,
+                             gdr_path path, bool *use_tc) {
+    const bool tc = gdr_host::tc_applies(dk, dv, chunk, dtype) && gate == GDR_GATE_PER_KEY_CHANNEL;
+    switch (path) {
+        case GDR_PATH_AUTO: *use_tc = tc; break;
+        case GDR_PATH_SIMT: *use_tc = false; break;
+        case GDR_PATH_TENSORCORE:
+            if (!tc) return GDR_ERR_UNSUPPORTED;
+            *use_tc = true;
+            break;
+        default: return GDR_ERR_INVALID;
+    }
+    if (!*use_tc && !simt_shape_ok(dk, dv, chunk)) return GDR_ERR_UNSUPPORTED;
+    return GDR_OK;
+}
+
 gdr_status check_fwd_shapes(int B, int T, int H, int dk, int dv, int chunk, int n_seq, bool varlen) {
     if (B < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return GDR_ERR_INVALID;
     if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return GDR_ERR_INVALID;
@@ -227,11 +249,21 @@ gdr_status gdr_decode_step(const void *q, const void *k, const void *v, const fl
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
+size_t gdr_fwd_gdn2_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk, int n_seq,
+                                   int varlen, gdr_dtype dtype, gdr_gate gate, gdr_path path) {
+    if (!valid_enum(dtype, gate)) return 0;
+    if (check_fwd_shapes(B, T, H, d_k, d_v, chunk, n_seq, varlen != 0) != GDR_OK) return 0;
+    bool use_tc = false;
+    if (resolve_gdn2_path(d_k, d_v, chunk, dtype, gate, path, &use_tc) != GDR_OK) return 0;
+    if (!use_tc) return 0;
+    return gdr_host::tc_workspace_bytes(B, T, H, n_seq, varlen, gate);
+}
+
 gdr_status gdr_fwd_gdn2(const void *q, const void *k, const void *v, const float *g,
                         const float *b, const float *w, const float *S0, void *out,
                         float *S_final, int B, int T, int H, int d_k, int d_v, int chunk,
                         const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype, gdr_gate gate,
-                        void *stream) {
+                        gdr_path path, void *workspace, size_t workspace_bytes, void *stream) {
     if ((long long)B * T > 0 && (!q || !k || !v || !g || !b || !w || !out)) return GDR_ERR_INVALID;
     if (!valid_enum(dtype, gate)) return GDR_ERR_INVALID;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(b) ||
@@ -241,16 +273,28 @@ gdr_status gdr_fwd_gdn2(const void *q, const void *k, const void *v, const float
     const bool varlen = cu_seqlens != nullptr;
     gdr_status st = check_fwd_shapes(B, T, H, d_k, d_v, chunk, n_seq, varlen);
     if (st != GDR_OK) return st;
-    if (!simt_shape_ok(d_k, d_v, chunk)) return GDR_ERR_UNSUPPORTED;
-    if (gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL, true) >
-        227u * 1024u)
-        return GDR_ERR_UNSUPPORTED;
+    bool use_tc = false;
+    st = resolve_gdn2_path(d_k, d_v, chunk, dtype, gate, path, &use_tc);
+    if (st != GDR_OK) return st;
+    const int nseq = varlen ? n_seq : B;
     cudaStream_t s = (cudaStream_t)stream;
-    gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_GDN2_SIMT, s);
-    cudaError_t e = gdr_host::fwd_simt_gdn2_dispatch(q, k, v, g, b, w, S0, out, S_final, T, H,
-                                                     d_k, d_v, chunk, cu_seqlens,
-                                                     varlen ? n_seq : B, B * T, dtype, gate, s);
-    gdr_host::prof_end(tk, s);
+    cudaError_t e;
+    if (use_tc) {  // the dispatcher accounts for its own launches
+        const size_t need = gdr_host::tc_workspace_bytes(B, T, H, n_seq, varlen, gate);
+        if (need && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
+            return GDR_ERR_INVALID;
+        e = gdr_host::fwd_tc_gdn2_dispatch(q, k, v, g, b, w, S0, out, S_final, B, T, H,
+                                           cu_seqlens, nseq, workspace, workspace_bytes,
+                                           gdr_host::device_error_word(), s);
+    } else {
+        if (gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL, true) >
+            227u * 1024u)
+            return GDR_ERR_UNSUPPORTED;
+        gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_GDN2_SIMT, s);
+        e = gdr_host::fwd_simt_gdn2_dispatch(q, k, v, g, b, w, S0, out, S_final, T, H, d_k, d_v,
+                                             chunk, cu_seqlens, nseq, B * T, dtype, gate, s);
+        gdr_host::prof_end(tk, s);
+    }
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -185,21 +185,26 @@ gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const fl
  * b = w = beta (broadcast) is gdr_fwd / gdr_decode_step.
  *
  * gdr_fwd_gdn2: the chunkwise prefill (that section's WY form: one triangular
- * solve serves both right-hand sides) on the CUDA cores (fp32 arithmetic).
+ * solve serves both right-hand sides).
  *  q, k     [B, T, H, d_k]   dtype;  v, out [B, T, H, d_v] dtype
  *  g        [B, T, H] or [B, T, H, d_k]  fp32 log-decay
  *  b        [B, T, H, d_k]   fp32 erase gate;  w [B, T, H, d_v] fp32 write gate
- *  S0, S_final, cu_seqlens, n_seq, chunk: as for gdr_fwd (chunk 16, 32 or 64;
- *  d_k, d_v multiples of 16 up to 128, else GDR_ERR_UNSUPPORTED).  No workspace.
+ *  S0, S_final, cu_seqlens, n_seq, chunk, path, workspace: as for gdr_fwd.  The
+ *  tensor-core path takes bf16 with d_k = d_v = 128, chunk 64 and the
+ *  per-channel decay (the page's setting); everything else (chunk 16, 32 or
+ *  64, d_k, d_v multiples of 16 up to 128) runs on the CUDA cores in fp32.
+ *  gdr_fwd_gdn2_workspace_size gives the workspace (0 on the CUDA-core path).
  * gdr_decode_step_gdn2: one token per sequence in place on S_inout, with
  *  b [N, H, d_k] and w [N, H, d_v]; otherwise as gdr_decode_step.
  * Pointers are caller-owned device memory, 16-byte aligned; errors as gdr_fwd.
  */
+size_t gdr_fwd_gdn2_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk, int n_seq,
+                                   int varlen, gdr_dtype dtype, gdr_gate gate, gdr_path path);
 gdr_status gdr_fwd_gdn2(const void *q, const void *k, const void *v, const float *g,
                         const float *b, const float *w, const float *S0, void *out,
                         float *S_final, int B, int T, int H, int d_k, int d_v, int chunk,
                         const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype, gdr_gate gate,
-                        void *stream);
+                        gdr_path path, void *workspace, size_t workspace_bytes, void *stream);
 gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, const float *g,
                                 const float *b, const float *w, float *S_inout, void *out, int N,
                                 int H, int d_k, int d_v, gdr_dtype dtype, gdr_gate gate,

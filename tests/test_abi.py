@@ -117,6 +117,14 @@ def test_product_rejects_on_host(kw, expect):
     assert product(**kw) == expect
 
 
+def test_gdn2_workspace_only_on_the_tensor_core_path():
+    assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 1, "auto") > 0
+    assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 0, "auto") == 0
+    assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 1, "simt") == 0
+    assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 1, "auto") == \
+        binding.fwd_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 1, "auto")
+
+
 def test_product_workspace_holds_the_virtual_sequence():
     """The product workspace covers q~, g~ and o~ for n_h T virtual steps plus
     the gated delta rule's own workspace for them."""
@@ -133,14 +141,16 @@ def test_product_workspace_holds_the_virtual_sequence():
 @pytest.mark.parametrize("kw,expect", [
     (dict(b=None), 1), (dict(dk=72), 2), (dict(chunk=128), 2), (dict(chunk=48), 1),
     (dict(w=ctypes.c_void_p(0x10008)), 1), (dict(cu=P, B=2), 1), (dict(gate=3), 1),
+    (dict(path=2), 2), (dict(dtype=1, dk=128, dv=128, path=2), 1), (dict(path=7), 1),
 ])
 def test_gdn2_fwd_rejects_on_host(kw, expect):
     a = dict(q=P, k=P, v=P, g=P, b=P, w=P, S0=None, out=P, SF=P, B=2, T=64, H=2, dk=64, dv=64,
-             chunk=64, cu=None, n_seq=2, dtype=0, gate=1)
+             chunk=64, cu=None, n_seq=2, dtype=0, gate=1, path=0, ws=None, ws_bytes=0)
     a.update(kw)
     st = binding.lib().gdr_fwd_gdn2(a["q"], a["k"], a["v"], a["g"], a["b"], a["w"], a["S0"],
                                     a["out"], a["SF"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
-                                    a["chunk"], a["cu"], a["n_seq"], a["dtype"], a["gate"], None)
+                                    a["chunk"], a["cu"], a["n_seq"], a["dtype"], a["gate"],
+                                    a["path"], a["ws"], a["ws_bytes"], None)
     assert st == expect
 
 

@@ -21,20 +21,21 @@ def cfg_of(**kw):
     return inputs.PREFILL["gdn2_prefill"].replace(**kw)
 
 
-def run_gpu(inp, dev, chunk=None):
+def run_gpu(inp, dev, chunk=None, path="auto"):
     c = inp.cfg
     q, k, v = (to_dev(x, c.dtype, dev) for x in (inp.q, inp.k, inp.v))
     g, b, w = (to_dev(x, "f32", dev) for x in (inp.g, inp.b, inp.w))
     S0 = to_dev(inp.S0, "f32", dev)
     cu = None if inp.cu_seqlens is None else torch.from_numpy(inp.cu_seqlens).to(dev)
-    out, SF = binding.gdr_fwd_gdn2(q, k, v, g, b, w, S0, chunk=chunk or c.chunk, cu_seqlens=cu)
+    out, SF = binding.gdr_fwd_gdn2(q, k, v, g, b, w, S0, chunk=chunk or c.chunk, cu_seqlens=cu,
+                                   path=path)
     torch.cuda.synchronize()
     assert binding.device_status() == binding.GDR_OK
     return to_np(out), to_np(SF)
 
 
-def check(inp, dev, chunk=None):
-    O, SF = run_gpu(inp, dev, chunk)
+def check(inp, dev, chunk=None, path="auto"):
+    O, SF = run_gpu(inp, dev, chunk, path)
     Or, SFr = oracle.gdn2_fwd(inp.q, inp.k, inp.v, inp.g, inp.b, inp.w, inp.S0, inp.cu_seqlens)
     eo, es = prefill_out_rel(O, Or, inp.cu_seqlens), state_rel(SF, SFr)
     tol = TOL[inp.cfg.dtype]
@@ -54,6 +55,42 @@ def test_gdn2_bf16_d128(cuda_device, gate):
     cfg = cfg_of(B=2, T=300, H=3, gate=gate, gate_scale=0.1 if gate == "scalar" else 0.05,
                  s0_var=0.01)
     check(inputs.gdn2_inputs(cfg, seed=602), cuda_device)
+
+
+@pytest.mark.parametrize("T", [64, 300, 1])
+def test_gdn2_tc_against_oracle(cuda_device, T):
+    """The tensor-core path (bf16, d = 128, C = 64, per-channel decay)."""
+    cfg = cfg_of(B=2, T=T, H=3, s0_var=0.01)
+    check(inputs.gdn2_inputs(cfg, seed=611), cuda_device, path="tc")
+
+
+def test_gdn2_tc_varlen_with_empty_and_unit_sequences(cuda_device):
+    cfg = cfg_of(B=1, T=600, H=2)
+    inp = inputs.gdn2_inputs(cfg, seed=612)
+    inp.cu_seqlens = np.array([0, 0, 1, 65, 129, 200, 200, 600], dtype=np.int32)
+    inp.S0 = np.random.default_rng(9).standard_normal((7, 2, 128, 128)).astype(np.float32) * 0.1
+    check(inp, cuda_device, path="tc")
+
+
+def test_gdn2_tc_matches_simt(cuda_device):
+    inp = inputs.gdn2_inputs(cfg_of(B=1, T=515, H=4, s0_var=0.01), seed=613)
+    O1, S1 = run_gpu(inp, cuda_device, path="tc")
+    O2, S2 = run_gpu(inp, cuda_device, path="simt")
+    assert prefill_out_rel(O1, O2) < 1e-2 and state_rel(S1, S2) < 1e-2
+
+
+def test_gdn2_tc_with_equal_gates_is_kda(cuda_device):
+    """b = w = beta on the tensor-core path against gdr_fwd's per-channel
+    (KDA) tensor-core path: the same maths through different roundings."""
+    cfg = inputs.PREFILL["kda_prefill"].replace(B=1, T=400, H=2, s0_var=0.01)
+    inp = inputs.prefill_inputs(cfg, seed=614)
+    dev = cuda_device
+    q, k, v = (to_dev(x, "bf16", dev) for x in (inp.q, inp.k, inp.v))
+    g, beta, S0 = (to_dev(x, "f32", dev) for x in (inp.g, inp.beta, inp.S0))
+    b = beta[..., None].expand(*beta.shape, 128).contiguous()
+    O1, S1 = binding.gdr_fwd_gdn2(q, k, v, g, b, b, S0, path="tc")
+    O2, S2 = binding.gdr_fwd(q, k, v, g, beta, S0, path="tc")
+    assert prefill_out_rel(to_np(O1), to_np(O2)) < 1e-2 and state_rel(to_np(S1), to_np(S2)) < 1e-2
 
 
 def test_gdn2_varlen_with_empty_and_unit_sequences(cuda_device):
