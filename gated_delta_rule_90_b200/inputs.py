@@ -17,6 +17,9 @@ varlen_prefill  16 packed sequences, sum T = 65536, lengths uniform in
 gdp_prefill     Gated DeltaProduct, n_h = 2 substeps per token: B=4, H=16,
                 T=2048 (4096 virtual steps), d=128, bf16, scalar gate,
                 S0 ~ N(0, 0.01)
+frame_prefill   implicit frame-level update: B=1, H=16, 16 frames of n=1024
+                tokens (T=16384), d=128, bf16, per-channel decay per frame,
+                writing strength gamma = (d_k / n) e^z, z ~ N(0, 1)
 gdn2_prefill    Gated DeltaNet-2 (erase gate b per key channel, write gate w
                 per value channel, b, w = sigmoid(N(0, 1))): B=2, H=16,
                 T=4096, d=128, bf16, per-channel decay, S0 = 0
@@ -272,6 +275,73 @@ def gdn2_inputs(cfg: PrefillConfig, seed: Optional[int] = None,
         cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     return Gdn2Inputs(cfg, round_to(q, cfg.dtype), round_to(k, cfg.dtype), round_to(v, cfg.dtype),
                       g, b, w, S0, cu)
+
+
+@dataclasses.dataclass(frozen=True)
+class FrameConfig:
+    name: str
+    B: int
+    T: int
+    H: int
+    d_k: int
+    d_v: int
+    n: int                # tokens per frame
+    dtype: str
+    gate: str             # "scalar" or "channel" (one decay per frame)
+    gate_scale: float
+    s0_var: float
+    seed_index: int = 7
+
+    @property
+    def frames(self) -> int:
+        return (self.T + self.n - 1) // self.n
+
+    def replace(self, **kw) -> "FrameConfig":
+        return dataclasses.replace(self, **kw)
+
+
+FRAME = {
+    "frame_prefill": FrameConfig("frame_prefill", 1, 16384, 16, 128, 128, 1024, "bf16", "channel",
+                                 0.05, 0.0),
+}
+
+
+@dataclasses.dataclass
+class FrameInputs:
+    cfg: FrameConfig
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    g: np.ndarray          # per frame [B, F, H] or [B, F, H, d_k]
+    gamma: np.ndarray      # per token [B, T, H]
+    S0: Optional[np.ndarray]
+
+
+def frame_inputs(cfg: FrameConfig, seed: Optional[int] = None,
+                 s0_var: Optional[float] = None) -> FrameInputs:
+    """Draw one batch for the implicit frame-level update.  Draw order: q, k, v,
+    writing-strength logits z, gate noise, S0.  gamma = (d_k / n) e^z: the
+    page's overall scale s = d_k / n, at which the old state and a frame take
+    about half each."""
+    if seed is None:
+        seed = BASE_SEED + cfg.seed_index
+    rng = np.random.default_rng(seed)
+    B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.d_k, cfg.d_v
+    f32 = np.float32
+    q = _l2_rows(rng.standard_normal((B, T, H, dk), dtype=f32))
+    k = _l2_rows(rng.standard_normal((B, T, H, dk), dtype=f32))
+    v = rng.standard_normal((B, T, H, dv), dtype=f32)
+    z = rng.standard_normal((B, T, H), dtype=f32)
+    gamma = (np.exp(z.astype(np.float64)) * (dk / cfg.n)).astype(f32)
+    F = cfg.frames
+    gshape = (B, F, H, dk) if cfg.gate == "channel" else (B, F, H)
+    g = (-_softplus(rng.standard_normal(gshape, dtype=f32)) * f32(cfg.gate_scale)).astype(f32)
+    var = cfg.s0_var if s0_var is None else s0_var
+    S0 = None
+    if var > 0:
+        S0 = (rng.standard_normal((B, H, dv, dk), dtype=f32) * f32(np.sqrt(var))).astype(f32)
+    return FrameInputs(cfg, round_to(q, cfg.dtype), round_to(k, cfg.dtype), round_to(v, cfg.dtype),
+                       g, gamma, S0)
 
 
 @dataclasses.dataclass

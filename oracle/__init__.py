@@ -20,6 +20,9 @@ Two independent fp64 CPU implementations live here:
   section "What decoupling actually means here"), and
   :func:`oracle.chunked.gdn2_chunked_fwd`, its chunkwise form from the same
   section, used only to pin it.
+* :func:`frame_fwd` -- the implicit frame-level update ("video-delta-rule",
+  section "A Different Route"): per frame of n tokens, Cholesky of I + G_t and
+  a solve of S_t (I + G_t) = S_{t-1} D_t + C_t.
 * :func:`oracle.chunked.chunked_fwd` -- the chunkwise WY/UT algorithm written
   from "Linear Attention, Visualized", sections "Gated DeltaNet (GDN) /
   Complete per-chunk algorithm" and "Kimi Delta Attention (KDA) / Complete
@@ -74,6 +77,8 @@ def _load():
             lib.oracle_gdn2_fwd.restype = ctypes.c_int
             lib.oracle_gdn2_fwd.argtypes = [dp] * 9 + [ctypes.c_int] * 5 + [ip, ctypes.c_int,
                                                                              ctypes.c_int]
+            lib.oracle_frame_fwd.restype = ctypes.c_int
+            lib.oracle_frame_fwd.argtypes = [dp] * 8 + [ctypes.c_int] * 7
             lib.oracle_gdr_decode_step.restype = ctypes.c_int
             lib.oracle_gdr_decode_step.argtypes = [dp, dp, dp, dp, dp, dp, dp,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -194,4 +199,23 @@ def gdn2_fwd(q, k, v, g, b, w, S0=None, cu_seqlens=None):
                                  1 if g.ndim == 4 else 0)
     if rc != 0:
         raise ValueError("oracle_gdn2_fwd rejected its arguments")
+    return out, S_final
+
+
+def frame_fwd(q, k, v, g, gamma, n, S0=None):
+    """Implicit frame-level update, fp64.  q, k ``[B,T,H,d_k]``; v ``[B,T,H,d_v]``;
+    gamma ``[B,T,H]`` (writing strength); g ``[B,F,H]`` or ``[B,F,H,d_k]`` with
+    F = ceil(T / n) (log-decay per frame).  Returns ``(O [B,T,H,d_v], S_final
+    [B,H,d_v,d_k])``."""
+    q, k, v, g, gamma = (_f64(x) for x in (q, k, v, g, gamma))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    S0a = None if S0 is None else _f64(S0)
+    out = np.zeros((B, T, H, dv))
+    S_final = np.zeros((B, H, dv, dk))
+    rc = _load().oracle_frame_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma), _ptr(S0a),
+                                  _ptr(out), _ptr(S_final), B, T, H, dk, dv, int(n),
+                                  1 if g.ndim == 4 else 0)
+    if rc != 0:
+        raise ValueError("oracle_frame_fwd rejected its arguments (%d)" % rc)
     return out, S_final

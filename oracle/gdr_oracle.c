@@ -333,3 +333,102 @@ int oracle_gdn2_fwd(const double *q, const double *k, const double *v, const dou
     free(u);
     return 0;
 }
+
+/*
+ * Implicit frame-level update ("video-delta-rule", sections "A First Attempt
+ * at Frame-Level Updates" and "A Different Route"): the tokens of a sequence
+ * are grouped into frames of n consecutive tokens (the last frame may be
+ * shorter); with the frame's erasure G_t = sum_i gamma_i k_i k_i^T and write
+ * C_t = sum_i gamma_i v_i k_i^T, the state takes one backward-Euler step
+ *     S_t (I + G_t) = S_{t-1} D_t + C_t
+ * (the frame's decay D_t first, as the forget gate at the frame boundary), and
+ * every query of frame t reads the same S_t: o_i = S_t q_i.  I + G_t is
+ * symmetric positive definite; it is factorised as L L^T (Cholesky) and each
+ * row of S_t solves x (L L^T) = b by forward then backward substitution.
+ *   q, k [B,T,H,dk]; v, out [B,T,H,dv]; gamma [B,T,H];
+ *   g [B,F,H] or [B,F,H,dk] with F = ceil(T / n) (log-decay per frame);
+ *   S0/S_final [B,H,dv,dk].
+ */
+int oracle_frame_fwd(const double *q, const double *k, const double *v, const double *g,
+                     const double *gamma, const double *S0, double *out, double *S_final, int B,
+                     int T, int H, int dk, int dv, int n, int per_channel) {
+    if (!q || !k || !v || !g || !gamma || !out || n < 1) return 1;
+    if (B <= 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return 1;
+    const int F = (T + n - 1) / n;
+    double *S = (double *)malloc(sizeof(double) * (size_t)dv * dk);
+    double *Bm = (double *)malloc(sizeof(double) * (size_t)dv * dk);
+    double *A = (double *)malloc(sizeof(double) * (size_t)dk * dk);
+    double *y = (double *)malloc(sizeof(double) * (size_t)dk);
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            const size_t soff = ((size_t)b * H + h) * (size_t)dv * dk;
+            if (S0) memcpy(S, S0 + soff, sizeof(double) * (size_t)dv * dk);
+            else memset(S, 0, sizeof(double) * (size_t)dv * dk);
+            for (int f = 0; f < F; ++f) {
+                const int t0 = f * n, t1 = (t0 + n < T) ? t0 + n : T;
+                const size_t fo = ((size_t)b * F + f) * H + h;
+                /* B = S D_t, A = I */
+                for (int i = 0; i < dv; ++i)
+                    for (int j = 0; j < dk; ++j) {
+                        const double a = per_channel ? exp(g[fo * dk + j]) : exp(g[fo]);
+                        Bm[(size_t)i * dk + j] = S[(size_t)i * dk + j] * a;
+                    }
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dk; ++j) A[(size_t)i * dk + j] = (i == j) ? 1.0 : 0.0;
+                /* A += gamma k k^T, B += gamma v k^T over the frame's tokens */
+                for (int t = t0; t < t1; ++t) {
+                    const size_t tok = ((size_t)b * T + t) * H + h;
+                    const double *kt = k + tok * dk, *vt = v + tok * dv, gm = gamma[tok];
+                    for (int i = 0; i < dk; ++i)
+                        for (int j = 0; j < dk; ++j) A[(size_t)i * dk + j] += gm * kt[i] * kt[j];
+                    for (int i = 0; i < dv; ++i)
+                        for (int j = 0; j < dk; ++j) Bm[(size_t)i * dk + j] += gm * vt[i] * kt[j];
+                }
+                /* Cholesky A = L L^T, L stored in the lower triangle of A */
+                for (int j = 0; j < dk; ++j) {
+                    double d = A[(size_t)j * dk + j];
+                    for (int m = 0; m < j; ++m) d -= A[(size_t)j * dk + m] * A[(size_t)j * dk + m];
+                    if (!(d > 0.0)) {
+                        free(S); free(Bm); free(A); free(y);
+                        return 2;
+                    }
+                    const double ljj = sqrt(d);
+                    A[(size_t)j * dk + j] = ljj;
+                    for (int i = j + 1; i < dk; ++i) {
+                        double s = A[(size_t)i * dk + j];
+                        for (int m = 0; m < j; ++m) s -= A[(size_t)i * dk + m] * A[(size_t)j * dk + m];
+                        A[(size_t)i * dk + j] = s / ljj;
+                    }
+                }
+                /* each row r of S_t: (L L^T) x = b_r^T (A is symmetric) */
+                for (int r = 0; r < dv; ++r) {
+                    const double *br = Bm + (size_t)r * dk;
+                    for (int i = 0; i < dk; ++i) {
+                        double s = br[i];
+                        for (int m = 0; m < i; ++m) s -= A[(size_t)i * dk + m] * y[m];
+                        y[i] = s / A[(size_t)i * dk + i];
+                    }
+                    double *xr = S + (size_t)r * dk;
+                    for (int i = dk - 1; i >= 0; --i) {
+                        double s = y[i];
+                        for (int m = i + 1; m < dk; ++m) s -= A[(size_t)m * dk + i] * xr[m];
+                        xr[i] = s / A[(size_t)i * dk + i];
+                    }
+                }
+                /* every query of the frame reads S_t */
+                for (int t = t0; t < t1; ++t) {
+                    const size_t tok = ((size_t)b * T + t) * H + h;
+                    const double *qt = q + tok * dk;
+                    for (int i = 0; i < dv; ++i) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * qt[j];
+                        out[tok * dv + i] = acc;
+                    }
+                }
+            }
+            if (S_final) memcpy(S_final + soff, S, sizeof(double) * (size_t)dv * dk);
+        }
+    }
+    free(S); free(Bm); free(A); free(y);
+    return 0;
+}
