@@ -21,7 +21,8 @@ GDR_F32, GDR_BF16 = 0, 1
 GDR_GATE_SCALAR, GDR_GATE_PER_KEY_CHANNEL = 0, 1
 PATHS = {"auto": 0, "simt": 1, "tc": 2}
 KERNELS = {"decode": 0, "fwd_simt": 1, "tc_plan": 2, "tc_wy": 3, "tc_state": 4, "gdp_remap": 5,
-           "gdn2_simt": 6, "gdn2_decode": 7}
+           "gdn2_simt": 6, "gdn2_decode": 7, "frame_gram": 8, "frame_solve": 9, "frame_chain": 10,
+           "frame_out": 11}
 
 _lib = None
 
@@ -64,6 +65,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_fwd_gdn2_workspace_size.argtypes = [i] * 11
         L.gdr_decode_step_gdn2.restype = i
         L.gdr_decode_step_gdn2.argtypes = [vp] * 8 + [i] * 6 + [vp]
+        L.gdr_fwd_frame_workspace_size.restype = sz
+        L.gdr_fwd_frame_workspace_size.argtypes = [i] * 6
+        L.gdr_fwd_frame.restype = i
+        L.gdr_fwd_frame.argtypes = [vp] * 8 + [i] * 8 + [vp, sz, vp]
         L.gdr_profile_enable.restype = None
         L.gdr_profile_enable.argtypes = [i]
         L.gdr_profile_read.restype = i
@@ -219,6 +224,36 @@ def gdr_decode_step_gdn2(q, k, v, g, b, w, S, *, out=None, stream=None) -> torch
     if st != GDR_OK:
         raise GdrError(st, "gdr_decode_step_gdn2")
     return out
+
+
+def fwd_frame_workspace_size(B, T, H, d_k, d_v, n) -> int:
+    return int(lib().gdr_fwd_frame_workspace_size(B, T, H, d_k, d_v, n))
+
+
+def gdr_fwd_frame(q, k, v, g, gamma, n: int, S0=None, *, out=None, S_final=None,
+                  want_final: bool = True, workspace=None,
+                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Implicit frame-level update: frames of n tokens, gamma [B,T,H], g per
+    frame [B,F,H] or [B,F,H,d_k]; returns (out [B,T,H,d_v], S_final [B,H,d_v,d_k])."""
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    dtype = _dtype_code(q)
+    gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
+    _need_contig(q, k, v, g, gamma, S0)
+    if out is None:
+        out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
+    if S_final is None and want_final:
+        S_final = torch.empty((B, H, d_v, d_k), dtype=torch.float32, device=q.device)
+    ws_bytes = fwd_frame_workspace_size(B, max(T, 1), H, d_k, d_v, n)
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    ws_avail = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdr_fwd_frame(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma), _ptr(S0), _ptr(out),
+                             _ptr(S_final), B, T, H, d_k, d_v, n, dtype, gate, _ptr(workspace),
+                             ws_avail, _stream(stream))
+    if st != GDR_OK:
+        raise GdrError(st, "gdr_fwd_frame")
+    return out, S_final
 
 
 def gdr_decode_step(q, k, v, g, beta, S, *, out=None, stream=None) -> torch.Tensor:

@@ -13,7 +13,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libgdr.so")
-SOURCES = ["gdr_api.cu", "decode.cu", "fwd_simt.cu", "fwd_tc.cu", "fwd_noalloc.cu", "product.cu"]
+SOURCES = ["gdr_api.cu", "decode.cu", "fwd_simt.cu", "fwd_tc.cu", "fwd_noalloc.cu", "product.cu",
+           "frame.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]

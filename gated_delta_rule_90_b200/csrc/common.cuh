@@ -10,7 +10,9 @@
 namespace gdr {
 
 // Device error word bits (see gdr_device_status).
-enum : unsigned int { kErrTimeout = 1u };
+// Bits of the device error word: a bounded wait expired; a factorisation met a
+// non-positive pivot (a negative writing strength, or NaN input).
+enum : unsigned int { kErrTimeout = 1u, kErrNumeric = 2u };
 
 // Token-storage loads/stores: fp32 or bf16, converted to/from fp32.
 __device__ __forceinline__ float ld_in(const float *p, size_t i) { return p[i]; }

@@ -1,0 +1,376 @@
+// Implicit frame-level update ("video-delta-rule", sections "A First Attempt at
+// Frame-Level Updates" and "A Different Route").
+//
+// The tokens of a sequence are grouped into frames of n consecutive tokens
+// (the last frame may be shorter).  Frame t has the erasure
+// G_t = K_t^T Gamma K_t and the write C_t = V_t^T Gamma K_t (Gamma = diag of
+// the tokens' writing strengths), and the state takes one implicit
+// (backward-Euler) step
+//     S_t (I + G_t) = S_{t-1} D_t + C_t,
+// with the frame's decay D_t applied first (the forget gate sits at frame
+// boundaries).  Every query of frame t reads S_t: o_i = S_t q_i.
+//
+// I + G_t is symmetric positive definite, so the page factorises it (Cholesky)
+// and solves.  The step is affine in S_{t-1}:
+//     S_t = S_{t-1} M_t + N_t,   M_t = D_t (I + G_t)^-1,   N_t = C_t (I + G_t)^-1,
+// and everything except the product chain over frames is independent per
+// frame.  Four passes:
+//   frame_gram   (frame, head, batch)    G_t, C_t                    fp32
+//   frame_affine (frame, head, batch)    Cholesky of I + G_t, then M_t, N_t by
+//                                        forward/backward substitution
+//   frame_chain  (batch*head, row block) S_t = S_{t-1} M_t + N_t over the frames
+//                                        (rows of S are independent)
+//   frame_out    (token tile, head, batch) o_i = S_t q_i
+// All arithmetic is fp32 on the CUDA cores.
+#include "common.cuh"
+
+namespace gdr {
+namespace frame {
+
+constexpr int kThreads = 256;
+constexpr int kTokTile = 32;   // tokens per smem tile in the Gram and output passes
+constexpr int kChainRows = 16; // state rows per CTA in the chain
+
+struct Dims {
+    int B, T, H, dk, dv, n, F;
+};
+
+__host__ __device__ inline size_t slot(const Dims &d, int b, int f, int h) {
+    return ((size_t)b * d.F + f) * d.H + h;
+}
+
+// G_t (d_k x d_k) then C_t (d_v x d_k): thread (ti, tj) owns an 8 x 8 block.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads)
+frame_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
+                  const float *__restrict__ gamma, float *__restrict__ Gw, float *__restrict__ Cw,
+                  Dims d) {
+    extern __shared__ float sm[];
+    const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int kst = d.dk + 1, vst = d.dv + 1;
+    float *Ks = sm, *Vs = Ks + kTokTile * kst, *gs = Vs + kTokTile * vst;
+    const int tid = threadIdx.x, ti = tid >> 4, tj = tid & 15;
+    const int t0 = f * d.n, t1 = min(d.T, t0 + d.n);
+    const size_t sl = slot(d, b, f, h);
+    for (int pass = 0; pass < 2; ++pass) {  // 0: G = K^T Gamma K, 1: C = V^T Gamma K
+        const int rows = pass ? d.dv : d.dk;
+        float acc[8][8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
+        for (int tt = t0; tt < t1; tt += kTokTile) {
+            const int cnt = min(kTokTile, t1 - tt);
+            __syncthreads();
+            for (int e = tid; e < kTokTile * d.dk; e += kThreads) {
+                const int r = e / d.dk, c = e % d.dk;
+                Ks[r * kst + c] = (r < cnt) ? ld_in(k, (((size_t)b * d.T + tt + r) * d.H + h) * d.dk + c) : 0.f;
+            }
+            if (pass)
+                for (int e = tid; e < kTokTile * d.dv; e += kThreads) {
+                    const int r = e / d.dv, c = e % d.dv;
+                    Vs[r * vst + c] = (r < cnt) ? ld_in(v, (((size_t)b * d.T + tt + r) * d.H + h) * d.dv + c) : 0.f;
+                }
+            if (tid < kTokTile) gs[tid] = (tid < cnt) ? gamma[((size_t)b * d.T + tt + tid) * d.H + h] : 0.f;
+            __syncthreads();
+            if (ti * 8 < rows && tj * 8 < d.dk) {
+                const float *Ls = pass ? Vs : Ks;
+                const int lst = pass ? vst : kst;
+                for (int r = 0; r < cnt; ++r) {
+                    float x[8], y[8];
+                    const float gr = gs[r];
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) x[a] = gr * Ls[r * lst + ti * 8 + a];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) y[c] = Ks[r * kst + tj * 8 + c];
+#pragma unroll
+                    for (int a = 0; a < 8; ++a)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(x[a], y[c], acc[a][c]);
+                }
+            }
+        }
+        if (ti * 8 < rows && tj * 8 < d.dk) {
+            float *dst = (pass ? Cw + sl * (size_t)d.dv * d.dk : Gw + sl * (size_t)d.dk * d.dk);
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) dst[(size_t)(ti * 8 + a) * d.dk + tj * 8 + c] = acc[a][c];
+        }
+    }
+}
+
+// Cholesky of I + G_t (right-looking, in shared memory), then the rows of
+// M_t = D_t (I + G_t)^-1 and N_t = C_t (I + G_t)^-1 by substitution: row x of
+// either solves x (L L^T) = r, i.e. L y = r^T, L^T x^T = y, one row per thread.
+// M_t overwrites G_t and N_t overwrites C_t in the workspace.
+__global__ void __launch_bounds__(kThreads)
+frame_affine_kernel(float *__restrict__ GM, float *__restrict__ CN, const float *__restrict__ g,
+                    int per_channel, Dims d, unsigned int *err) {
+    extern __shared__ float sm[];
+    const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int dk = d.dk, ast = dk + 1;
+    float *A = sm, *R = A + dk * ast;  // R: (dk + dv) rows of length dk (+1 pad)
+    const int tid = threadIdx.x;
+    const size_t sl = slot(d, b, f, h);
+    float *Gp = GM + sl * (size_t)dk * dk, *Cp = CN + sl * (size_t)d.dv * dk;
+    for (int e = tid; e < dk * dk; e += kThreads) {
+        const int i = e / dk, j = e % dk;
+        A[i * ast + j] = Gp[e] + (i == j ? 1.f : 0.f);
+    }
+    // right-hand sides: rows of D_t, then rows of C_t
+    for (int e = tid; e < dk * dk; e += kThreads) {
+        const int i = e / dk, j = e % dk;
+        const float a = per_channel ? __expf(g[sl * dk + i]) : __expf(g[sl]);
+        R[i * ast + j] = (i == j) ? a : 0.f;
+    }
+    for (int e = tid; e < d.dv * dk; e += kThreads) {
+        const int i = e / dk, j = e % dk;
+        R[(dk + i) * ast + j] = Cp[e];
+    }
+    __syncthreads();
+    // right-looking Cholesky: column j, then the trailing update
+    for (int j = 0; j < dk; ++j) {
+        const float ajj = A[j * ast + j];
+        const float ljj = sqrtf(fmaxf(ajj, 1e-30f));
+        __syncthreads();
+        if (tid == 0) {
+            if (!(ajj > 0.f)) atomicOr(err, kErrNumeric);
+            A[j * ast + j] = ljj;
+        }
+        for (int i = j + 1 + tid; i < dk; i += kThreads) A[i * ast + j] /= ljj;
+        __syncthreads();
+        const int m = dk - j - 1;  // trailing block (j+1.., j+1..), lower triangle
+        for (int e = tid; e < m * m; e += kThreads) {
+            const int i = j + 1 + e / m, c = j + 1 + e % m;
+            if (c <= i) A[i * ast + c] -= A[i * ast + j] * A[c * ast + j];
+        }
+        __syncthreads();
+    }
+    // substitution, one right-hand side row per thread
+    for (int r = tid; r < dk + d.dv; r += kThreads) {
+        float *x = R + r * ast;
+        for (int i = 0; i < dk; ++i) {  // L y = r
+            float s = x[i];
+            for (int m2 = 0; m2 < i; ++m2) s = fmaf(-A[i * ast + m2], x[m2], s);
+            x[i] = s / A[i * ast + i];
+        }
+        for (int i = dk - 1; i >= 0; --i) {  // L^T x = y
+            float s = x[i];
+            for (int m2 = i + 1; m2 < dk; ++m2) s = fmaf(-A[m2 * ast + i], x[m2], s);
+            x[i] = s / A[i * ast + i];
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < dk * dk; e += kThreads) Gp[e] = R[(e / dk) * ast + e % dk];
+    for (int e = tid; e < d.dv * dk; e += kThreads) Cp[e] = R[(dk + e / dk) * ast + e % dk];
+}
+
+// S_t = S_{t-1} M_t + N_t for kChainRows rows of S; every S_t is stored for
+// the output pass, the last one also as S_final.
+__global__ void __launch_bounds__(kThreads)
+frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Nw,
+                   const float *__restrict__ S0, float *__restrict__ Sw,
+                   float *__restrict__ S_final, Dims d) {
+    extern __shared__ float sm[];
+    const int bh = blockIdx.x, b = bh / d.H, h = bh % d.H;
+    const int r0 = blockIdx.y * kChainRows;
+    const int nr = min(kChainRows, d.dv - r0);
+    const int dk = d.dk, ast = dk + 1;
+    float *M = sm, *S = M + dk * ast, *Sn = S + kChainRows * ast;
+    const int tid = threadIdx.x;
+    const size_t soff = ((size_t)b * d.H + h) * (size_t)d.dv * dk;
+    for (int e = tid; e < kChainRows * dk; e += kThreads) {
+        const int r = e / dk, c = e % dk;
+        S[r * ast + c] = (S0 && r < nr) ? S0[soff + (size_t)(r0 + r) * dk + c] : 0.f;
+    }
+    for (int f = 0; f < d.F; ++f) {
+        const size_t sl = slot(d, b, f, h);
+        __syncthreads();
+        for (int e = tid; e < dk * dk; e += kThreads) M[(e / dk) * ast + e % dk] = Mw[sl * (size_t)dk * dk + e];
+        __syncthreads();
+        for (int e = tid; e < nr * dk; e += kThreads) {
+            const int r = e / dk, c = e % dk;
+            float acc = Nw[sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c];
+            for (int m = 0; m < dk; ++m) acc = fmaf(S[r * ast + m], M[m * ast + c], acc);
+            Sn[r * ast + c] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < nr * dk; e += kThreads) {
+            const int r = e / dk, c = e % dk;
+            const float x = Sn[r * ast + c];
+            S[r * ast + c] = x;
+            Sw[sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c] = x;
+        }
+    }
+    __syncthreads();
+    if (S_final)
+        for (int e = tid; e < nr * dk; e += kThreads) {
+            const int r = e / dk, c = e % dk;
+            S_final[soff + (size_t)(r0 + r) * dk + c] = S[r * ast + c];
+        }
+}
+
+// o_i = S_t q_i for a tile of kTokTile tokens inside one frame.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads)
+frame_out_kernel(const Tin *__restrict__ q, const float *__restrict__ Sw, Tin *__restrict__ out,
+                 Dims d) {
+    extern __shared__ float sm[];
+    const int tiles_per_frame = (d.n + kTokTile - 1) / kTokTile;
+    const int f = blockIdx.x / tiles_per_frame, tile = blockIdx.x % tiles_per_frame;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int tt = f * d.n + tile * kTokTile;
+    const int cnt = min(kTokTile, min(d.T, (f + 1) * d.n) - tt);
+    if (cnt <= 0) return;  // whole CTA, before any barrier
+    const int dk = d.dk, ast = dk + 1;
+    float *Ss = sm, *Qs = Ss + d.dv * ast;
+    const int tid = threadIdx.x;
+    const size_t sl = slot(d, b, f, h);
+    for (int e = tid; e < d.dv * dk; e += kThreads) Ss[(e / dk) * ast + e % dk] = Sw[sl * (size_t)d.dv * dk + e];
+    for (int e = tid; e < kTokTile * dk; e += kThreads) {
+        const int r = e / dk, c = e % dk;
+        Qs[r * ast + c] = (r < cnt) ? ld_in(q, (((size_t)b * d.T + tt + r) * d.H + h) * dk + c) : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < cnt * d.dv; e += kThreads) {
+        const int r = e / d.dv, i = e % d.dv;
+        float acc = 0.f;
+        for (int m = 0; m < dk; ++m) acc = fmaf(Ss[i * ast + m], Qs[r * ast + m], acc);
+        st_out(out, (((size_t)b * d.T + tt + r) * d.H + h) * d.dv + i, acc);
+    }
+}
+
+}  // namespace frame
+}  // namespace gdr
+
+using namespace gdr;
+using namespace gdr::frame;
+
+namespace {
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct FrameLayout {
+    size_t GM, CN, Sw, total;
+};
+
+FrameLayout frame_layout(int B, int T, int H, int dk, int dv, int n) {
+    FrameLayout L;
+    const size_t slots = (size_t)B * ((T + n - 1) / n) * H;
+    size_t o = 0;
+    L.GM = o; o += up256(slots * dk * dk * 4);
+    L.CN = o; o += up256(slots * (size_t)dv * dk * 4);
+    L.Sw = o; o += up256(slots * (size_t)dv * dk * 4);
+    L.total = o;
+    return L;
+}
+
+bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
+
+bool frame_shape_ok(int dk, int dv) {
+    return dk >= 16 && dk <= 128 && dk % 8 == 0 && dv >= 8 && dv <= 128 && dv % 8 == 0;
+}
+
+size_t affine_smem(int dk, int dv) { return sizeof(float) * (size_t)(dk + dk + dv) * (dk + 1); }
+
+template <typename Tin>
+cudaError_t frame_launch(const void *q, const void *k, const void *v, const float *g,
+                         const float *gamma, const float *S0, void *out, float *S_final,
+                         const Dims &d, int per_channel, uint8_t *ws, cudaStream_t st,
+                         unsigned int *err) {
+    const FrameLayout L = frame_layout(d.B, d.T, d.H, d.dk, d.dv, d.n);
+    float *GM = (float *)(ws + L.GM), *CN = (float *)(ws + L.CN), *Sw = (float *)(ws + L.Sw);
+    cudaError_t e;
+    const size_t sm_gram = sizeof(float) * (size_t)(kTokTile * (d.dk + 1) + kTokTile * (d.dv + 1) + kTokTile);
+    const size_t sm_aff = affine_smem(d.dk, d.dv);
+    const size_t sm_chain = sizeof(float) * (size_t)(d.dk + 2 * kChainRows) * (d.dk + 1);
+    const size_t sm_out = sizeof(float) * (size_t)(d.dv + kTokTile) * (d.dk + 1);
+    if ((e = cudaFuncSetAttribute(frame_gram_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gram)) ||
+        (e = cudaFuncSetAttribute(frame_affine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_aff)) ||
+        (e = cudaFuncSetAttribute(frame_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_chain)) ||
+        (e = cudaFuncSetAttribute(frame_out_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out)))
+        return e;
+    const dim3 gf((unsigned)d.F, (unsigned)d.H, (unsigned)d.B);
+    {
+        gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_GRAM, st);
+        frame_gram_kernel<Tin><<<gf, kThreads, sm_gram, st>>>((const Tin *)k, (const Tin *)v, gamma, GM, CN, d);
+        gdr_host::prof_end(tk, st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_SOLVE, st);
+        frame_affine_kernel<<<gf, kThreads, sm_aff, st>>>(GM, CN, g, per_channel, d, err);
+        gdr_host::prof_end(tk, st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_CHAIN, st);
+        const dim3 gc((unsigned)(d.B * d.H), (unsigned)((d.dv + kChainRows - 1) / kChainRows));
+        frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, S0, Sw, S_final, d);
+        gdr_host::prof_end(tk, st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_OUT, st);
+        const int tiles = (d.n + kTokTile - 1) / kTokTile;
+        const dim3 go((unsigned)(d.F * tiles), (unsigned)d.H, (unsigned)d.B);
+        frame_out_kernel<Tin><<<go, kThreads, sm_out, st>>>((const Tin *)q, Sw, (Tin *)out, d);
+        gdr_host::prof_end(tk, st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdr_fwd_frame_workspace_size(int B, int T, int H, int d_k, int d_v, int n) {
+    if (B < 1 || T < 1 || H < 1 || n < 1 || !frame_shape_ok(d_k, d_v)) return 0;
+    return frame_layout(B, T, H, d_k, d_v, n).total;
+}
+
+gdr_status gdr_fwd_frame(const void *q, const void *k, const void *v, const float *g,
+                         const float *gamma, const float *S0, void *out, float *S_final, int B,
+                         int T, int H, int d_k, int d_v, int n, gdr_dtype dtype, gdr_gate gate,
+                         void *workspace, size_t workspace_bytes, void *stream) {
+    if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || n < 1) return GDR_ERR_INVALID;
+    if (!(dtype == GDR_F32 || dtype == GDR_BF16) ||
+        !(gate == GDR_GATE_SCALAR || gate == GDR_GATE_PER_KEY_CHANNEL))
+        return GDR_ERR_INVALID;
+    if (!frame_shape_ok(d_k, d_v)) return GDR_ERR_UNSUPPORTED;
+    if ((double)B * T * H * (d_k > d_v ? d_k : d_v) > 9.0e15 || (double)B * T > 2.0e9 ||
+        (double)B * H * ((T + n - 1) / n) > 2.0e9)
+        return GDR_ERR_INVALID;
+    if (affine_smem(d_k, d_v) > 227u * 1024u) return GDR_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535) return GDR_ERR_UNSUPPORTED;  // grid y / z extents
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(gamma) ||
+        !aligned16(S0) || !aligned16(out) || !aligned16(S_final) || !aligned16(workspace))
+        return GDR_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (T == 0) {  // no frames: the state passes through
+        if (S_final && S0 != S_final) {
+            const size_t bytes = sizeof(float) * (size_t)B * H * d_v * d_k;
+            cudaError_t e = S0 ? cudaMemcpyAsync(S_final, S0, bytes, cudaMemcpyDeviceToDevice, st)
+                               : cudaMemsetAsync(S_final, 0, bytes, st);
+            return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+        }
+        return GDR_OK;
+    }
+    if (!q || !k || !v || !g || !gamma || !out) return GDR_ERR_INVALID;
+    const FrameLayout L = frame_layout(B, T, H, d_k, d_v, n);
+    if (!workspace || workspace_bytes < L.total) return GDR_ERR_INVALID;
+    Dims d{B, T, H, d_k, d_v, n, (T + n - 1) / n};
+    unsigned int *err = gdr_host::device_error_word();
+    if (!err) return GDR_ERR_CUDA;
+    const int ch = gate == GDR_GATE_PER_KEY_CHANNEL;
+    cudaError_t e = dtype == GDR_BF16
+                        ? frame_launch<__nv_bfloat16>(q, k, v, g, gamma, S0, out, S_final, d, ch,
+                                                      (uint8_t *)workspace, st, err)
+                        : frame_launch<float>(q, k, v, g, gamma, S0, out, S_final, d, ch,
+                                              (uint8_t *)workspace, st, err);
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+}  // extern "C"

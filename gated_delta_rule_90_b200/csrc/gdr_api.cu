@@ -343,7 +343,8 @@ gdr_status gdr_device_status(void *stream) {
         return GDR_ERR_CUDA;
     if (word && cudaMemcpyToSymbol(g_gdr_device_error, &zero, sizeof(zero)) != cudaSuccess)
         return GDR_ERR_CUDA;
-    return (word & gdr::kErrTimeout) ? GDR_ERR_TIMEOUT : GDR_OK;
+    if (word & gdr::kErrTimeout) return GDR_ERR_TIMEOUT;
+    return (word & gdr::kErrNumeric) ? GDR_ERR_INVALID : GDR_OK;
 }
 
 void gdr_profile_enable(int on) {

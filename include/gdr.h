@@ -211,6 +211,34 @@ gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, con
                                 void *stream);
 
 /*
+ * Implicit frame-level update ("video-delta-rule", sections "A First Attempt
+ * at Frame-Level Updates" and "A Different Route").  The tokens of each
+ * sequence form frames of n consecutive tokens (the last may be shorter).
+ * Frame t has the erasure G_t = sum_i gamma_i k_i k_i^T and the write
+ * C_t = sum_i gamma_i v_i k_i^T over its tokens, and the state takes the
+ * backward-Euler step
+ *     S_t (I + G_t) = S_{t-1} D_t + C_t
+ * (D_t = the frame's decay, applied first); every query of frame t reads S_t:
+ * o_i = S_t q_i.  I + G_t is factorised by Cholesky; n = 1 is the gated delta
+ * rule with step size gamma / (1 + gamma).
+ *  q, k     [B, T, H, d_k]  dtype;  v, out [B, T, H, d_v]  dtype
+ *  gamma    [B, T, H]       fp32 writing strength, >= 0 (a negative value can
+ *                           make I + G_t indefinite: gdr_device_status then
+ *                           reports GDR_ERR_INVALID)
+ *  g        [B, F, H] or [B, F, H, d_k] fp32 log-decay per frame, F = ceil(T / n)
+ *  S0       [B, H, d_v, d_k] fp32 or NULL (zero);  S_final likewise or NULL
+ *  d_k a multiple of 8 in [16, 128]; d_v a multiple of 8 in [8, 128]
+ *  workspace: gdr_fwd_frame_workspace_size(B, T, H, d_k, d_v, n) bytes,
+ *           caller-owned device memory (per frame: G/M_t, C/N_t and S_t, fp32).
+ * fp32 arithmetic on the CUDA cores.  Errors as gdr_fwd.
+ */
+size_t gdr_fwd_frame_workspace_size(int B, int T, int H, int d_k, int d_v, int n);
+gdr_status gdr_fwd_frame(const void *q, const void *k, const void *v, const float *g,
+                         const float *gamma, const float *S0, void *out, float *S_final, int B,
+                         int T, int H, int d_k, int d_v, int n, gdr_dtype dtype, gdr_gate gate,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * gdr_fwd_noalloc -- the prefill for callers that cannot allocate device
  * memory at call time (their memory manager owns the whole device heap and
  * forbids further cudaMalloc, or an allocation's device synchronisation is not
@@ -242,8 +270,9 @@ size_t gdr_fwd_noalloc_scratch_bytes(void);
  * Per-kernel launch accounting and timing (a small built-in profiler).
  * Kernel ids: GDR_K_DECODE, GDR_K_FWD_SIMT, GDR_K_TC_PLAN, GDR_K_TC_WY,
  * GDR_K_TC_STATE, GDR_K_GDP_REMAP (the Gated DeltaProduct expand/gather),
- * GDR_K_GDN2_SIMT and GDR_K_GDN2_DECODE (Gated DeltaNet-2).  Launches are
- * always counted.  While timing is enabled,
+ * GDR_K_GDN2_SIMT and GDR_K_GDN2_DECODE (Gated DeltaNet-2), GDR_K_FRAME_GRAM,
+ * GDR_K_FRAME_SOLVE, GDR_K_FRAME_CHAIN and GDR_K_FRAME_OUT (the implicit frame
+ * update's passes).  Launches are always counted.  While timing is enabled,
  * every launch is bracketed by two CUDA events recorded on the launch's own
  * stream.  gdr_profile_read waits for the recorded events, returns the
  * launches and the summed device time (ms) of kernel `id` since the last read
@@ -252,7 +281,8 @@ size_t gdr_fwd_noalloc_scratch_bytes(void);
  */
 enum { GDR_K_DECODE = 0, GDR_K_FWD_SIMT = 1, GDR_K_TC_PLAN = 2, GDR_K_TC_WY = 3,
        GDR_K_TC_STATE = 4, GDR_K_GDP_REMAP = 5, GDR_K_GDN2_SIMT = 6, GDR_K_GDN2_DECODE = 7,
-       GDR_K_COUNT = 8 };
+       GDR_K_FRAME_GRAM = 8, GDR_K_FRAME_SOLVE = 9, GDR_K_FRAME_CHAIN = 10, GDR_K_FRAME_OUT = 11,
+       GDR_K_COUNT = 12 };
 void gdr_profile_enable(int on);
 gdr_status gdr_profile_read(int id, long long *launches, double *total_ms);
 

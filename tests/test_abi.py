@@ -163,3 +163,25 @@ def test_gdn2_decode_rejects_on_host(kw, expect):
                                             a["S"], a["out"], a["N"], a["H"], a["dk"], a["dv"],
                                             a["dtype"], a["gate"], None)
     assert st == expect
+
+
+@nogpu
+@pytest.mark.parametrize("kw,expect", [
+    (dict(n=0), 1), (dict(dk=12), 2), (dict(dv=136), 2), (dict(gamma=None), 1),
+    (dict(ws=None, ws_bytes=0), 1), (dict(q=ctypes.c_void_p(0x10006)), 1), (dict(gate=4), 1),
+])
+def test_frame_rejects_on_host(kw, expect):
+    a = dict(q=P, k=P, v=P, g=P, gamma=P, S0=None, out=P, SF=P, B=1, T=64, H=2, dk=64, dv=64, n=16,
+             dtype=0, gate=1, ws=P, ws_bytes=16)
+    a.update(kw)
+    st = binding.lib().gdr_fwd_frame(a["q"], a["k"], a["v"], a["g"], a["gamma"], a["S0"], a["out"],
+                                     a["SF"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["n"],
+                                     a["dtype"], a["gate"], a["ws"], a["ws_bytes"], None)
+    assert st == expect
+
+
+def test_frame_workspace_size():
+    B, T, H, d, n = 1, 1000, 3, 128, 256
+    F = -(-T // n)
+    assert binding.fwd_frame_workspace_size(B, T, H, d, d, n) >= 3 * B * F * H * d * d * 4
+    assert binding.fwd_frame_workspace_size(B, T, H, 12, d, n) == 0
