@@ -294,6 +294,40 @@ class PrefillRun:
         return ms, h2d, d2h
 
 
+# ----------------------------------------------------------------- frame update
+class FrameRun:
+    """The implicit frame-level update over a batch of frames."""
+
+    def __init__(self, cfg, device, seed):
+        self.cfg = cfg
+        self.device = device
+        self.inp = inp = inputs.frame_inputs(cfg, seed=seed)
+        self.q, self.k, self.v = (dev_tensor(x, cfg.dtype, device) for x in (inp.q, inp.k, inp.v))
+        self.g, self.gamma = dev_tensor(inp.g, "f32", device), dev_tensor(inp.gamma, "f32", device)
+        self.S0 = dev_tensor(inp.S0, "f32", device)
+        self.out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.d_v), dtype=self.q.dtype, device=device)
+        self.SF = torch.empty((cfg.B, cfg.H, cfg.d_v, cfg.d_k), dtype=torch.float32, device=device)
+        ws = binding.fwd_frame_workspace_size(cfg.B, cfg.T, cfg.H, cfg.d_k, cfg.d_v, cfg.n)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+        self.n_seq = cfg.B
+
+    def step(self):
+        binding.gdr_fwd_frame(self.q, self.k, self.v, self.g, self.gamma, self.cfg.n, self.S0,
+                              out=self.out, S_final=self.SF, workspace=self.ws)
+
+    def tokens(self):
+        return self.cfg.B * self.cfg.T
+
+
+def frame_flops_per_token_head(dk, dv, n):
+    """G_t and C_t (2 d_k (d_k + d_v) per token), the output (2 d_k d_v per
+    token), and per frame the Cholesky (d_k^3 / 3), the substitutions for
+    M_t, N_t (2 d_k^2 (d_k + d_v)) and the chain product (2 d_v d_k^2), spread
+    over the frame's n tokens."""
+    per_frame = dk ** 3 / 3 + 2 * dk * dk * (dk + dv) + 2 * dv * dk * dk
+    return 2 * dk * (dk + dv) + 2 * dk * dv + per_frame / n
+
+
 # ----------------------------------------------------------------- decode
 class DecodeRun:
     """The decode workload: fresh tokens every step (drawn on the device from a
@@ -372,6 +406,26 @@ def oracle_prefill_sample(cfg, seed, budget_s):
                                                f"tokens ({token_heads} token-heads, {dt:.2f} s)"), dt
 
 
+def oracle_frame_sample(cfg, seed, budget_s):
+    """The frame-update oracle on the first h heads (single-threaded)."""
+    import oracle
+
+    inp = inputs.frame_inputs(cfg, seed=seed)
+
+    def run(h):
+        sl = lambda x: np.ascontiguousarray(x[:, :, :h])
+        S0 = None if inp.S0 is None else np.ascontiguousarray(inp.S0[:, :h])
+        t = time.perf_counter()
+        oracle.frame_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.g), sl(inp.gamma), cfg.n, S0)
+        return time.perf_counter() - t
+
+    t1 = run(1)
+    h = int(max(1, min(cfg.H, budget_s / max(t1, 1e-6))))
+    dt = run(h) if h > 1 else t1
+    return (cfg.B * cfg.T * h / cfg.H) / dt, 1, (f"{h} of {cfg.H} heads x all {cfg.B * cfg.T} "
+                                                 f"tokens ({dt:.2f} s)"), dt
+
+
 def oracle_decode_sample(cfg, seed, budget_s):
     import oracle
 
@@ -399,6 +453,10 @@ def workload_config(name):
                    **({"n_seq": c.n_seq} if c.n_seq else {}),
                    **({"n_h": c.n_h} if c.n_h > 1 else {}),
                    **({"variant": c.variant} if c.variant else {})}
+    if name in inputs.FRAME:
+        c = inputs.FRAME[name]
+        return c, {"workload": name, "B": c.B, "T": c.T, "H": c.H, "d_k": c.d_k, "d_v": c.d_v,
+                   "frame_tokens": c.n, "frames": c.frames, "gate": c.gate, "dtype_io": c.dtype}
     c = inputs.DECODE[name]
     return c, {"workload": name, "N": c.N, "H": c.H, "d_k": c.d_k, "d_v": c.d_v, "gate": c.gate,
                "dtype_io": c.dtype, "steps_per_sequence": c.steps}
@@ -448,6 +506,12 @@ def run_reference(args, rank, world):
                                                        budget)
             if i >= args.warmup:
                 vals.append(v)
+    elif isinstance(cfg, inputs.FrameConfig):
+        for i in range(args.warmup + args.steps):
+            v, cores, sample, _ = oracle_frame_sample(cfg, inputs.BASE_SEED + cfg.seed_index,
+                                                      budget)
+            if i >= args.warmup:
+                vals.append(v)
     else:
         for i in range(args.warmup + args.steps):
             v, cores, sample, _ = oracle_prefill_sample(cfg, inputs.BASE_SEED + cfg.seed_index,
@@ -472,7 +536,9 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
     cfg, conf = workload_config(name)
     seed = (inputs.BASE_SEED + cfg.seed_index) * 1000 + rank
     is_decode = isinstance(cfg, inputs.DecodeConfig)
+    is_frame = isinstance(cfg, inputs.FrameConfig)
     run = (DecodeRun(cfg, device, seed, steps + warmup) if is_decode
+           else FrameRun(cfg, device, seed) if is_frame
            else PrefillRun(cfg, device, seed, path))
     flush = None if is_decode else L2Flush(device)
     for _ in range(warmup):
@@ -512,6 +578,18 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                 "peak_source": peak_kind + " hbm_gbs", "algorithmic_bytes_per_launch": B_,
                 "frac_of_8TBps_spec": ach / 8000.0}
         conf["l2"] = "no flush: the 512 MiB state is larger than L2 and is streamed every step"
+    elif is_frame:
+        th = cfg.B * cfg.T * cfg.H
+        flops = frame_flops_per_token_head(cfg.d_k, cfg.d_v, cfg.n) * th
+        peak = SM_COUNT * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        ach = flops / (ms * 1e-3) / 1e12
+        roof = {"bound": "alu", "kernel": "frame step (4 passes)", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
+                "algorithmic_flops_per_launch": flops, "dominant_pass": dom}
+        conf["l2"] = (f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then a "
+                      f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer, outside the "
+                      "per-step CUDA-event intervals)")
     else:
         th = cfg.B * cfg.T * cfg.H * cfg.n_h  # virtual steps when a token has substeps
         f_all = prefill_flops_per_token_head(cfg.chunk, cfg.d_k, cfg.d_v)
@@ -545,7 +623,7 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
     res = {"value": value, "ms_per_step": ms, "wall_s_incl_flush": wall, "roofline": roof,
            "kernels": kernels, "gpu_launches": launches, "clocks": clocks, "config": conf,
            "cfg": cfg, "run": run}
-    if with_e2e and not is_decode:
+    if with_e2e and not is_decode and not is_frame:
         e_ms, h2d, d2h = run.e2e(max(1, min(steps, 5)))
         e_ms = max_over_ranks(e_ms, world)
         res["e2e"] = {"value": tokens_all / (e_ms * 1e-3), "unit": "tokens/s",
@@ -553,6 +631,8 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
     if with_cpu and rank == 0 and world == 1:
         if is_decode:
             v, cores, sample, _ = oracle_decode_sample(cfg, seed, 10.0)
+        elif is_frame:
+            v, cores, sample, _ = oracle_frame_sample(cfg, seed, 10.0)
         else:
             v, cores, sample, _ = oracle_prefill_sample(cfg, seed, 10.0)
         res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -567,9 +647,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gdn_prefill",
-                    choices=list(inputs.PREFILL) + list(inputs.DECODE))
+                    choices=list(inputs.PREFILL) + list(inputs.DECODE) + list(inputs.FRAME))
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
-    ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill,gdp_prefill,gdn2_prefill",
+    ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill,gdp_prefill,gdn2_prefill,frame_prefill",
                     help="comma-separated workloads measured after the main one ('' for none)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
