@@ -21,8 +21,14 @@
 //   frame_chain  (batch*head, row block) S_t = S_{t-1} M_t + N_t over the frames
 //                                        (rows of S are independent)
 //   frame_out    (token tile, head, batch) o_i = S_t q_i
-// All arithmetic is fp32 on the CUDA cores.
+// The factorisation, the affine pair and the chain are fp32 on the CUDA cores.
+// The two dense contractions over tokens -- the Gram pass and the output pass
+// -- run on the tensor cores for bf16 inputs with d_k = d_v = 128 (tcgen05,
+// operands staged by TMA, fp32 accumulators in TMEM), and on the CUDA cores
+// in fp32 otherwise.
 #include "common.cuh"
+#include "sm100.cuh"
+#include "tmap.cuh"
 
 namespace gdr {
 namespace frame {
@@ -171,7 +177,7 @@ frame_affine_kernel(float *__restrict__ GM, float *__restrict__ CN, const float 
 __global__ void __launch_bounds__(kThreads)
 frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Nw,
                    const float *__restrict__ S0, float *__restrict__ Sw,
-                   float *__restrict__ S_final, Dims d) {
+                   __nv_bfloat16 *__restrict__ Sb, float *__restrict__ S_final, Dims d) {
     extern __shared__ float sm[];
     const int bh = blockIdx.x, b = bh / d.H, h = bh % d.H;
     const int r0 = blockIdx.y * kChainRows;
@@ -200,7 +206,9 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Nw,
             const int r = e / dk, c = e % dk;
             const float x = Sn[r * ast + c];
             S[r * ast + c] = x;
-            Sw[sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c] = x;
+            const size_t o = sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c;
+            if (Sb) Sb[o] = __float2bfloat16_rn(x);  // operand of the tensor-core output pass
+            else Sw[o] = x;
         }
     }
     __syncthreads();
@@ -241,6 +249,219 @@ frame_out_kernel(const Tin *__restrict__ q, const float *__restrict__ Sw, Tin *_
     }
 }
 
+// ---------------------------------------------------------------- tensor cores
+using namespace sm100;
+constexpr int kTD = 128;                 // d_k = d_v on the tensor-core passes
+constexpr int kGT = 64;                  // tokens per Gram tile (K = 64 per tile)
+constexpr uint32_t kGStage = 3 * 16384;  // K, V, gamma . K (bf16, two 64-column atoms each)
+constexpr uint32_t kSpinF = 1u << 24;
+
+// G_t = K^T (Gamma K) and C_t = V^T (Gamma K) on the tensor cores: M = N = 128
+// (features), K = the frame's tokens, 64 per tile, two TMA stages.  K and V
+// are MN-major A operands straight from their TMA tiles; Gamma K is a scaled
+// copy (MN-major B).  Rows past the frame end get gamma = 0.
+__global__ void __launch_bounds__(256)
+frame_gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const float *__restrict__ gamma, float *__restrict__ Gw, float *__restrict__ Cw,
+                     Dims d, unsigned int *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + 2 * kGStage);  // [2]
+    uint64_t *done = full + 2;                                         // [2]
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(done + 2);
+    float *gs = reinterpret_cast<float *>(tslot + 4);                  // [2][64]
+    const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = f * d.n, t1 = min(d.T, t0 + d.n);
+    const int ntiles = (t1 - t0 + kGT - 1) / kGT;
+    const int x0 = h * kTD;
+    const long yb = (long)b * d.T + t0;
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(&done[0], 1);
+        mbar_init(&done[1], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;  // G at [0,128), C at [128,256)
+    auto issue = [&](int i) {
+        uint8_t *st = sm + (i & 1) * kGStage;
+        const int y = (int)(yb + (long)i * kGT);
+        mbar_arrive_expect_tx(&full[i & 1], 4 * 8192);
+        tma_load_2d(st, &tm_k, &full[i & 1], x0, y);
+        tma_load_2d(st + 8192, &tm_k, &full[i & 1], x0 + 64, y);
+        tma_load_2d(st + 16384, &tm_v, &full[i & 1], x0, y);
+        tma_load_2d(st + 16384 + 8192, &tm_v, &full[i & 1], x0 + 64, y);
+    };
+    int issued = 0;  // tiles whose loads tid 0 issued
+    if (tid == 0) {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        for (; issued < 2 && issued < ntiles; ++issued) issue(issued);
+    }
+    bool ok = true;
+    const uint32_t id = idesc_bf16(128, 128, 1, 1);
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i & 1;
+        uint8_t *st = sm + s * kGStage;
+        if (tid < kGT) {
+            const int tok = t0 + i * kGT + tid;
+            gs[s * kGT + tid] = (tok < t1) ? gamma[((size_t)b * d.T + tok) * d.H + h] : 0.f;
+        }
+        const bool okw = mbar_wait_bounded(&full[s], (i >> 1) & 1, kSpinF, err);
+        if (!__syncthreads_and(okw)) { ok = false; break; }
+        // gamma . K (element-wise, so the swizzled layout carries over)
+        for (int e = tid; e < kGT * 16; e += 256) {
+            const int r = e >> 4, c = e & 15;
+            const uint32_t off = (c >> 3) * 8192 + r * 128 + (c & 7) * 16;
+            float x[8];
+            unpack8(*reinterpret_cast<const uint4 *>(st + off), x);
+            const float gr = gs[s * kGT + r];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] *= gr;
+            *reinterpret_cast<uint4 *>(st + 32768 + off) = pack8(x);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t dk_ = sdesc_sw128(smem_u32(st), 8192, 1024);
+            const uint64_t dv_ = sdesc_sw128(smem_u32(st + 16384), 8192, 1024);
+            const uint64_t dg_ = sdesc_sw128(smem_u32(st + 32768), 8192, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                mma_bf16_ss(tmem, sdesc_add(dk_, kk * 2048), sdesc_add(dg_, kk * 2048), id, (i | kk) > 0);
+                mma_bf16_ss(tmem + 128, sdesc_add(dv_, kk * 2048), sdesc_add(dg_, kk * 2048), id, (i | kk) > 0);
+            }
+            mma_commit(&done[s]);
+            if (i + 2 < ntiles) {  // this stage is free once its MMAs are done
+                if (mbar_wait_bounded(&done[s], (i >> 1) & 1, kSpinF, err)) {
+                    issue(i + 2);
+                    issued = i + 3;
+                }
+            }
+        }
+    }
+    // the last tile's MMAs cover all earlier ones
+    if (ok && ntiles > 0) ok = mbar_wait_bounded(&done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, kSpinF, err);
+    tc_fence_after();
+    if (ok) {
+        const int qd = warp & 3, hf = warp >> 2, row = qd * 32 + lane;
+        const uint32_t lb = (uint32_t)(qd * 32) << 16;
+        const size_t sl = slot(d, b, f, h);
+        for (int m = 0; m < 2; ++m) {  // G, then C
+            float *dst = (m ? Cw : Gw) + sl * (size_t)kTD * kTD + (size_t)row * kTD + hf * 64;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                float x[16];
+                if (ntiles > 0) {
+                    tmem_ld16(tmem + m * 128 + lb + hf * 64 + cb * 16, x);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) x[j] = 0.f;
+                }
+                float4 *d4 = reinterpret_cast<float4 *>(dst + cb * 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) d4[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+            }
+        }
+    }
+    // loads still in flight (error path) must land before the CTA exits
+    if (tid == 0) {
+        for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait_bounded(&full[i & 1], (i >> 1) & 1, kSpinF, err);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// o_i = S_t q_i for a tile of 128 tokens of one frame on the tensor cores:
+// D[128 tokens x 128] = Q (K-major A) * S_t^T (bf16 copy of S_t, K-major B).
+__global__ void __launch_bounds__(128)
+frame_out_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_s,
+                    __nv_bfloat16 *__restrict__ out, Dims d, unsigned int *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 65536);  // [2]: loads, MMAs
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 2);
+    const int tiles = (d.n + 127) / 128;
+    const int f = blockIdx.x / tiles, tile = blockIdx.x % tiles;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int tt = f * d.n + tile * 128;
+    const int cnt = min(128, min(d.T, (f + 1) * d.n) - tt);
+    if (cnt <= 0) return;  // whole CTA, before any barrier
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    // Q: two 64-feature atoms of [128 tokens][64]; S_t: two atoms of [128 rows (d_v)][64 (d_k)]
+    if (tid == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_s);
+        const int y = (int)((long)b * d.T + tt);
+        const int ys = (int)(slot(d, b, f, h) * kTD);
+        mbar_arrive_expect_tx(&bar[0], 65536);
+        tma_load_2d(sm, &tm_q, &bar[0], h * kTD, y);
+        tma_load_2d(sm + 8192, &tm_q, &bar[0], h * kTD, y + 64);
+        tma_load_2d(sm + 16384, &tm_q, &bar[0], h * kTD + 64, y);
+        tma_load_2d(sm + 16384 + 8192, &tm_q, &bar[0], h * kTD + 64, y + 64);
+        tma_load_2d(sm + 32768, &tm_s, &bar[0], 0, ys);
+        tma_load_2d(sm + 32768 + 16384, &tm_s, &bar[0], 64, ys);
+    }
+    bool ok = mbar_wait_bounded(&bar[0], 0, kSpinF, err);
+    if (__syncthreads_and(ok) && tid == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, 128, 0, 0);
+        const uint64_t da = sdesc_sw128(smem_u32(sm), 16, 1024);
+        const uint64_t db = sdesc_sw128(smem_u32(sm + 32768), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ss(tmem, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32),
+                        sdesc_add(db, (kk >> 2) * 16384 + (kk & 3) * 32), id, kk > 0);
+        mma_commit(&bar[1]);
+    }
+    ok = ok && mbar_wait_bounded(&bar[1], 0, kSpinF, err);
+    tc_fence_after();
+    if (ok) {  // thread = token row
+        const int r = warp * 32 + lane;
+        const uint32_t lb = (uint32_t)(warp * 32) << 16;
+        __nv_bfloat16 *orow = out + (((size_t)b * d.T + tt + r) * d.H + h) * kTD;
+#pragma unroll
+        for (int cb = 0; cb < 8; ++cb) {
+            float x[16];
+            tmem_ld16(tmem + lb + cb * 16, x);
+            tmem_wait_ld();
+            if (r < cnt) {
+                uint4 *o4 = reinterpret_cast<uint4 *>(orow + cb * 16);
+                o4[0] = pack8(x);
+                o4[1] = pack8(x + 8);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
 }  // namespace frame
 }  // namespace gdr
 
@@ -252,7 +473,7 @@ namespace {
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct FrameLayout {
-    size_t GM, CN, Sw, total;
+    size_t GM, CN, Sw, total;  // Sw holds fp32 S_t, or their bf16 copies on the tensor-core path
 };
 
 FrameLayout frame_layout(int B, int T, int H, int dk, int dv, int n) {
@@ -274,6 +495,8 @@ bool frame_shape_ok(int dk, int dv) {
 
 size_t affine_smem(int dk, int dv) { return sizeof(float) * (size_t)(dk + dk + dv) * (dk + 1); }
 
+bool frame_tc_applies(const Dims &d, bool bf16) { return bf16 && d.dk == kTD && d.dv == kTD; }
+
 template <typename Tin>
 cudaError_t frame_launch(const void *q, const void *k, const void *v, const float *g,
                          const float *gamma, const float *S0, void *out, float *S_final,
@@ -281,7 +504,20 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
                          unsigned int *err) {
     const FrameLayout L = frame_layout(d.B, d.T, d.H, d.dk, d.dv, d.n);
     float *GM = (float *)(ws + L.GM), *CN = (float *)(ws + L.CN), *Sw = (float *)(ws + L.Sw);
+    __nv_bfloat16 *Sb = (__nv_bfloat16 *)(ws + L.Sw);
+    const bool tc = frame_tc_applies(d, sizeof(Tin) == 2);
     cudaError_t e;
+    CUtensorMap mk, mv, mq, ms;
+    if (tc) {
+        using namespace gdr_host::tmap;
+        const uint64_t rows = (uint64_t)d.B * d.T, HD = (uint64_t)d.H * kTD;
+        const uint64_t srows = (uint64_t)d.B * d.F * d.H * kTD;
+        if (!make_map(&mk, kBF, k, HD, rows, HD * 2, 64, 64, kSW) ||
+            !make_map(&mv, kBF, v, HD, rows, HD * 2, 64, 64, kSW) ||
+            !make_map(&mq, kBF, q, HD, rows, HD * 2, 64, 64, kSW) ||
+            !make_map(&ms, kBF, Sb, kTD, srows, kTD * 2, 64, 128, kSW))
+            return cudaErrorInvalidValue;
+    }
     const size_t sm_gram = sizeof(float) * (size_t)(kTokTile * (d.dk + 1) + kTokTile * (d.dv + 1) + kTokTile);
     const size_t sm_aff = affine_smem(d.dk, d.dv);
     const size_t sm_chain = sizeof(float) * (size_t)(d.dk + 2 * kChainRows) * (d.dk + 1);
@@ -292,9 +528,17 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
         (e = cudaFuncSetAttribute(frame_out_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out)))
         return e;
     const dim3 gf((unsigned)d.F, (unsigned)d.H, (unsigned)d.B);
+    const size_t sm_gram_tc = 1024 + 2 * kGStage + 1024, sm_out_tc = 1024 + 65536 + 64;
+    if (tc &&
+        ((e = cudaFuncSetAttribute(frame_gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gram_tc)) ||
+         (e = cudaFuncSetAttribute(frame_out_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out_tc))))
+        return e;
     {
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_GRAM, st);
-        frame_gram_kernel<Tin><<<gf, kThreads, sm_gram, st>>>((const Tin *)k, (const Tin *)v, gamma, GM, CN, d);
+        if (tc)
+            frame_gram_tc_kernel<<<gf, 256, sm_gram_tc, st>>>(mk, mv, gamma, GM, CN, d, err);
+        else
+            frame_gram_kernel<Tin><<<gf, kThreads, sm_gram, st>>>((const Tin *)k, (const Tin *)v, gamma, GM, CN, d);
         gdr_host::prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -307,15 +551,20 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
     {
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_CHAIN, st);
         const dim3 gc((unsigned)(d.B * d.H), (unsigned)((d.dv + kChainRows - 1) / kChainRows));
-        frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, S0, Sw, S_final, d);
+        frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, S0, Sw, tc ? Sb : nullptr, S_final, d);
         gdr_host::prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_OUT, st);
-        const int tiles = (d.n + kTokTile - 1) / kTokTile;
-        const dim3 go((unsigned)(d.F * tiles), (unsigned)d.H, (unsigned)d.B);
-        frame_out_kernel<Tin><<<go, kThreads, sm_out, st>>>((const Tin *)q, Sw, (Tin *)out, d);
+        if (tc) {
+            const dim3 go((unsigned)(d.F * ((d.n + 127) / 128)), (unsigned)d.H, (unsigned)d.B);
+            frame_out_tc_kernel<<<go, 128, sm_out_tc, st>>>(mq, ms, (__nv_bfloat16 *)out, d, err);
+        } else {
+            const int tiles = (d.n + kTokTile - 1) / kTokTile;
+            const dim3 go((unsigned)(d.F * tiles), (unsigned)d.H, (unsigned)d.B);
+            frame_out_kernel<Tin><<<go, kThreads, sm_out, st>>>((const Tin *)q, Sw, (Tin *)out, d);
+        }
         gdr_host::prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

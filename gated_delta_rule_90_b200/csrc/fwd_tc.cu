@@ -41,6 +41,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tmap.cuh"
 
 namespace gdr {
 namespace tc {
@@ -75,31 +76,6 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 }
 
 // bf16x8 <-> float8 helpers (16-byte chunks of a tile)
-__device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 x = __bfloat1622float2(h[i]);
-        f[2 * i] = x.x;
-        f[2 * i + 1] = x.y;
-    }
-}
-__device__ __forceinline__ void ld8(const float *p, float *f) {  // 32-byte aligned
-    const float4 x = reinterpret_cast<const float4 *>(p)[0], y = reinterpret_cast<const float4 *>(p)[1];
-    f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
-    f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
-}
-
-__device__ __forceinline__ uint4 pack8(const float *f) {
-    uint4 u;
-    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-    return u;
-}
-
-// Locate chunk `gcid` of the packed or regular batch: sequence index, first
-// token row and valid length.  Returns false for an unused slot.
 __device__ __forceinline__ bool locate_chunk(const Geo &geo, const int32_t *cu, const Ws &ws,
                                              int gcid, long &tstart, int &len) {
     long t0, t1;
@@ -1021,40 +997,7 @@ WsLayout ws_layout(int B, int T, int H, int n_seq, int varlen) {
     return L;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
-    }
-    return fn;
-}
-
-// 2-D tensor map: inner extent `inner` elements, `rows` rows, row pitch
-// `pitch` bytes, box box0 x box1, zero fill out of bounds.
-bool make_map(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t inner,
-              uint64_t rows, uint64_t pitch, uint32_t box0, uint32_t box1,
-              CUtensorMapSwizzle swz) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {pitch};
-    cuuint32_t box[2] = {box0, box1};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, type, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-constexpr CUtensorMapDataType kBF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-constexpr CUtensorMapDataType kF32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-constexpr CUtensorMapSwizzle kSW = CU_TENSOR_MAP_SWIZZLE_128B;
-constexpr CUtensorMapSwizzle kNoSW = CU_TENSOR_MAP_SWIZZLE_NONE;
+using namespace gdr_host::tmap;
 
 size_t wy_smem_bytes(bool ch) {  // + 1024 for the in-kernel alignment
     return 1024 + WySmem::small(ch) + WySmem::small_bytes(ch);
