@@ -33,6 +33,9 @@
 namespace gdr {
 namespace frame {
 
+using namespace sm100;
+constexpr uint32_t kSpinF = 1u << 24;  // poll limit of every mbarrier wait
+
 constexpr int kThreads = 256;
 constexpr int kTokTile = 32;   // tokens per smem tile in the Gram and output passes
 constexpr int kChainRows = 16; // state rows per CTA in the chain
@@ -107,35 +110,50 @@ frame_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
 }
 
 // Cholesky of I + G_t (right-looking, in shared memory), then the rows of
-// M_t = D_t (I + G_t)^-1 and N_t = C_t (I + G_t)^-1 by substitution: row x of
-// either solves x (L L^T) = r, i.e. L y = r^T, L^T x^T = y, one row per thread.
-// M_t overwrites G_t and N_t overwrites C_t in the workspace.
+// M_t = D_t (I + G_t)^-1 and N_t = C_t (I + G_t)^-1: each solves
+// x (L L^T) = r, i.e. y L^T = r (forward) and x L = y (backward), for all
+// d_k + d_v right-hand sides at once, one row per thread, blocked by 16
+// columns: the part of a block that depends on earlier blocks is a small GEMM
+// with 16 independent sums per thread, the rest a 16 x 16 triangular solve.
+// The forward pass reads L by columns, so the factorisation also stores L^T in
+// the free upper triangle.  M_t overwrites G_t and N_t overwrites C_t.
+constexpr int kAffB = 16;  // column block of the substitution
 __global__ void __launch_bounds__(kThreads)
 frame_affine_kernel(float *__restrict__ GM, float *__restrict__ CN, const float *__restrict__ g,
                     int per_channel, Dims d, unsigned int *err) {
     extern __shared__ float sm[];
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int dk = d.dk, ast = dk + 1;
-    float *A = sm, *R = A + dk * ast;  // R: (dk + dv) rows of length dk (+1 pad)
+    const int dk = d.dk, ast = dk + 4, rst = dk + 1;  // A rows 16-byte aligned
+    const int nrhs = dk + d.dv;
+    float *A = sm, *R = A + dk * ast;  // R: nrhs rows of length dk (+1 pad)
     const int tid = threadIdx.x;
     const size_t sl = slot(d, b, f, h);
     float *Gp = GM + sl * (size_t)dk * dk, *Cp = CN + sl * (size_t)d.dv * dk;
-    for (int e = tid; e < dk * dk; e += kThreads) {
-        const int i = e / dk, j = e % dk;
-        A[i * ast + j] = Gp[e] + (i == j ? 1.f : 0.f);
+    const int q4 = dk / 4;
+#pragma unroll 4
+    for (int e = tid; e < dk * q4; e += kThreads) {  // A = I + G (16-byte loads)
+        const int i = e / q4, j = (e % q4) * 4;
+        const float4 x = reinterpret_cast<const float4 *>(Gp)[e];
+        float *Ai = A + i * ast + j;
+        Ai[0] = x.x + (i == j ? 1.f : 0.f);
+        Ai[1] = x.y + (i == j + 1 ? 1.f : 0.f);
+        Ai[2] = x.z + (i == j + 2 ? 1.f : 0.f);
+        Ai[3] = x.w + (i == j + 3 ? 1.f : 0.f);
     }
-    // right-hand sides: rows of D_t, then rows of C_t
-    for (int e = tid; e < dk * dk; e += kThreads) {
+#pragma unroll 4
+    for (int e = tid; e < d.dv * q4; e += kThreads) {  // rows of C_t
+        const int i = e / q4, j = (e % q4) * 4;
+        const float4 x = reinterpret_cast<const float4 *>(Cp)[e];
+        float *Ri = R + (dk + i) * rst + j;
+        Ri[0] = x.x; Ri[1] = x.y; Ri[2] = x.z; Ri[3] = x.w;
+    }
+    for (int e = tid; e < dk * dk; e += kThreads) {  // rows of D_t
         const int i = e / dk, j = e % dk;
         const float a = per_channel ? __expf(g[sl * dk + i]) : __expf(g[sl]);
-        R[i * ast + j] = (i == j) ? a : 0.f;
-    }
-    for (int e = tid; e < d.dv * dk; e += kThreads) {
-        const int i = e / dk, j = e % dk;
-        R[(dk + i) * ast + j] = Cp[e];
+        R[i * rst + j] = (i == j) ? a : 0.f;
     }
     __syncthreads();
-    // right-looking Cholesky: column j, then the trailing update
+    // right-looking Cholesky: column j, then the trailing update; L^T mirrored
     for (int j = 0; j < dk; ++j) {
         const float ajj = A[j * ast + j];
         const float ljj = sqrtf(fmaxf(ajj, 1e-30f));
@@ -144,79 +162,192 @@ frame_affine_kernel(float *__restrict__ GM, float *__restrict__ CN, const float 
             if (!(ajj > 0.f)) atomicOr(err, kErrNumeric);
             A[j * ast + j] = ljj;
         }
-        for (int i = j + 1 + tid; i < dk; i += kThreads) A[i * ast + j] /= ljj;
+        for (int i = j + 1 + tid; i < dk; i += kThreads) {
+            const float lij = A[i * ast + j] / ljj;
+            A[i * ast + j] = lij;
+            A[j * ast + i] = lij;  // L^T in the upper triangle
+        }
         __syncthreads();
-        const int m = dk - j - 1;  // trailing block (j+1.., j+1..), lower triangle
-        for (int e = tid; e < m * m; e += kThreads) {
-            const int i = j + 1 + e / m, c = j + 1 + e % m;
-            if (c <= i) A[i * ast + c] -= A[i * ast + j] * A[c * ast + j];
+        // trailing update A[i][c] -= L[i][j] L[c][j] for i, c > j: a warp per
+        // row, lanes along c, L[c][j] read from the mirrored row j.  The whole
+        // square is updated; its upper part is rewritten by later mirror rows.
+        // Each lane keeps its four L[c][j] in registers; rows are unrolled so
+        // that the loads of several rows are in flight together.
+        const int warp = tid >> 5, lane = tid & 31;
+        float lj[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = lane + 32 * u;
+            lj[u] = (c > j && c < dk) ? A[j * ast + c] : 0.f;
+        }
+#pragma unroll 4
+        for (int i = j + 1 + warp; i < dk; i += kThreads / 32) {
+            const float lij = A[i * ast + j];
+            float *Ai = A + i * ast;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = lane + 32 * u;
+                if (c > j && c < dk) Ai[c] = fmaf(-lij, lj[u], Ai[c]);
+            }
         }
         __syncthreads();
     }
-    // substitution, one right-hand side row per thread
-    for (int r = tid; r < dk + d.dv; r += kThreads) {
-        float *x = R + r * ast;
-        for (int i = 0; i < dk; ++i) {  // L y = r
-            float s = x[i];
-            for (int m2 = 0; m2 < i; ++m2) s = fmaf(-A[i * ast + m2], x[m2], s);
-            x[i] = s / A[i * ast + i];
+    for (int r = tid; r < nrhs; r += kThreads) {
+        float *x = R + r * rst;
+        // forward: y_c = (r_c - sum_{m<c} y_m L[c][m]) / L[c][c]
+        for (int j0 = 0; j0 < dk; j0 += kAffB) {
+            float acc[kAffB];
+#pragma unroll
+            for (int c = 0; c < kAffB; ++c) acc[c] = x[j0 + c];
+            for (int m = 0; m < j0; ++m) {
+                const float ym = x[m];
+                const float4 *lt = reinterpret_cast<const float4 *>(A + m * ast + j0);  // L[j0..][m]
+#pragma unroll
+                for (int c4 = 0; c4 < kAffB / 4; ++c4) {
+                    const float4 l = lt[c4];
+                    acc[4 * c4] = fmaf(-ym, l.x, acc[4 * c4]);
+                    acc[4 * c4 + 1] = fmaf(-ym, l.y, acc[4 * c4 + 1]);
+                    acc[4 * c4 + 2] = fmaf(-ym, l.z, acc[4 * c4 + 2]);
+                    acc[4 * c4 + 3] = fmaf(-ym, l.w, acc[4 * c4 + 3]);
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < kAffB; ++c) {
+#pragma unroll
+                for (int c2 = 0; c2 < c; ++c2) acc[c] = fmaf(-acc[c2], A[(j0 + c) * ast + j0 + c2], acc[c]);
+                acc[c] /= A[(j0 + c) * ast + j0 + c];
+            }
+#pragma unroll
+            for (int c = 0; c < kAffB; ++c) x[j0 + c] = acc[c];
         }
-        for (int i = dk - 1; i >= 0; --i) {  // L^T x = y
-            float s = x[i];
-            for (int m2 = i + 1; m2 < dk; ++m2) s = fmaf(-A[m2 * ast + i], x[m2], s);
-            x[i] = s / A[i * ast + i];
+        // backward: x_c = (y_c - sum_{m>c} x_m L[m][c]) / L[c][c]
+        for (int j0 = dk - kAffB; j0 >= 0; j0 -= kAffB) {
+            float acc[kAffB];
+#pragma unroll
+            for (int c = 0; c < kAffB; ++c) acc[c] = x[j0 + c];
+            for (int m = j0 + kAffB; m < dk; ++m) {
+                const float xm = x[m];
+                const float4 *lr = reinterpret_cast<const float4 *>(A + m * ast + j0);  // L[m][j0..]
+#pragma unroll
+                for (int c4 = 0; c4 < kAffB / 4; ++c4) {
+                    const float4 l = lr[c4];
+                    acc[4 * c4] = fmaf(-xm, l.x, acc[4 * c4]);
+                    acc[4 * c4 + 1] = fmaf(-xm, l.y, acc[4 * c4 + 1]);
+                    acc[4 * c4 + 2] = fmaf(-xm, l.z, acc[4 * c4 + 2]);
+                    acc[4 * c4 + 3] = fmaf(-xm, l.w, acc[4 * c4 + 3]);
+                }
+            }
+#pragma unroll
+            for (int c = kAffB - 1; c >= 0; --c) {
+#pragma unroll
+                for (int c2 = c + 1; c2 < kAffB; ++c2) acc[c] = fmaf(-acc[c2], A[(j0 + c2) * ast + j0 + c], acc[c]);
+                acc[c] /= A[(j0 + c) * ast + j0 + c];
+            }
+#pragma unroll
+            for (int c = 0; c < kAffB; ++c) x[j0 + c] = acc[c];
         }
     }
     __syncthreads();
-    for (int e = tid; e < dk * dk; e += kThreads) Gp[e] = R[(e / dk) * ast + e % dk];
-    for (int e = tid; e < d.dv * dk; e += kThreads) Cp[e] = R[(dk + e / dk) * ast + e % dk];
+    for (int e = tid; e < dk * q4; e += kThreads) {
+        const int i = e / q4, j = (e % q4) * 4;
+        const float *Ri = R + i * rst + j;
+        reinterpret_cast<float4 *>(Gp)[e] = make_float4(Ri[0], Ri[1], Ri[2], Ri[3]);
+    }
+    for (int e = tid; e < d.dv * q4; e += kThreads) {
+        const int i = e / q4, j = (e % q4) * 4;
+        const float *Ri = R + (dk + i) * rst + j;
+        reinterpret_cast<float4 *>(Cp)[e] = make_float4(Ri[0], Ri[1], Ri[2], Ri[3]);
+    }
 }
 
 // S_t = S_{t-1} M_t + N_t for kChainRows rows of S; every S_t is stored for
-// the output pass, the last one also as S_final.
+// the output pass (fp32, or its bf16 copy for the tensor-core output pass), the
+// last one also as S_final.  M_t arrives by bulk copy into one of two buffers,
+// one frame ahead; thread (row r, 8 columns) keeps 8 independent sums.
 __global__ void __launch_bounds__(kThreads)
 frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Nw,
                    const float *__restrict__ S0, float *__restrict__ Sw,
-                   __nv_bfloat16 *__restrict__ Sb, float *__restrict__ S_final, Dims d) {
-    extern __shared__ float sm[];
+                   __nv_bfloat16 *__restrict__ Sb, float *__restrict__ S_final, Dims d,
+                   unsigned int *err) {
+    extern __shared__ __align__(16) float sm[];
     const int bh = blockIdx.x, b = bh / d.H, h = bh % d.H;
     const int r0 = blockIdx.y * kChainRows;
     const int nr = min(kChainRows, d.dv - r0);
-    const int dk = d.dk, ast = dk + 1;
-    float *M = sm, *S = M + dk * ast, *Sn = S + kChainRows * ast;
-    const int tid = threadIdx.x;
+    const int dk = d.dk;
+    float *Mb = sm, *S = Mb + 2 * dk * dk;  // M_t double buffer (unpadded), S rows [16][dk]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(S + kChainRows * dk);  // [2]
+    const int tid = threadIdx.x, r = tid >> 4, c0 = (tid & 15) * 8;
+    const bool mine = r < nr && c0 < dk;
+    const uint32_t mbytes = (uint32_t)(dk * dk * 4);
     const size_t soff = ((size_t)b * d.H + h) * (size_t)d.dv * dk;
-    for (int e = tid; e < kChainRows * dk; e += kThreads) {
-        const int r = e / dk, c = e % dk;
-        S[r * ast + c] = (S0 && r < nr) ? S0[soff + (size_t)(r0 + r) * dk + c] : 0.f;
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
     }
-    for (int f = 0; f < d.F; ++f) {
-        const size_t sl = slot(d, b, f, h);
-        __syncthreads();
-        for (int e = tid; e < dk * dk; e += kThreads) M[(e / dk) * ast + e % dk] = Mw[sl * (size_t)dk * dk + e];
-        __syncthreads();
-        for (int e = tid; e < nr * dk; e += kThreads) {
-            const int r = e / dk, c = e % dk;
-            float acc = Nw[sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c];
-            for (int m = 0; m < dk; ++m) acc = fmaf(S[r * ast + m], M[m * ast + c], acc);
-            Sn[r * ast + c] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nr * dk; e += kThreads) {
-            const int r = e / dk, c = e % dk;
-            const float x = Sn[r * ast + c];
-            S[r * ast + c] = x;
-            const size_t o = sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c;
-            if (Sb) Sb[o] = __float2bfloat16_rn(x);  // operand of the tensor-core output pass
-            else Sw[o] = x;
-        }
+    for (int e = tid; e < kChainRows * dk; e += kThreads) {
+        const int rr = e / dk, c = e % dk;
+        S[e] = (S0 && rr < nr) ? S0[soff + (size_t)(r0 + rr) * dk + c] : 0.f;
     }
     __syncthreads();
-    if (S_final)
-        for (int e = tid; e < nr * dk; e += kThreads) {
-            const int r = e / dk, c = e % dk;
-            S_final[soff + (size_t)(r0 + r) * dk + c] = S[r * ast + c];
+    int issued = 0;
+    if (tid == 0)
+        for (; issued < 2 && issued < d.F; ++issued) {
+            mbar_arrive_expect_tx(&bar[issued], mbytes);
+            bulk_load(Mb + issued * dk * dk, Mw + slot(d, b, issued, h) * (size_t)dk * dk, mbytes,
+                      &bar[issued]);
         }
+    bool ok = true;
+    for (int f = 0; f < d.F; ++f) {
+        const size_t sl = slot(d, b, f, h);
+        const float *Mf = Mb + (f & 1) * dk * dk;
+        float acc[8];
+        if (mine) {
+            const float *np = Nw + sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c0;
+            ld8(np, acc);
+        }
+        const bool okw = mbar_wait_bounded(&bar[f & 1], (f >> 1) & 1, kSpinF, err);
+        if (!__syncthreads_and(okw)) { ok = false; break; }
+        if (mine) {
+            const float *Sr = S + r * dk;
+            for (int m = 0; m < dk; ++m) {
+                const float sv = Sr[m];
+                float mm[8];
+                ld8(Mf + m * dk + c0, mm);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = fmaf(sv, mm[j], acc[j]);
+            }
+        }
+        __syncthreads();  // S and this M buffer are read
+        if (tid == 0 && f + 2 < d.F) {
+            mbar_arrive_expect_tx(&bar[f & 1], mbytes);
+            bulk_load(Mb + (f & 1) * dk * dk, Mw + slot(d, b, f + 2, h) * (size_t)dk * dk, mbytes,
+                      &bar[f & 1]);
+            issued = f + 3;
+        }
+        if (mine) {
+            float *Sr = S + r * dk + c0;
+            const size_t o = sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) Sr[j] = acc[j];
+            if (Sb) {  // operand of the tensor-core output pass
+                *reinterpret_cast<uint4 *>(Sb + o) = pack8(acc);
+            } else {
+                float4 *o4 = reinterpret_cast<float4 *>(Sw + o);
+                o4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                o4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
+        }
+        __syncthreads();
+    }
+    if (ok && S_final && mine) {
+        float4 *o4 = reinterpret_cast<float4 *>(S_final + soff + (size_t)(r0 + r) * dk + c0);
+        const float *Sr = S + r * dk + c0;
+        o4[0] = make_float4(Sr[0], Sr[1], Sr[2], Sr[3]);
+        o4[1] = make_float4(Sr[4], Sr[5], Sr[6], Sr[7]);
+    }
+    if (tid == 0)  // copies still in flight (error path) land before exit
+        for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait_bounded(&bar[i & 1], (i >> 1) & 1, kSpinF, err);
 }
 
 // o_i = S_t q_i for a tile of kTokTile tokens inside one frame.
@@ -250,11 +381,9 @@ frame_out_kernel(const Tin *__restrict__ q, const float *__restrict__ Sw, Tin *_
 }
 
 // ---------------------------------------------------------------- tensor cores
-using namespace sm100;
 constexpr int kTD = 128;                 // d_k = d_v on the tensor-core passes
 constexpr int kGT = 64;                  // tokens per Gram tile (K = 64 per tile)
 constexpr uint32_t kGStage = 3 * 16384;  // K, V, gamma . K (bf16, two 64-column atoms each)
-constexpr uint32_t kSpinF = 1u << 24;
 
 // G_t = K^T (Gamma K) and C_t = V^T (Gamma K) on the tensor cores: M = N = 128
 // (features), K = the frame's tokens, 64 per tile, two TMA stages.  K and V
@@ -490,10 +619,12 @@ FrameLayout frame_layout(int B, int T, int H, int dk, int dv, int n) {
 bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
 
 bool frame_shape_ok(int dk, int dv) {
-    return dk >= 16 && dk <= 128 && dk % 8 == 0 && dv >= 8 && dv <= 128 && dv % 8 == 0;
+    return dk >= 16 && dk <= 128 && dk % 16 == 0 && dv >= 8 && dv <= 128 && dv % 8 == 0;
 }
 
-size_t affine_smem(int dk, int dv) { return sizeof(float) * (size_t)(dk + dk + dv) * (dk + 1); }
+size_t affine_smem(int dk, int dv) {
+    return sizeof(float) * ((size_t)dk * (dk + 4) + (size_t)(dk + dv) * (dk + 1));
+}
 
 bool frame_tc_applies(const Dims &d, bool bf16) { return bf16 && d.dk == kTD && d.dv == kTD; }
 
@@ -520,7 +651,7 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
     }
     const size_t sm_gram = sizeof(float) * (size_t)(kTokTile * (d.dk + 1) + kTokTile * (d.dv + 1) + kTokTile);
     const size_t sm_aff = affine_smem(d.dk, d.dv);
-    const size_t sm_chain = sizeof(float) * (size_t)(d.dk + 2 * kChainRows) * (d.dk + 1);
+    const size_t sm_chain = sizeof(float) * (size_t)(2 * d.dk * d.dk + kChainRows * d.dk) + 64;
     const size_t sm_out = sizeof(float) * (size_t)(d.dv + kTokTile) * (d.dk + 1);
     if ((e = cudaFuncSetAttribute(frame_gram_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gram)) ||
         (e = cudaFuncSetAttribute(frame_affine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_aff)) ||
@@ -551,7 +682,8 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
     {
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_CHAIN, st);
         const dim3 gc((unsigned)(d.B * d.H), (unsigned)((d.dv + kChainRows - 1) / kChainRows));
-        frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, S0, Sw, tc ? Sb : nullptr, S_final, d);
+        frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, S0, Sw, tc ? Sb : nullptr, S_final, d,
+                                                           err);
         gdr_host::prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

@@ -227,7 +227,7 @@ gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, con
  *                           reports GDR_ERR_INVALID)
  *  g        [B, F, H] or [B, F, H, d_k] fp32 log-decay per frame, F = ceil(T / n)
  *  S0       [B, H, d_v, d_k] fp32 or NULL (zero);  S_final likewise or NULL
- *  d_k a multiple of 8 in [16, 128]; d_v a multiple of 8 in [8, 128]
+ *  d_k a multiple of 16 in [16, 128]; d_v a multiple of 8 in [8, 128]
  *  workspace: gdr_fwd_frame_workspace_size(B, T, H, d_k, d_v, n) bytes,
  *           caller-owned device memory (per frame: G/M_t, C/N_t and S_t, fp32).
  * fp32 arithmetic on the CUDA cores.  Errors as gdr_fwd.
