@@ -42,10 +42,10 @@ SM_COUNT = 148
 _TC_SRC = ('csrc/fwd_tc.cu', 'csrc/sm100.cuh', 'csrc/common.cuh')
 _DEC_SRC = ('csrc/decode.cu', 'csrc/common.cuh')
 NCU_TRAFFIC = {
-    ("tc_wy", "gdn_prefill"): (_TC_SRC, "53402063a98e7810", 206.236928e6 + 254.719488e6),
-    ("tc_state", "gdn_prefill"): (_TC_SRC, "53402063a98e7810", 308.370432e6 + 57.609728e6),
-    ("tc_wy", "kda_prefill"): (_TC_SRC, "53402063a98e7810", 680.951040e6 + 565.304576e6),
-    ("decode", "decode"): (_DEC_SRC, "9fc20c5d1e64ce78", 543.248896e6 + 482.370048e6),
+    ("tc_wy", "gdn_prefill"): (_TC_SRC, "ab41361bf6724bc7", 206.262272e6 + 256.316672e6),
+    ("tc_state", "gdn_prefill"): (_TC_SRC, "ab41361bf6724bc7", 308.345088e6 + 57.322240e6),
+    ("tc_wy", "kda_prefill"): (_TC_SRC, "ab41361bf6724bc7", 681.604608e6 + 565.627648e6),
+    ("decode", "decode"): (_DEC_SRC, "82e1f5016f476188", 543.250944e6 + 482.361600e6),
 }
 
 
