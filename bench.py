@@ -104,6 +104,18 @@ def prefill_min_bytes(cfg, n_seq):
     return th * per + states
 
 
+def prefill_kernel_min_bytes(cfg, n_seq, kernel):
+    """A prefill kernel's share of prefill_min_bytes: the WY pass reads the
+    token inputs (q, k, v, g and beta or the GDN-2 gates) once; the state pass
+    reads S0 and writes out and S_final once."""
+    e = 2 if cfg.dtype == "bf16" else 4
+    th = cfg.B * cfg.T * cfg.H
+    states = n_seq * cfg.H * cfg.d_k * cfg.d_v * 4 * ((1 if cfg.s0_var > 0 else 0) + 1)
+    out = th * cfg.d_v * e
+    total = prefill_min_bytes(cfg, n_seq)
+    return total - out - states if kernel == "tc_wy" else out + states
+
+
 def decode_bytes(cfg):
     e = 2 if cfg.dtype == "bf16" else 4
     heads = cfg.N * cfg.H
@@ -579,14 +591,27 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                 "frac_of_8TBps_spec": ach / 8000.0}
         conf["l2"] = "no flush: the 512 MiB state is larger than L2 and is streamed every step"
     elif is_frame:
+        # the dominant pass against its own roof: the token contractions (Gram,
+        # output) run on the tensor cores for bf16 d = 128, the factorisation and
+        # the chain are fp32 CUDA-core work
         th = cfg.B * cfg.T * cfg.H
-        flops = frame_flops_per_token_head(cfg.d_k, cfg.d_v, cfg.n) * th
-        peak = SM_COUNT * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        ach = flops / (ms * 1e-3) / 1e12
-        roof = {"bound": "alu", "kernel": "frame step (4 passes)", "achieved": ach, "peak": peak,
-                "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
-                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
-                "algorithmic_flops_per_launch": flops, "dominant_pass": dom}
+        fh = cfg.B * cfg.frames * cfg.H
+        dk, dv = cfg.d_k, cfg.d_v
+        tc_path = cfg.dtype == "bf16" and dk == 128 and dv == 128
+        pflops = {"frame_gram": 2 * dk * (dk + dv) * th, "frame_out": 2 * dk * dv * th,
+                  "frame_solve": (dk ** 3 / 3 + 2 * dk * dk * (dk + dv)) * fh,
+                  "frame_chain": 2 * dv * dk * dk * fh}
+        flops = pflops.get(dom, 0)
+        on_tc = tc_path and dom in ("frame_gram", "frame_out")
+        alu_peak = SM_COUNT * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        peak = peaks["bf16_tflops"] if on_tc else alu_peak
+        ach = flops / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor" if on_tc else "alu", "kernel": dom, "achieved": ach,
+                "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                "peak_source": (peak_kind + " bf16_tflops (burst)") if on_tc else
+                "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
+                "algorithmic_flops_per_launch": flops,
+                "step": {"tflops": frame_flops_per_token_head(dk, dv, cfg.n) * th / (ms * 1e-3) / 1e12}}
         conf["l2"] = (f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then a "
                       f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer, outside the "
                       "per-step CUDA-event intervals)")
@@ -604,12 +629,28 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                     "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
                     "algorithmic_flops_per_launch": flops}
         else:
-            peak = peaks["bf16_tflops"]
-            ach = flops / (dom_ms * 1e-3) / 1e12
-            roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak,
-                    "unit": "TFLOP/s", "frac": ach / peak, "traffic": ncu_traffic(dom, name),
-                    "peak_source": peak_kind + " bf16_tflops (burst)",
-                    "algorithmic_flops_per_launch": flops}
+            # Both roofs of the kernel's share of the step's algorithmic work: its
+            # share of the chunk GEMM flops, and its share of the minimum bytes
+            # (the WY pass reads the inputs once, the state pass reads S0 and
+            # writes out and S_final once).  The binding roof is the one that
+            # takes longer at the measured peaks.
+            sh_bytes = prefill_kernel_min_bytes(cfg, run.n_seq, dom)
+            t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+            t_hbm = sh_bytes / (peaks["hbm_gbs"] * 1e9)
+            sec = dom_ms * 1e-3
+            tc = {"achieved": flops / sec / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                  "frac": flops / sec / 1e12 / peaks["bf16_tflops"],
+                  "algorithmic_flops_per_launch": flops,
+                  "peak_source": peak_kind + " bf16_tflops (burst)"}
+            hb = {"achieved": sh_bytes / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                  "frac": sh_bytes / sec / 1e9 / peaks["hbm_gbs"],
+                  "algorithmic_bytes_per_launch": sh_bytes,
+                  "peak_source": peak_kind + " hbm_gbs"}
+            top = hb if t_hbm > t_tc else tc
+            roof = {"bound": "hbm" if t_hbm > t_tc else "tensor", "kernel": dom,
+                    "achieved": top["achieved"], "peak": top["peak"], "unit": top["unit"],
+                    "frac": top["frac"], "traffic": ncu_traffic(dom, name),
+                    "peak_source": top["peak_source"], "tensor_view": tc, "hbm_view": hb}
         min_bytes = prefill_min_bytes(cfg, run.n_seq)
         roof["step"] = {"tflops": f_all * th / (ms * 1e-3) / 1e12,
                         "tc_frac": f_all * th / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
