@@ -690,7 +690,8 @@ def main():
     ap.add_argument("--workload", default="gdn_prefill",
                     choices=list(inputs.PREFILL) + list(inputs.DECODE) + list(inputs.FRAME))
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
-    ap.add_argument("--extra", default="decode,kda_prefill,varlen_prefill,gdp_prefill,gdn2_prefill,frame_prefill",
+    ap.add_argument("--extra", default=("decode,kda_decode,kda_prefill,varlen_prefill,gdp_prefill,"
+                                        "gdn2_prefill,frame_prefill,gdn_prefill_c16,gdn_prefill_c128"),
                     help="comma-separated workloads measured after the main one ('' for none)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -720,7 +721,7 @@ def main():
                            args.steps, args.warmup, not args.no_cpu, not args.no_e2e, sampler)
         extra = {}
         for name in [x for x in args.extra.split(",") if x and x != args.workload]:
-            steps = 20 if name != "decode" else 200
+            steps = 200 if name in inputs.DECODE else 20
             r = measure(args, name, device, rank, world, peaks, peak_kind, args.path, steps, 3,
                         False, False, None)
             extra[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],

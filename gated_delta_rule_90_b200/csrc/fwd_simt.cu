@@ -241,14 +241,297 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     }
 }
 
+// ------------------------------------------------------------------ wide chunks
+// The same chunk algorithm for chunks whose resident tiles do not fit in
+// shared memory (C = 128 with d_k = 128 would need 380 to 510 KB above).
+// Only the C x C matrices, the CTA's state rows and the P/Z tiles stay
+// resident; the chunk's key-side inputs (k, q, g and the erase vectors) pass
+// through shared memory in blocks of kWideKB key channels, twice per chunk:
+//   pass 1, per block: L and A accumulate their partial channel sums (the
+//           decay ratio exp(G_lc - G_mc) formed per channel as above), then the
+//           block is decayed in place and K<- S^T, Q<- S^T accumulate in
+//           registers;
+//   solve:  (I + N) T = diag(beta) column by column, T stored transposed in
+//           the strict upper triangle of N's buffer (T's diagonal is beta);
+//   Z = T P, O = Q<- S^T + A Z;
+//   pass 2, per block: K-> formed in place, S's columns of the block updated.
+// Every product is the one the resident kernel forms; only the order of the
+// channel sums differs.
+constexpr int kWideKB = 16;    // key channels per block
+constexpr int kWideMaxC = 128;
+constexpr int kWideRegs = kWideMaxC * kSimtRows / kSimtThreads;  // P / Q<-S^T entries per thread
+constexpr int kWideSegs = kSimtThreads / kWideKB;                // scan segments per channel
+
+struct WideSmem {
+    int NT, Am, Kb, Qb, Gb, Eb, Pm, Zm, Ss, bt, Gs, seg, total;
+    int bst, sst;  // row strides of the channel blocks and of the state rows
+};
+
+__host__ __device__ inline WideSmem wide_layout(int C, int dk, bool channel, bool dec) {
+    WideSmem L;
+    L.bst = kWideKB + 1;
+    L.sst = dk + 1;
+    int o = 0;
+    L.NT = o; o += C * C;
+    L.Am = o; o += C * C;
+    L.Kb = o; o += C * L.bst;
+    L.Qb = o; o += C * L.bst;
+    L.Gb = o; o += channel ? C * L.bst : 0;
+    L.Eb = o; o += dec ? C * L.bst : 0;
+    L.Pm = o; o += C * kSimtRows;
+    L.Zm = o; o += C * kSimtRows;
+    L.Ss = o; o += kSimtRows * L.sst;
+    L.bt = o; o += C;
+    L.Gs = o; o += C;
+    L.seg = o; o += kWideSegs * kWideKB;
+    L.total = o;
+    return L;
+}
+
+// Row l and column m (m <= l) of the p-th entry of a row-major lower triangle.
+__device__ __forceinline__ void tri_index(int p, int &l, int &m) {
+    int r = (int)((sqrtf(8.f * (float)p + 1.f) - 1.f) * 0.5f);
+    while ((r + 1) * (r + 2) / 2 <= p) ++r;
+    while (r * (r + 1) / 2 > p) --r;
+    l = r;
+    m = p - r * (r + 1) / 2;
+}
+
+template <typename Tin, bool CH, bool DEC>
+__global__ void __launch_bounds__(kSimtThreads)
+fwd_simt_wide_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                     const float *__restrict__ g, const float *__restrict__ beta,
+                     const float *__restrict__ eg, const float *__restrict__ wg,
+                     const float *__restrict__ S0, Tin *__restrict__ out, float *__restrict__ S_final,
+                     int T, int H, int dk, int dv, int C, const int32_t *__restrict__ cu,
+                     int T_total) {
+    extern __shared__ float sm[];
+    const WideSmem L = wide_layout(C, dk, CH, DEC);
+    float *NT = sm + L.NT, *Am = sm + L.Am, *Kb = sm + L.Kb, *Qb = sm + L.Qb, *Gb = sm + L.Gb;
+    float *Eb = sm + L.Eb, *Pm = sm + L.Pm, *Zm = sm + L.Zm, *Ss = sm + L.Ss, *bt = sm + L.bt;
+    float *Gs = sm + L.Gs, *seg = sm + L.seg;
+    const int bst = L.bst, sst = L.sst;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int s = blockIdx.x / H, h = blockIdx.x % H;
+    const int r0 = blockIdx.y * kSimtRows;
+    const int nr = min(kSimtRows, dv - r0);
+    const int npairs = C * (C + 1) / 2;
+    const int seglen = (C + kWideSegs - 1) / kWideSegs;
+    long t0, t1;
+    seq_bounds(cu, s, T, T_total, t0, t1);
+
+    const size_t soff = ((size_t)s * H + h) * (size_t)dv * dk;
+    for (int e = tid; e < kSimtRows * dk; e += kSimtThreads) {
+        const int r = e / dk, c = e % dk;
+        Ss[r * sst + c] = (S0 && r < nr) ? S0[soff + (size_t)(r0 + r) * dk + c] : 0.f;
+    }
+
+    // Load channels [cb, cb + kWideKB) of the chunk's keys (and queries, gate,
+    // erase vectors); with CH the gate block becomes its cumulative sum over
+    // the chunk.  Ends with the block visible to the whole CTA.
+    auto load_block = [&](long c0, int len, int cb, bool with_q) {
+        for (int i = tid; i < C * kWideKB; i += kSimtThreads) {
+            const int l = i / kWideKB, c = i % kWideKB;
+            float kv = 0.f, qv = 0.f, gv = 0.f, ev = 0.f;
+            if (l < len) {
+                const size_t off = ((size_t)(c0 + l) * H + h) * dk + cb + c;
+                kv = ld_in(k, off);
+                if (with_q) qv = ld_in(q, off);
+                if (CH) gv = g[off];
+                if (DEC) ev = kv * eg[off];
+            }
+            Kb[l * bst + c] = kv;
+            if (with_q) Qb[l * bst + c] = qv;
+            if (CH) Gb[l * bst + c] = gv;
+            if (DEC) Eb[l * bst + c] = ev;
+        }
+        __syncthreads();
+        if (CH) {  // segmented scan: channel tid % KB, rows of segment tid / KB
+            const int c = tid % kWideKB, sg = tid / kWideKB;
+            const int la = sg * seglen, lb = min(C, la + seglen);
+            float acc = 0.f;
+            for (int l = la; l < lb; ++l) {
+                acc += Gb[l * bst + c];
+                Gb[l * bst + c] = acc;
+            }
+            seg[sg * kWideKB + c] = acc;
+            __syncthreads();
+            float pre = 0.f;
+            for (int j = 0; j < sg; ++j) pre += seg[j * kWideKB + c];
+            for (int l = la; l < lb; ++l) Gb[l * bst + c] += pre;
+            __syncthreads();
+        }
+    };
+
+    for (long c0 = t0; c0 < t1; c0 += C) {
+        const int len = (int)min((long)C, t1 - c0);
+        __syncthreads();  // the previous chunk is done with every buffer
+        for (int l = tid; l < C; l += kSimtThreads) {
+            const size_t off = (size_t)(c0 + l) * H + h;
+            bt[l] = (l < len) ? (DEC ? 1.f : beta[off]) : 0.f;
+            if (!CH) Gs[l] = (l < len) ? g[off] : 0.f;
+        }
+        __syncthreads();
+        if (!CH && tid == 0) {
+            float acc = 0.f;
+            for (int l = 0; l < C; ++l) {
+                acc += Gs[l];
+                Gs[l] = acc;
+            }
+        }
+        // ---- pass 1: L, A (shared memory), K<- S^T and Q<- S^T (registers) ----
+        float pacc[kWideRegs], qacc[kWideRegs];
+#pragma unroll
+        for (int i = 0; i < kWideRegs; ++i) pacc[i] = qacc[i] = 0.f;
+        const float *Rb = DEC ? Eb : Kb;  // reading direction
+        for (int cb = 0; cb < dk; cb += kWideKB) {
+            load_block(c0, len, cb, true);
+            for (int p = tid; p < npairs; p += kSimtThreads) {
+                int l, m;
+                tri_index(p, l, m);
+                float lv = 0.f, av = 0.f;
+#pragma unroll 4
+                for (int c = 0; c < kWideKB; ++c) {
+                    float w = Kb[m * bst + c];
+                    if (CH) w *= expf(Gb[l * bst + c] - Gb[m * bst + c]);
+                    lv = fmaf(Rb[l * bst + c], w, lv);
+                    av = fmaf(Qb[l * bst + c], w, av);
+                }
+                if (cb) {
+                    lv += NT[l * C + m];
+                    av += Am[l * C + m];
+                }
+                NT[l * C + m] = lv;  // the diagonal is overwritten below
+                Am[l * C + m] = av;
+            }
+            if (CH) {  // decay the block in place: K<- (or E<-) and Q<-
+                __syncthreads();
+                for (int i = tid; i < C * kWideKB; i += kSimtThreads) {
+                    const int l = i / kWideKB, c = i % kWideKB;
+                    const float w = expf(Gb[l * bst + c]);
+                    Qb[l * bst + c] *= w;
+                    if (DEC) Eb[l * bst + c] *= w;
+                    else Kb[l * bst + c] *= w;
+                }
+                __syncthreads();
+            }
+#pragma unroll
+            for (int i = 0; i < kWideRegs; ++i) {
+                const int l = warp + (kSimtThreads / kSimtRows) * i;
+                if (l < C) {
+                    float pa = pacc[i], qa = qacc[i];
+#pragma unroll 4
+                    for (int c = 0; c < kWideKB; ++c) {
+                        const float sv = Ss[lane * sst + cb + c];
+                        pa = fmaf(Rb[l * bst + c], sv, pa);
+                        qa = fmaf(Qb[l * bst + c], sv, qa);
+                    }
+                    pacc[i] = pa;
+                    qacc[i] = qa;
+                }
+            }
+            __syncthreads();  // the next block overwrites this one
+        }
+        // ---- finish L -> N = diag(beta) L and A; P = V - K<- S^T ----
+        for (int p = tid; p < npairs; p += kSimtThreads) {
+            int l, m;
+            tri_index(p, l, m);
+            const float w = CH ? 1.f : expf(Gs[l] - Gs[m]);
+            NT[l * C + m] = (m < l) ? bt[l] * NT[l * C + m] * w : 0.f;
+            Am[l * C + m] *= w;
+        }
+#pragma unroll
+        for (int i = 0; i < kWideRegs; ++i) {
+            const int l = warp + (kSimtThreads / kSimtRows) * i;
+            if (l < C) {
+                float pv = 0.f;
+                if (lane < nr && l < len) {
+                    const float dl = CH ? 1.f : expf(Gs[l]);
+                    const size_t vo = ((size_t)(c0 + l) * H + h) * dv + r0 + lane;
+                    pv = (DEC ? ld_in(v, vo) * wg[vo] : ld_in(v, vo)) - dl * pacc[i];
+                    qacc[i] *= dl;
+                }
+                Pm[l * kSimtRows + lane] = pv;
+            }
+        }
+        __syncthreads();
+        // ---- T: (I + N) T = diag(beta); T[i][j] (i > j) goes to NT[j][i] ----
+        for (int j = tid; j < C; j += kSimtThreads) {
+            const float bj = bt[j];
+            for (int i = j + 1; i < C; ++i) {
+                float acc = -NT[i * C + j] * bj;
+                for (int m = j + 1; m < i; ++m) acc = fmaf(-NT[i * C + m], NT[j * C + m], acc);
+                NT[j * C + i] = acc;
+            }
+        }
+        __syncthreads();
+        // ---- Z = T P ----
+#pragma unroll
+        for (int i = 0; i < kWideRegs; ++i) {
+            const int l = warp + (kSimtThreads / kSimtRows) * i;
+            if (l < C) {
+                float z = bt[l] * Pm[l * kSimtRows + lane];
+                for (int m = 0; m < l; ++m) z = fmaf(NT[m * C + l], Pm[m * kSimtRows + lane], z);
+                Zm[l * kSimtRows + lane] = z;
+            }
+        }
+        __syncthreads();
+        // ---- O = Q<- S^T + A Z ----
+#pragma unroll
+        for (int i = 0; i < kWideRegs; ++i) {
+            const int l = warp + (kSimtThreads / kSimtRows) * i;
+            if (l < len && lane < nr) {
+                float o = qacc[i];
+                for (int m = 0; m <= l; ++m) o = fmaf(Am[l * C + m], Zm[m * kSimtRows + lane], o);
+                st_out(out, ((size_t)(c0 + l) * H + h) * dv + r0 + lane, o);
+            }
+        }
+        // ---- pass 2: S <- S Diag(exp(G_C)) + Z^T K-> ----
+        for (int cb = 0; cb < dk; cb += kWideKB) {
+            __syncthreads();  // Kb / Gb free
+            load_block(c0, len, cb, false);
+            for (int i = tid; i < C * kWideKB; i += kSimtThreads) {
+                const int l = i / kWideKB, c = i % kWideKB;
+                const float gap = CH ? Gb[(C - 1) * bst + c] - Gb[l * bst + c] : Gs[C - 1] - Gs[l];
+                Kb[l * bst + c] *= expf(gap);
+            }
+            __syncthreads();
+            for (int i = tid; i < kSimtRows * kWideKB; i += kSimtThreads) {
+                const int r = i / kWideKB, c = i % kWideKB;
+                const float gC = CH ? Gb[(C - 1) * bst + c] : Gs[C - 1];
+                float acc = Ss[r * sst + cb + c] * expf(gC);
+                for (int l = 0; l < C; ++l) acc = fmaf(Zm[l * kSimtRows + r], Kb[l * bst + c], acc);
+                Ss[r * sst + cb + c] = acc;
+            }
+        }
+    }
+    __syncthreads();
+    if (S_final) {
+        for (int e = tid; e < nr * dk; e += kSimtThreads) {
+            const int r = e / dk, c = e % dk;
+            S_final[soff + (size_t)(r0 + r) * dk + c] = Ss[r * sst + c];
+        }
+    }
+}
+
 }  // namespace gdr
 
 using namespace gdr;
 
 namespace gdr_host {
 
+static constexpr size_t kSimtSmemCap = 227u * 1024u;
+
+// The resident layout where it fits, else the channel-blocked one.
+static bool simt_wide(int C, int dk, bool channel, bool dec) {
+    return sizeof(float) * (size_t)simt_layout(C, dk, channel, dec).total > kSimtSmemCap;
+}
+
 size_t simt_smem_bytes(int C, int dk, bool channel, bool dec) {
-    return sizeof(float) * (size_t)simt_layout(C, dk, channel, dec).total;
+    if (!simt_wide(C, dk, channel, dec))
+        return sizeof(float) * (size_t)simt_layout(C, dk, channel, dec).total;
+    if (C > kWideMaxC || dk % kWideKB) return SIZE_MAX;
+    return sizeof(float) * (size_t)wide_layout(C, dk, channel, dec).total;
 }
 
 template <typename Tin, bool CH, bool DEC = false>
@@ -258,11 +541,13 @@ static cudaError_t launch_simt(const void *q, const void *k, const void *v, cons
                                int T_total, cudaStream_t st, const float *eg = nullptr,
                                const float *wg = nullptr) {
     const size_t smem = simt_smem_bytes(C, dk, CH, DEC);
-    cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<Tin, CH, DEC>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool wide = simt_wide(C, dk, CH, DEC);
+    auto kern = wide ? fwd_simt_wide_kernel<Tin, CH, DEC> : fwd_simt_kernel<Tin, CH, DEC>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(n_seq * H), (unsigned)((dv + kSimtRows - 1) / kSimtRows));
-    fwd_simt_kernel<Tin, CH, DEC><<<grid, kSimtThreads, smem, st>>>(
+    kern<<<grid, kSimtThreads, smem, st>>>(
         (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, eg, wg, S0, (Tin *)out, S_final,
         T, H, dk, dv, C, cu, T_total);
     return cudaGetLastError();

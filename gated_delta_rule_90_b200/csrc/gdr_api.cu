@@ -115,7 +115,7 @@ bool valid_enum(gdr_dtype d, gdr_gate g) {
 
 bool simt_shape_ok(int dk, int dv, int chunk) {
     return dk >= 16 && dk <= 128 && dk % 16 == 0 && dv >= 16 && dv <= 128 && dv % 16 == 0 &&
-           (chunk == 16 || chunk == 32 || chunk == 64);
+           (chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128);
 }
 
 // Resolve the path; returns GDR_OK and sets *use_tc, or an error.

@@ -88,7 +88,11 @@ size_t gdr_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk, 
  *  out      [B, T, H, d_v]   dtype, written for every token
  *           (with B*T == 0 the token tensors may be NULL; S_final = S0)
  *  S_final  [N, H, d_v, d_k] fp32 final states, or NULL to skip
- *  chunk    16, 32 or 64 (SIMT); 64 (tensor-core path)
+ *  chunk    16, 32, 64 or 128 (SIMT); 64 (tensor-core path).  Every chunk size
+ *           gives the token recurrence's result up to rounding.  At 128 the
+ *           SIMT path streams the chunk's key channels through shared memory
+ *           in blocks of 16 (one CTA per SM); smaller chunks keep whole tiles
+ *           resident.
  *  cu_seqlens  NULL: N = B sequences of length T.  Otherwise a DEVICE int32
  *           array [n_seq + 1] of token offsets into a packed batch (B must be
  *           1, cu_seqlens[0] = 0, cu_seqlens[n_seq] = T, non-decreasing); the
@@ -191,8 +195,8 @@ gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const fl
  *  b        [B, T, H, d_k]   fp32 erase gate;  w [B, T, H, d_v] fp32 write gate
  *  S0, S_final, cu_seqlens, n_seq, chunk, path, workspace: as for gdr_fwd.  The
  *  tensor-core path takes bf16 with d_k = d_v = 128, chunk 64 and the
- *  per-channel decay (the page's setting); everything else (chunk 16, 32 or
- *  64, d_k, d_v multiples of 16 up to 128) runs on the CUDA cores in fp32.
+ *  per-channel decay (the page's setting); everything else (chunk 16, 32, 64
+ *  or 128, d_k, d_v multiples of 16 up to 128) runs on the CUDA cores in fp32.
  *  gdr_fwd_gdn2_workspace_size gives the workspace (0 on the CUDA-core path).
  * gdr_decode_step_gdn2: one token per sequence in place on S_inout, with
  *  b [N, H, d_k] and w [N, H, d_v]; otherwise as gdr_decode_step.

@@ -68,7 +68,8 @@ def fwd(**kw):
     (dict(dtype=7), 1), (dict(gate=3), 1), (dict(path=9), 1),
     (dict(q=ctypes.c_void_p(0x10004)), 1), (dict(S_final=ctypes.c_void_p(0x10008)), 1),
     (dict(cu=P, B=2, n_seq=2), 1), (dict(cu=P, B=1, n_seq=0), 1),
-    (dict(dk=256, dv=64), 2), (dict(dk=24), 2), (dict(chunk=128), 2),
+    (dict(dk=256, dv=64), 2), (dict(dk=24), 2), (dict(chunk=256), 1),
+    (dict(chunk=128, path=2, dtype=1, dk=128, dv=128), 2),
     (dict(path=2, dtype=0), 2), (dict(path=2, dtype=1, dk=64, dv=64), 2),
 ])
 def test_fwd_rejects_on_host(kw, expect):
@@ -139,7 +140,8 @@ def test_product_workspace_holds_the_virtual_sequence():
 
 @nogpu
 @pytest.mark.parametrize("kw,expect", [
-    (dict(b=None), 1), (dict(dk=72), 2), (dict(chunk=128), 2), (dict(chunk=48), 1),
+    (dict(b=None), 1), (dict(dk=72), 2), (dict(chunk=48), 1),
+    (dict(chunk=128, dtype=1, dk=128, dv=128, path=2), 2),
     (dict(w=ctypes.c_void_p(0x10008)), 1), (dict(cu=P, B=2), 1), (dict(gate=3), 1),
     (dict(path=2), 2), (dict(dtype=1, dk=128, dv=128, path=2), 1), (dict(path=7), 1),
 ])

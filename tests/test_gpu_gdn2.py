@@ -42,7 +42,7 @@ def check(inp, dev, chunk=None, path="auto"):
     assert eo <= tol and es <= tol, (eo, es)
 
 
-@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
 @pytest.mark.parametrize("gate", ["scalar", "channel"])
 def test_gdn2_fp32_every_chunk_size(cuda_device, chunk, gate):
     cfg = cfg_of(B=2, T=203, H=2, d_k=64, d_v=48, dtype="f32", gate=gate,
@@ -51,10 +51,11 @@ def test_gdn2_fp32_every_chunk_size(cuda_device, chunk, gate):
 
 
 @pytest.mark.parametrize("gate", ["scalar", "channel"])
-def test_gdn2_bf16_d128(cuda_device, gate):
+@pytest.mark.parametrize("chunk", [64, 128])
+def test_gdn2_bf16_d128(cuda_device, gate, chunk):
     cfg = cfg_of(B=2, T=300, H=3, gate=gate, gate_scale=0.1 if gate == "scalar" else 0.05,
                  s0_var=0.01)
-    check(inputs.gdn2_inputs(cfg, seed=602), cuda_device)
+    check(inputs.gdn2_inputs(cfg, seed=602), cuda_device, chunk)
 
 
 @pytest.mark.parametrize("T", [64, 300, 1])

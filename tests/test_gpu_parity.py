@@ -57,7 +57,7 @@ def test_tiny_fp32_workload(cuda_device):
     check(inputs.prefill_inputs(inputs.PREFILL["tiny_fp32"]), cuda_device)
 
 
-@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
 @pytest.mark.parametrize("gate", ["scalar", "channel"])
 def test_simt_fp32_every_chunk_size(cuda_device, chunk, gate):
     cfg = small_cfg(B=2, T=203, H=2, d_k=64, d_v=48, dtype="f32", gate=gate, chunk=chunk,
@@ -71,14 +71,32 @@ def test_simt_bf16_d128(cuda_device, gate):
     check(inputs.prefill_inputs(cfg, seed=102), cuda_device, path="simt")
 
 
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_simt_bf16_d128_chunk128(cuda_device, gate):
+    """Chunk 128 at d = 128: the channel-blocked kernel (two full chunks and a
+    44-token tail per sequence)."""
+    cfg = small_cfg(B=2, T=300, H=3, gate=gate, gate_scale=0.1 if gate == "scalar" else 0.05,
+                    chunk=128)
+    check(inputs.prefill_inputs(cfg, seed=105), cuda_device)
+
+
+def test_simt_chunk128_fp32_d128_strong_gates(cuda_device):
+    """fp32 at d = 128, chunk 128, with decays strong enough that a whole chunk
+    spans several orders of magnitude: the per-channel ratios stay formed from
+    differences of cumulative sums."""
+    cfg = small_cfg(B=1, T=257, H=2, dtype="f32", gate="channel", gate_scale=0.3, chunk=128)
+    check(inputs.prefill_inputs(cfg, seed=106), cuda_device)
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_simt_varlen_with_empty_and_unit_sequences(cuda_device, dtype):
+@pytest.mark.parametrize("chunk", [32, 128])
+def test_simt_varlen_with_empty_and_unit_sequences(cuda_device, dtype, chunk):
     cfg = inputs.PREFILL["varlen_prefill"].replace(T=400, H=2, d_k=64, d_v=64, dtype=dtype,
                                                    n_seq=0, s0_var=0.01)
     inp = inputs.prefill_inputs(cfg, seed=103)
     inp.cu_seqlens = np.array([0, 0, 1, 65, 129, 200, 200, 400], dtype=np.int32)
     inp.S0 = np.random.default_rng(5).standard_normal((7, 2, 64, 64)).astype(np.float32) * 0.1
-    check(inp, cuda_device, path="simt", chunk=32)
+    check(inp, cuda_device, path="simt", chunk=chunk)
 
 
 def test_simt_zero_length_batch_copies_state(cuda_device):
@@ -177,10 +195,12 @@ def test_decode_small(cuda_device, dtype, gate, dk, dv):
     assert eo <= TOL[dtype] and es <= TOL[dtype], (eo, es)
 
 
-def test_decode_full_size_sampled(cuda_device):
-    """The decode workload at full size (256 x 32 heads, d = 128) for 1000
-    steps; the oracle follows a fixed sample of 8 sequences x 8 heads."""
-    cfg = inputs.DECODE["decode"]
+@pytest.mark.parametrize("name", ["decode", "kda_decode"])
+def test_decode_full_size_sampled(cuda_device, name):
+    """The decode workloads at full size (256 x 32 heads, d = 128; scalar and
+    per-key-channel decay) for 1000 steps; the oracle follows a fixed sample of
+    8 sequences x 8 heads."""
+    cfg = inputs.DECODE[name]
     dev = cuda_device
     S = inputs.decode_state(cfg)
     Sd = torch.from_numpy(S).to(dev)
