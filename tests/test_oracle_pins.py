@@ -186,13 +186,13 @@ def pin_swap_is_reflection(impl):
 def pin_chunkwise_equals_recurrence(impl):
     """Every chunk size gives the exact result ("Linear Attention, Visualized",
     Chunkwise algorithm / Cost): the independent chunkwise WY/UT form
-    (oracle.chunked) agrees at C in {1, 16, 37, 64}, with a partial last chunk,
+    (oracle.chunked) agrees at C in {1, 16, 37, 64, 128}, with a partial last chunk,
     scalar and per-channel gates, nonzero S0 and a packed variable-length
     batch."""
     for gate in ("scalar", "channel"):
         q, k, v, g, b, S0 = rand_case(5, B=1, T=150, H=1, dk=6, dv=4, gate=gate, g_scale=0.1)
         O, SF = impl(q, k, v, g, b, S0)
-        for C in (1, 16, 37, 64):
+        for C in (1, 16, 37, 64, 128):
             Oc, SFc = chunked_fwd(q, k, v, g, b, C, S0=S0)
             assert rel(Oc, O) < 1e-11 and rel(SFc, SF) < 1e-11, (gate, C)
     q, k, v, g, b, _ = rand_case(6, B=1, T=90, H=2, dk=5, dv=3, g_scale=0.2)
