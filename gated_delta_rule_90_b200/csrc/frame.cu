@@ -10,18 +10,18 @@
 // with the frame's decay D_t applied first (the forget gate sits at frame
 // boundaries).  Every query of frame t reads S_t: o_i = S_t q_i.
 //
-// I + G_t is symmetric positive definite, so the page factorises it (Cholesky)
-// and solves.  The step is affine in S_{t-1}:
-//     S_t = S_{t-1} M_t + N_t,   M_t = D_t (I + G_t)^-1,   N_t = C_t (I + G_t)^-1,
+// I + G_t is symmetric positive definite (the page factorises it by Cholesky
+// and solves).  The step is affine in S_{t-1}:
+//     S_t = (S_{t-1} D_t + C_t) W_t,   W_t = (I + G_t)^-1,
 // and everything except the product chain over frames is independent per
 // frame.  Four passes:
-//   frame_gram   (frame, head, batch)    G_t, C_t                    fp32
-//   frame_affine (frame, head, batch)    Cholesky of I + G_t, then M_t, N_t by
-//                                        forward/backward substitution
-//   frame_chain  (batch*head, row block) S_t = S_{t-1} M_t + N_t over the frames
-//                                        (rows of S are independent)
-//   frame_out    (token tile, head, batch) o_i = S_t q_i
-// The factorisation, the affine pair and the chain are fp32 on the CUDA cores.
+//   frame_gram    (frame, head, batch)    G_t, C_t                    fp32
+//   frame_inverse (frame, head, batch)    W_t by the symmetric sweep
+//                                         (Gauss-Jordan) of I + G_t
+//   frame_chain   (batch*head, row block) S_t = (S_{t-1} D_t + C_t) W_t over
+//                                         the frames (rows of S are independent)
+//   frame_out     (token tile, head, batch) o_i = S_t q_i
+// The inverse and the chain are fp32 on the CUDA cores.
 // The two dense contractions over tokens -- the Gram pass and the output pass
 // -- run on the tensor cores for bf16 inputs with d_k = d_v = 128 (tcgen05,
 // operands staged by TMA, fp32 accumulators in TMEM), and on the CUDA cores
@@ -109,163 +109,111 @@ frame_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
     }
 }
 
-// Cholesky of I + G_t (right-looking, in shared memory), then the rows of
-// M_t = D_t (I + G_t)^-1 and N_t = C_t (I + G_t)^-1: each solves
-// x (L L^T) = r, i.e. y L^T = r (forward) and x L = y (backward), for all
-// d_k + d_v right-hand sides at once, one row per thread, blocked by 16
-// columns: the part of a block that depends on earlier blocks is a small GEMM
-// with 16 independent sums per thread, the rest a 16 x 16 triangular solve.
-// The forward pass reads L by columns, so the factorisation also stores L^T in
-// the free upper triangle.  M_t overwrites G_t and N_t overwrites C_t.
-constexpr int kAffB = 16;  // column block of the substitution
-__global__ void __launch_bounds__(kThreads)
-frame_affine_kernel(float *__restrict__ GM, float *__restrict__ CN, const float *__restrict__ g,
-                    int per_channel, Dims d, unsigned int *err) {
-    extern __shared__ float sm[];
+// W_t = (I + G_t)^-1 by the symmetric sweep (Gauss-Jordan) operator: sweeping
+// pivot k maps a_kk -> -1/a_kk, a_ik -> a_ik / a_kk, a_kj -> a_kj / a_kk and
+// a_ij -> a_ij - a_ik a_kj / a_kk; after every pivot the matrix is -(I + G_t)^-1.
+// I + G_t is symmetric with eigenvalues >= 1, so every pivot (a Schur
+// complement's diagonal) is >= 1 and no pivoting is needed.  G_t is
+// symmetrised as (G + G^T) / 2 on load, and each update a_ij -= (a_ik a_kj) /
+// a_kk is symmetric in i and j, so the matrix stays exactly symmetric and row
+// k stands in for column k.  Thread (row r, quarter) holds d_k / 4 entries of
+// row r in registers; the pivot row passes through a double buffer in shared
+// memory, written by its own row's threads during the previous step: one
+// barrier per pivot.  W_t overwrites G_t.
+constexpr int kSwThreads = 512;  // 4 threads per row, d_k <= 128
+template <int CW>  // columns per thread: d_k / 4
+__global__ void __launch_bounds__(kSwThreads, 2)
+frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
+    __shared__ __align__(16) float buf[2][128 + 16];  // pivot rows, +4 floats per quarter
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int dk = d.dk, ast = dk + 4, rst = dk + 1;  // A rows 16-byte aligned
-    const int nrhs = dk + d.dv;
-    float *A = sm, *R = A + dk * ast;  // R: nrhs rows of length dk (+1 pad)
-    const int tid = threadIdx.x;
+    const int dk = 4 * CW;
+    const int tid = threadIdx.x, r = tid >> 2, qd = tid & 3, j0 = qd * CW;
+    const bool act = r < dk;
     const size_t sl = slot(d, b, f, h);
-    float *Gp = GM + sl * (size_t)dk * dk, *Cp = CN + sl * (size_t)d.dv * dk;
-    const int q4 = dk / 4;
-#pragma unroll 4
-    for (int e = tid; e < dk * q4; e += kThreads) {  // A = I + G (16-byte loads)
-        const int i = e / q4, j = (e % q4) * 4;
-        const float4 x = reinterpret_cast<const float4 *>(Gp)[e];
-        float *Ai = A + i * ast + j;
-        Ai[0] = x.x + (i == j ? 1.f : 0.f);
-        Ai[1] = x.y + (i == j + 1 ? 1.f : 0.f);
-        Ai[2] = x.z + (i == j + 2 ? 1.f : 0.f);
-        Ai[3] = x.w + (i == j + 3 ? 1.f : 0.f);
-    }
-#pragma unroll 4
-    for (int e = tid; e < d.dv * q4; e += kThreads) {  // rows of C_t
-        const int i = e / q4, j = (e % q4) * 4;
-        const float4 x = reinterpret_cast<const float4 *>(Cp)[e];
-        float *Ri = R + (dk + i) * rst + j;
-        Ri[0] = x.x; Ri[1] = x.y; Ri[2] = x.z; Ri[3] = x.w;
-    }
-    for (int e = tid; e < dk * dk; e += kThreads) {  // rows of D_t
-        const int i = e / dk, j = e % dk;
-        const float a = per_channel ? __expf(g[sl * dk + i]) : __expf(g[sl]);
-        R[i * rst + j] = (i == j) ? a : 0.f;
-    }
-    __syncthreads();
-    // right-looking Cholesky: column j, then the trailing update; L^T mirrored
-    for (int j = 0; j < dk; ++j) {
-        const float ajj = A[j * ast + j];
-        const float ljj = sqrtf(fmaxf(ajj, 1e-30f));
-        __syncthreads();
-        if (tid == 0) {
-            if (!(ajj > 0.f)) atomicOr(err, kErrNumeric);
-            A[j * ast + j] = ljj;
+    float *Gp = GW + sl * (size_t)dk * dk;
+    // quarter q of a pivot row starts at q * (CW + 4): the quarters fall on
+    // different banks
+    const int pr = r + 4 * (r / CW), pj = j0 + 4 * qd;
+    float a[CW];
+    if (act) {
+#pragma unroll
+        for (int u4 = 0; u4 < CW / 4; ++u4) {
+            const float4 x = *reinterpret_cast<const float4 *>(Gp + (size_t)r * dk + j0 + 4 * u4);
+            a[4 * u4] = x.x; a[4 * u4 + 1] = x.y; a[4 * u4 + 2] = x.z; a[4 * u4 + 3] = x.w;
         }
-        for (int i = j + 1 + tid; i < dk; i += kThreads) {
-            const float lij = A[i * ast + j] / ljj;
-            A[i * ast + j] = lij;
-            A[j * ast + i] = lij;  // L^T in the upper triangle
+#pragma unroll
+        for (int u = 0; u < CW; ++u) {
+            const int j = j0 + u;
+            a[u] = 0.5f * (a[u] + Gp[(size_t)j * dk + r]) + (j == r ? 1.f : 0.f);
         }
-        __syncthreads();
-        // trailing update A[i][c] -= L[i][j] L[c][j] for i, c > j: a warp per
-        // row, lanes along c, L[c][j] read from the mirrored row j.  The whole
-        // square is updated; its upper part is rewritten by later mirror rows.
-        // Each lane keeps its four L[c][j] in registers; rows are unrolled so
-        // that the loads of several rows are in flight together.
-        const int warp = tid >> 5, lane = tid & 31;
-        float lj[4];
+        if (r == 0) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int c = lane + 32 * u;
-            lj[u] = (c > j && c < dk) ? A[j * ast + c] : 0.f;
-        }
-#pragma unroll 4
-        for (int i = j + 1 + warp; i < dk; i += kThreads / 32) {
-            const float lij = A[i * ast + j];
-            float *Ai = A + i * ast;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int c = lane + 32 * u;
-                if (c > j && c < dk) Ai[c] = fmaf(-lij, lj[u], Ai[c]);
-            }
-        }
-        __syncthreads();
-    }
-    for (int r = tid; r < nrhs; r += kThreads) {
-        float *x = R + r * rst;
-        // forward: y_c = (r_c - sum_{m<c} y_m L[c][m]) / L[c][c]
-        for (int j0 = 0; j0 < dk; j0 += kAffB) {
-            float acc[kAffB];
-#pragma unroll
-            for (int c = 0; c < kAffB; ++c) acc[c] = x[j0 + c];
-            for (int m = 0; m < j0; ++m) {
-                const float ym = x[m];
-                const float4 *lt = reinterpret_cast<const float4 *>(A + m * ast + j0);  // L[j0..][m]
-#pragma unroll
-                for (int c4 = 0; c4 < kAffB / 4; ++c4) {
-                    const float4 l = lt[c4];
-                    acc[4 * c4] = fmaf(-ym, l.x, acc[4 * c4]);
-                    acc[4 * c4 + 1] = fmaf(-ym, l.y, acc[4 * c4 + 1]);
-                    acc[4 * c4 + 2] = fmaf(-ym, l.z, acc[4 * c4 + 2]);
-                    acc[4 * c4 + 3] = fmaf(-ym, l.w, acc[4 * c4 + 3]);
-                }
-            }
-#pragma unroll
-            for (int c = 0; c < kAffB; ++c) {
-#pragma unroll
-                for (int c2 = 0; c2 < c; ++c2) acc[c] = fmaf(-acc[c2], A[(j0 + c) * ast + j0 + c2], acc[c]);
-                acc[c] /= A[(j0 + c) * ast + j0 + c];
-            }
-#pragma unroll
-            for (int c = 0; c < kAffB; ++c) x[j0 + c] = acc[c];
-        }
-        // backward: x_c = (y_c - sum_{m>c} x_m L[m][c]) / L[c][c]
-        for (int j0 = dk - kAffB; j0 >= 0; j0 -= kAffB) {
-            float acc[kAffB];
-#pragma unroll
-            for (int c = 0; c < kAffB; ++c) acc[c] = x[j0 + c];
-            for (int m = j0 + kAffB; m < dk; ++m) {
-                const float xm = x[m];
-                const float4 *lr = reinterpret_cast<const float4 *>(A + m * ast + j0);  // L[m][j0..]
-#pragma unroll
-                for (int c4 = 0; c4 < kAffB / 4; ++c4) {
-                    const float4 l = lr[c4];
-                    acc[4 * c4] = fmaf(-xm, l.x, acc[4 * c4]);
-                    acc[4 * c4 + 1] = fmaf(-xm, l.y, acc[4 * c4 + 1]);
-                    acc[4 * c4 + 2] = fmaf(-xm, l.z, acc[4 * c4 + 2]);
-                    acc[4 * c4 + 3] = fmaf(-xm, l.w, acc[4 * c4 + 3]);
-                }
-            }
-#pragma unroll
-            for (int c = kAffB - 1; c >= 0; --c) {
-#pragma unroll
-                for (int c2 = c + 1; c2 < kAffB; ++c2) acc[c] = fmaf(-acc[c2], A[(j0 + c2) * ast + j0 + c], acc[c]);
-                acc[c] /= A[(j0 + c) * ast + j0 + c];
-            }
-#pragma unroll
-            for (int c = 0; c < kAffB; ++c) x[j0 + c] = acc[c];
+            for (int u = 0; u < CW; ++u) buf[0][pj + u] = a[u];
         }
     }
     __syncthreads();
-    for (int e = tid; e < dk * q4; e += kThreads) {
-        const int i = e / q4, j = (e % q4) * 4;
-        const float *Ri = R + i * rst + j;
-        reinterpret_cast<float4 *>(Gp)[e] = make_float4(Ri[0], Ri[1], Ri[2], Ri[3]);
+    for (int kq = 0; kq < 4; ++kq) {  // the pivot's quarter
+#pragma unroll
+        for (int kk = 0; kk < CW; ++kk) {  // the pivot's column inside it (CW is even)
+            const int k = kq * CW + kk;
+            const float *bk = buf[kk & 1];
+            const float dkk = bk[k + 4 * kq];
+            if (tid == 0 && !(dkk > 0.f)) atomicOr(err, kErrNumeric);
+            const float inv = 1.f / dkk;
+            if (act) {
+                const float br = bk[pr];
+                if (r == k) {
+#pragma unroll
+                    for (int u = 0; u < CW; ++u) a[u] = (u == kk && qd == kq) ? -inv : a[u] * inv;
+                } else {
+#pragma unroll
+                    for (int u4 = 0; u4 < CW / 4; ++u4) {
+                        const float4 bj = *reinterpret_cast<const float4 *>(bk + pj + 4 * u4);
+                        a[4 * u4] = fmaf(-(br * bj.x), inv, a[4 * u4]);
+                        a[4 * u4 + 1] = fmaf(-(br * bj.y), inv, a[4 * u4 + 1]);
+                        a[4 * u4 + 2] = fmaf(-(br * bj.z), inv, a[4 * u4 + 2]);
+                        a[4 * u4 + 3] = fmaf(-(br * bj.w), inv, a[4 * u4 + 3]);
+                    }
+                    if (qd == kq) a[kk] = br * inv;  // column k
+                }
+                if (r == k + 1) {
+                    float *bn = buf[(kk + 1) & 1];
+#pragma unroll
+                    for (int u = 0; u < CW; ++u) bn[pj + u] = a[u];
+                }
+            }
+            __syncthreads();
+        }
     }
-    for (int e = tid; e < d.dv * q4; e += kThreads) {
-        const int i = e / q4, j = (e % q4) * 4;
-        const float *Ri = R + (dk + i) * rst + j;
-        reinterpret_cast<float4 *>(Cp)[e] = make_float4(Ri[0], Ri[1], Ri[2], Ri[3]);
+    if (act) {
+#pragma unroll
+        for (int u4 = 0; u4 < CW / 4; ++u4)
+            *reinterpret_cast<float4 *>(Gp + (size_t)r * dk + j0 + 4 * u4) =
+                make_float4(-a[4 * u4], -a[4 * u4 + 1], -a[4 * u4 + 2], -a[4 * u4 + 3]);
     }
 }
 
-// S_t = S_{t-1} M_t + N_t for kChainRows rows of S; every S_t is stored for
-// the output pass (fp32, or its bf16 copy for the tensor-core output pass), the
-// last one also as S_final.  M_t arrives by bulk copy into one of two buffers,
-// one frame ahead; thread (row r, 8 columns) keeps 8 independent sums.
+static cudaError_t launch_inverse(float *GW, const Dims &d, unsigned int *err, cudaStream_t st) {
+    const dim3 gf((unsigned)d.F, (unsigned)d.H, (unsigned)d.B);
+    switch (d.dk / 4) {
+#define GDR_INV(CW) \
+    case CW: frame_inverse_kernel<CW><<<gf, kSwThreads, 0, st>>>(GW, d, err); break
+        GDR_INV(4); GDR_INV(8); GDR_INV(12); GDR_INV(16);
+        GDR_INV(20); GDR_INV(24); GDR_INV(28); GDR_INV(32);
+#undef GDR_INV
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+// S_t = (S_{t-1} D_t + C_t) W_t for kChainRows rows of S; every S_t is stored
+// for the output pass (fp32, or its bf16 copy for the tensor-core output pass),
+// the last one also as S_final.  W_t arrives by bulk copy into one of two
+// buffers, one frame ahead; thread (row r, 8 columns) first forms its 8 entries
+// of S_{t-1} D_t + C_t, then keeps 8 independent sums of the product with W_t.
 __global__ void __launch_bounds__(kThreads)
-frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Nw,
+frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
+                   const float *__restrict__ g, int per_channel,
                    const float *__restrict__ S0, float *__restrict__ Sw,
                    __nv_bfloat16 *__restrict__ Sb, float *__restrict__ S_final, Dims d,
                    unsigned int *err) {
@@ -274,7 +222,7 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Nw,
     const int r0 = blockIdx.y * kChainRows;
     const int nr = min(kChainRows, d.dv - r0);
     const int dk = d.dk;
-    float *Mb = sm, *S = Mb + 2 * dk * dk;  // M_t double buffer (unpadded), S rows [16][dk]
+    float *Mb = sm, *S = Mb + 2 * dk * dk;  // W_t double buffer (unpadded), S rows [16][dk]
     uint64_t *bar = reinterpret_cast<uint64_t *>(S + kChainRows * dk);  // [2]
     const int tid = threadIdx.x, r = tid >> 4, c0 = (tid & 15) * 8;
     const bool mine = r < nr && c0 < dk;
@@ -302,9 +250,16 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Nw,
         const size_t sl = slot(d, b, f, h);
         const float *Mf = Mb + (f & 1) * dk * dk;
         float acc[8];
-        if (mine) {
-            const float *np = Nw + sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c0;
-            ld8(np, acc);
+        if (mine) {  // S_{t-1} D_t + C_t, this thread's entries
+            float cv[8];
+            ld8(Cw + sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c0, cv);
+            float *Sr = S + r * dk + c0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float a = expf(per_channel ? g[sl * dk + c0 + j] : g[sl]);
+                Sr[j] = fmaf(Sr[j], a, cv[j]);
+                acc[j] = 0.f;
+            }
         }
         const bool okw = mbar_wait_bounded(&bar[f & 1], (f >> 1) & 1, kSpinF, err);
         if (!__syncthreads_and(okw)) { ok = false; break; }
@@ -622,10 +577,6 @@ bool frame_shape_ok(int dk, int dv) {
     return dk >= 16 && dk <= 128 && dk % 16 == 0 && dv >= 8 && dv <= 128 && dv % 8 == 0;
 }
 
-size_t affine_smem(int dk, int dv) {
-    return sizeof(float) * ((size_t)dk * (dk + 4) + (size_t)(dk + dv) * (dk + 1));
-}
-
 bool frame_tc_applies(const Dims &d, bool bf16) { return bf16 && d.dk == kTD && d.dv == kTD; }
 
 template <typename Tin>
@@ -650,11 +601,9 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
             return cudaErrorInvalidValue;
     }
     const size_t sm_gram = sizeof(float) * (size_t)(kTokTile * (d.dk + 1) + kTokTile * (d.dv + 1) + kTokTile);
-    const size_t sm_aff = affine_smem(d.dk, d.dv);
     const size_t sm_chain = sizeof(float) * (size_t)(2 * d.dk * d.dk + kChainRows * d.dk) + 64;
     const size_t sm_out = sizeof(float) * (size_t)(d.dv + kTokTile) * (d.dk + 1);
     if ((e = cudaFuncSetAttribute(frame_gram_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gram)) ||
-        (e = cudaFuncSetAttribute(frame_affine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_aff)) ||
         (e = cudaFuncSetAttribute(frame_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_chain)) ||
         (e = cudaFuncSetAttribute(frame_out_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out)))
         return e;
@@ -675,15 +624,15 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
     }
     {
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_SOLVE, st);
-        frame_affine_kernel<<<gf, kThreads, sm_aff, st>>>(GM, CN, g, per_channel, d, err);
+        e = launch_inverse(GM, d, err, st);
         gdr_host::prof_end(tk, st);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
     }
     {
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_CHAIN, st);
         const dim3 gc((unsigned)(d.B * d.H), (unsigned)((d.dv + kChainRows - 1) / kChainRows));
-        frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, S0, Sw, tc ? Sb : nullptr, S_final, d,
-                                                           err);
+        frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, g, per_channel, S0, Sw,
+                                                           tc ? Sb : nullptr, S_final, d, err);
         gdr_host::prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -724,7 +673,6 @@ gdr_status gdr_fwd_frame(const void *q, const void *k, const void *v, const floa
     if ((double)B * T * H * (d_k > d_v ? d_k : d_v) > 9.0e15 || (double)B * T > 2.0e9 ||
         (double)B * H * ((T + n - 1) / n) > 2.0e9)
         return GDR_ERR_INVALID;
-    if (affine_smem(d_k, d_v) > 227u * 1024u) return GDR_ERR_UNSUPPORTED;
     if (B > 65535 || H > 65535) return GDR_ERR_UNSUPPORTED;  // grid y / z extents
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(gamma) ||
         !aligned16(S0) || !aligned16(out) || !aligned16(S_final) || !aligned16(workspace))

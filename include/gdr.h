@@ -223,8 +223,9 @@ gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, con
  * backward-Euler step
  *     S_t (I + G_t) = S_{t-1} D_t + C_t
  * (D_t = the frame's decay, applied first); every query of frame t reads S_t:
- * o_i = S_t q_i.  I + G_t is factorised by Cholesky; n = 1 is the gated delta
- * rule with step size gamma / (1 + gamma).
+ * o_i = S_t q_i.  The kernels form W_t = (I + G_t)^-1 (symmetric sweep, no
+ * pivoting: every pivot of I + G_t is >= 1) and S_t = (S_{t-1} D_t + C_t) W_t;
+ * n = 1 is the gated delta rule with step size gamma / (1 + gamma).
  *  q, k     [B, T, H, d_k]  dtype;  v, out [B, T, H, d_v]  dtype
  *  gamma    [B, T, H]       fp32 writing strength, >= 0 (a negative value can
  *                           make I + G_t indefinite: gdr_device_status then
@@ -233,8 +234,10 @@ gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, con
  *  S0       [B, H, d_v, d_k] fp32 or NULL (zero);  S_final likewise or NULL
  *  d_k a multiple of 16 in [16, 128]; d_v a multiple of 8 in [8, 128]
  *  workspace: gdr_fwd_frame_workspace_size(B, T, H, d_k, d_v, n) bytes,
- *           caller-owned device memory (per frame: G/M_t, C/N_t and S_t, fp32).
- * fp32 arithmetic on the CUDA cores.  Errors as gdr_fwd.
+ *           caller-owned device memory (per frame: G_t then W_t, C_t and S_t).
+ * The Gram and output passes run on the tensor cores for bf16 with
+ * d_k = d_v = 128 (bf16 operands, fp32 accumulation); the inverse and the
+ * chain are fp32 on the CUDA cores.  Errors as gdr_fwd.
  */
 size_t gdr_fwd_frame_workspace_size(int B, int T, int H, int d_k, int d_v, int n);
 gdr_status gdr_fwd_frame(const void *q, const void *k, const void *v, const float *g,

@@ -46,6 +46,26 @@ def test_frame_fp32(cuda_device, n, gate):
     check(inputs.frame_inputs(cfg, seed=701), cuda_device)
 
 
+@pytest.mark.parametrize("dk,dv", [(16, 8), (48, 40), (112, 128), (128, 128)])
+def test_frame_fp32_key_widths(cuda_device, dk, dv):
+    """Every register layout of the inverse pass (d_k / 4 columns per thread)
+    that the shapes reach, on the fp32 path."""
+    cfg = cfg_of(B=1, T=150, H=2, d_k=dk, d_v=dv, n=40, dtype="f32", gate="channel",
+                 s0_var=0.01)
+    check(inputs.frame_inputs(cfg, seed=704), cuda_device)
+
+
+@pytest.mark.parametrize("scale", [20.0, 200.0])
+def test_frame_fp32_strong_writes(cuda_device, scale):
+    """Writing strengths scaled up so that I + G_t is far from the identity
+    (eigenvalues in the hundreds to thousands): the inverse still meets the fp32
+    tolerance."""
+    cfg = cfg_of(B=1, T=256, H=2, d_k=64, d_v=64, n=64, dtype="f32", gate="scalar", s0_var=0.01)
+    inp = inputs.frame_inputs(cfg, seed=705)
+    inp.gamma = (inp.gamma * np.float32(scale)).astype(np.float32)
+    check(inp, cuda_device)
+
+
 @pytest.mark.parametrize("n", [64, 256])
 def test_frame_bf16_d128(cuda_device, n):
     cfg = cfg_of(B=1, T=1000, H=3, n=n, s0_var=0.01)
