@@ -114,72 +114,81 @@ frame_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
 // a_ij -> a_ij - a_ik a_kj / a_kk; after every pivot the matrix is -(I + G_t)^-1.
 // I + G_t is symmetric with eigenvalues >= 1, so every pivot (a Schur
 // complement's diagonal) is >= 1 and no pivoting is needed.  G_t is
-// symmetrised as (G + G^T) / 2 on load, and each update a_ij -= (a_ik a_kj) /
-// a_kk is symmetric in i and j, so the matrix stays exactly symmetric and row
-// k stands in for column k.  Thread (row r, quarter) holds d_k / 4 entries of
-// row r in registers; the pivot row passes through a double buffer in shared
-// memory, written by its own row's threads during the previous step: one
-// barrier per pivot.  W_t overwrites G_t.
-constexpr int kSwThreads = 512;  // 4 threads per row, d_k <= 128
-template <int CW>  // columns per thread: d_k / 4
+// symmetrised as (G + G^T) / 2 on load; with s = a_kk^-1/2 and c = s b (b =
+// pivot row) the update a_ij -= c_i c_j is symmetric in i and j, so the matrix
+// stays exactly symmetric and row k stands in for column k.  A thread holds a
+// 4 x 8 tile in registers and reads 12 pivot-row values per step; the pivot
+// row passes through a double buffer in shared memory, written by its own
+// row's threads during the previous step: one barrier per pivot.  W_t
+// overwrites G_t.
+constexpr int kSwThreads = 512;  // (d_k / 4) x (d_k / 8) tiles of 4 x 8, d_k <= 128
+template <int DK>
 __global__ void __launch_bounds__(kSwThreads, 2)
 frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
-    __shared__ __align__(16) float buf[2][128 + 16];  // pivot rows, +4 floats per quarter
+    __shared__ __align__(16) float buf[2][128];  // pivot rows
+    constexpr int NCG = DK / 8, NRG = DK / 4;     // column / row groups
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int dk = 4 * CW;
-    const int tid = threadIdx.x, r = tid >> 2, qd = tid & 3, j0 = qd * CW;
-    const bool act = r < dk;
+    const int tid = threadIdx.x, cg = tid % NCG, rg = tid / NCG;
+    const bool act = rg < NRG;
+    const int r0 = 4 * rg, j0 = 8 * cg;
     const size_t sl = slot(d, b, f, h);
-    float *Gp = GW + sl * (size_t)dk * dk;
-    // quarter q of a pivot row starts at q * (CW + 4): the quarters fall on
-    // different banks
-    const int pr = r + 4 * (r / CW), pj = j0 + 4 * qd;
-    float a[CW];
+    float *Gp = GW + sl * (size_t)DK * DK;
+    float a[4][8];
     if (act) {
 #pragma unroll
-        for (int u4 = 0; u4 < CW / 4; ++u4) {
-            const float4 x = *reinterpret_cast<const float4 *>(Gp + (size_t)r * dk + j0 + 4 * u4);
-            a[4 * u4] = x.x; a[4 * u4 + 1] = x.y; a[4 * u4 + 2] = x.z; a[4 * u4 + 3] = x.w;
+        for (int i = 0; i < 4; ++i) {
+            const float4 x = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + j0);
+            const float4 y = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + j0 + 4);
+            a[i][0] = x.x; a[i][1] = x.y; a[i][2] = x.z; a[i][3] = x.w;
+            a[i][4] = y.x; a[i][5] = y.y; a[i][6] = y.z; a[i][7] = y.w;
         }
 #pragma unroll
-        for (int u = 0; u < CW; ++u) {
-            const int j = j0 + u;
-            a[u] = 0.5f * (a[u] + Gp[(size_t)j * dk + r]) + (j == r ? 1.f : 0.f);
-        }
-        if (r == 0) {
+        for (int u = 0; u < 8; ++u) {  // G^T: column j0 + u, rows r0..r0+3
+            const float4 t = *reinterpret_cast<const float4 *>(Gp + (size_t)(j0 + u) * DK + r0);
+            const float tv[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-            for (int u = 0; u < CW; ++u) buf[0][pj + u] = a[u];
+            for (int i = 0; i < 4; ++i)
+                a[i][u] = 0.5f * (a[i][u] + tv[i]) + (r0 + i == j0 + u ? 1.f : 0.f);
+        }
+        if (rg == 0) {
+            *reinterpret_cast<float4 *>(&buf[0][j0]) = make_float4(a[0][0], a[0][1], a[0][2], a[0][3]);
+            *reinterpret_cast<float4 *>(&buf[0][j0 + 4]) = make_float4(a[0][4], a[0][5], a[0][6], a[0][7]);
         }
     }
     __syncthreads();
-    for (int kq = 0; kq < 4; ++kq) {  // the pivot's quarter
+    for (int k8 = 0; k8 < DK; k8 += 8) {
 #pragma unroll
-        for (int kk = 0; kk < CW; ++kk) {  // the pivot's column inside it (CW is even)
-            const int k = kq * CW + kk;
+        for (int kk = 0; kk < 8; ++kk) {
+            const int k = k8 + kk;
             const float *bk = buf[kk & 1];
-            const float dkk = bk[k + 4 * kq];
+            const float dkk = bk[k];
             if (tid == 0 && !(dkk > 0.f)) atomicOr(err, kErrNumeric);
-            const float inv = 1.f / dkk;
+            const float sq = rsqrtf(dkk);
             if (act) {
-                const float br = bk[pr];
-                if (r == k) {
+                const float4 br4 = *reinterpret_cast<const float4 *>(bk + r0);
+                const float4 bj0 = *reinterpret_cast<const float4 *>(bk + j0);
+                const float4 bj1 = *reinterpret_cast<const float4 *>(bk + j0 + 4);
+                const float cr[4] = {br4.x * sq, br4.y * sq, br4.z * sq, br4.w * sq};
+                const float cj[8] = {bj0.x * sq, bj0.y * sq, bj0.z * sq, bj0.w * sq,
+                                     bj1.x * sq, bj1.y * sq, bj1.z * sq, bj1.w * sq};
+                const bool krow = (k >> 2) == rg, kcol = (k >> 3) == cg;
+                const int ki = kk & 3;  // the pivot's row inside a tile (unrolled: a constant)
 #pragma unroll
-                    for (int u = 0; u < CW; ++u) a[u] = (u == kk && qd == kq) ? -inv : a[u] * inv;
-                } else {
+                for (int i = 0; i < 4; ++i) {
+                    if (i == ki && krow) {  // row k
 #pragma unroll
-                    for (int u4 = 0; u4 < CW / 4; ++u4) {
-                        const float4 bj = *reinterpret_cast<const float4 *>(bk + pj + 4 * u4);
-                        a[4 * u4] = fmaf(-(br * bj.x), inv, a[4 * u4]);
-                        a[4 * u4 + 1] = fmaf(-(br * bj.y), inv, a[4 * u4 + 1]);
-                        a[4 * u4 + 2] = fmaf(-(br * bj.z), inv, a[4 * u4 + 2]);
-                        a[4 * u4 + 3] = fmaf(-(br * bj.w), inv, a[4 * u4 + 3]);
+                        for (int u = 0; u < 8; ++u) a[i][u] = (u == kk && kcol) ? -(sq * sq) : cj[u] * sq;
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) a[i][u] = fmaf(-cr[i], cj[u], a[i][u]);
+                        if (kcol) a[i][kk] = cr[i] * sq;  // column k
                     }
-                    if (qd == kq) a[kk] = br * inv;  // column k
                 }
-                if (r == k + 1) {
+                const int ni = (kk + 1) & 3;  // the next pivot's row inside a tile
+                if (((k + 1) >> 2) == rg) {
                     float *bn = buf[(kk + 1) & 1];
-#pragma unroll
-                    for (int u = 0; u < CW; ++u) bn[pj + u] = a[u];
+                    *reinterpret_cast<float4 *>(bn + j0) = make_float4(a[ni][0], a[ni][1], a[ni][2], a[ni][3]);
+                    *reinterpret_cast<float4 *>(bn + j0 + 4) = make_float4(a[ni][4], a[ni][5], a[ni][6], a[ni][7]);
                 }
             }
             __syncthreads();
@@ -187,19 +196,21 @@ frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
     }
     if (act) {
 #pragma unroll
-        for (int u4 = 0; u4 < CW / 4; ++u4)
-            *reinterpret_cast<float4 *>(Gp + (size_t)r * dk + j0 + 4 * u4) =
-                make_float4(-a[4 * u4], -a[4 * u4 + 1], -a[4 * u4 + 2], -a[4 * u4 + 3]);
+        for (int i = 0; i < 4; ++i) {
+            float4 *o = reinterpret_cast<float4 *>(Gp + (size_t)(r0 + i) * DK + j0);
+            o[0] = make_float4(-a[i][0], -a[i][1], -a[i][2], -a[i][3]);
+            o[1] = make_float4(-a[i][4], -a[i][5], -a[i][6], -a[i][7]);
+        }
     }
 }
 
 static cudaError_t launch_inverse(float *GW, const Dims &d, unsigned int *err, cudaStream_t st) {
     const dim3 gf((unsigned)d.F, (unsigned)d.H, (unsigned)d.B);
-    switch (d.dk / 4) {
-#define GDR_INV(CW) \
-    case CW: frame_inverse_kernel<CW><<<gf, kSwThreads, 0, st>>>(GW, d, err); break
-        GDR_INV(4); GDR_INV(8); GDR_INV(12); GDR_INV(16);
-        GDR_INV(20); GDR_INV(24); GDR_INV(28); GDR_INV(32);
+    switch (d.dk) {
+#define GDR_INV(DK) \
+    case DK: frame_inverse_kernel<DK><<<gf, kSwThreads, 0, st>>>(GW, d, err); break
+        GDR_INV(16); GDR_INV(32); GDR_INV(48); GDR_INV(64);
+        GDR_INV(80); GDR_INV(96); GDR_INV(112); GDR_INV(128);
 #undef GDR_INV
         default: return cudaErrorInvalidValue;
     }
@@ -263,14 +274,17 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
         }
         const bool okw = mbar_wait_bounded(&bar[f & 1], (f >> 1) & 1, kSpinF, err);
         if (!__syncthreads_and(okw)) { ok = false; break; }
-        if (mine) {
+        if (mine) {  // 8 rows of W_t per round, every load issued before the FMAs
             const float *Sr = S + r * dk;
-            for (int m = 0; m < dk; ++m) {
-                const float sv = Sr[m];
-                float mm[8];
-                ld8(Mf + m * dk + c0, mm);
+            for (int m0 = 0; m0 < dk; m0 += 8) {
+                float sv[8], mm[8][8];
+                ld8(Sr + m0, sv);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] = fmaf(sv, mm[j], acc[j]);
+                for (int i = 0; i < 8; ++i) ld8(Mf + (m0 + i) * dk + c0, mm[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[j] = fmaf(sv[i], mm[i][j], acc[j]);
             }
         }
         __syncthreads();  // S and this M buffer are read
