@@ -232,11 +232,15 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
     const int bh = blockIdx.x, b = bh / d.H, h = bh % d.H;
     const int r0 = blockIdx.y * kChainRows;
     const int nr = min(kChainRows, d.dv - r0);
-    const int dk = d.dk;
-    float *Mb = sm, *S = Mb + 2 * dk * dk;  // W_t double buffer (unpadded), S rows [16][dk]
-    uint64_t *bar = reinterpret_cast<uint64_t *>(S + kChainRows * dk);  // [2]
-    const int tid = threadIdx.x, r = tid >> 4, c0 = (tid & 15) * 8;
-    const bool mine = r < nr && c0 < dk;
+    const int dk = d.dk, sst = dk + 4;
+    // W_t double buffer (unpadded, as copied), then S rows [16][dk + 4]
+    float *Mb = sm, *S = Mb + 2 * dk * dk;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(S + kChainRows * sst);  // [2]
+    // thread (row r, group cg): columns ca..ca+3 and cb..cb+3 of the row, so
+    // that each float4 read of a W_t row by 16 threads covers 256 contiguous bytes
+    const int tid = threadIdx.x, r = tid >> 4, cg = tid & 15;
+    const int ca = 4 * cg, cb = dk / 2 + 4 * cg;
+    const bool mine = r < nr && cg < dk / 8;
     const uint32_t mbytes = (uint32_t)(dk * dk * 4);
     const size_t soff = ((size_t)b * d.H + h) * (size_t)d.dv * dk;
     if (tid == 0) {
@@ -246,7 +250,7 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
     }
     for (int e = tid; e < kChainRows * dk; e += kThreads) {
         const int rr = e / dk, c = e % dk;
-        S[e] = (S0 && rr < nr) ? S0[soff + (size_t)(r0 + rr) * dk + c] : 0.f;
+        S[rr * sst + c] = (S0 && rr < nr) ? S0[soff + (size_t)(r0 + rr) * dk + c] : 0.f;
     }
     __syncthreads();
     int issued = 0;
@@ -257,37 +261,50 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
                       &bar[issued]);
         }
     bool ok = true;
+    float *Sr = S + r * sst;
     for (int f = 0; f < d.F; ++f) {
         const size_t sl = slot(d, b, f, h);
         const float *Mf = Mb + (f & 1) * dk * dk;
         float acc[8];
         if (mine) {  // S_{t-1} D_t + C_t, this thread's entries
-            float cv[8];
-            ld8(Cw + sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c0, cv);
-            float *Sr = S + r * dk + c0;
+            const float *crow = Cw + sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk;
+            const float4 x = *reinterpret_cast<const float4 *>(crow + ca);
+            const float4 y = *reinterpret_cast<const float4 *>(crow + cb);
+            const float cv[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float a = expf(per_channel ? g[sl * dk + c0 + j] : g[sl]);
-                Sr[j] = fmaf(Sr[j], a, cv[j]);
+                const int c = (j < 4 ? ca : cb - 4) + j;
+                const float a = expf(per_channel ? g[sl * dk + c] : g[sl]);
+                Sr[c] = fmaf(Sr[c], a, cv[j]);
                 acc[j] = 0.f;
             }
         }
         const bool okw = mbar_wait_bounded(&bar[f & 1], (f >> 1) & 1, kSpinF, err);
         if (!__syncthreads_and(okw)) { ok = false; break; }
-        if (mine) {  // 8 rows of W_t per round, every load issued before the FMAs
-            const float *Sr = S + r * dk;
-            for (int m0 = 0; m0 < dk; m0 += 8) {
-                float sv[8], mm[8][8];
-                ld8(Sr + m0, sv);
+        if (mine) {  // 4 rows of W_t per round, every load issued before the FMAs
+            for (int m0 = 0; m0 < dk; m0 += 4) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(Sr + m0);
+                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+                float4 wa[4], wb[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) ld8(Mf + (m0 + i) * dk + c0, mm[i]);
+                for (int i = 0; i < 4; ++i) {
+                    wa[i] = *reinterpret_cast<const float4 *>(Mf + (m0 + i) * dk + ca);
+                    wb[i] = *reinterpret_cast<const float4 *>(Mf + (m0 + i) * dk + cb);
+                }
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[j] = fmaf(sv[i], mm[i][j], acc[j]);
+                for (int i = 0; i < 4; ++i) {
+                    acc[0] = fmaf(sv[i], wa[i].x, acc[0]);
+                    acc[1] = fmaf(sv[i], wa[i].y, acc[1]);
+                    acc[2] = fmaf(sv[i], wa[i].z, acc[2]);
+                    acc[3] = fmaf(sv[i], wa[i].w, acc[3]);
+                    acc[4] = fmaf(sv[i], wb[i].x, acc[4]);
+                    acc[5] = fmaf(sv[i], wb[i].y, acc[5]);
+                    acc[6] = fmaf(sv[i], wb[i].z, acc[6]);
+                    acc[7] = fmaf(sv[i], wb[i].w, acc[7]);
+                }
             }
         }
-        __syncthreads();  // S and this M buffer are read
+        __syncthreads();  // S and this W buffer are read
         if (tid == 0 && f + 2 < d.F) {
             mbar_arrive_expect_tx(&bar[f & 1], mbytes);
             bulk_load(Mb + (f & 1) * dk * dk, Mw + slot(d, b, f + 2, h) * (size_t)dk * dk, mbytes,
@@ -295,25 +312,27 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
             issued = f + 3;
         }
         if (mine) {
-            float *Sr = S + r * dk + c0;
-            const size_t o = sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk + c0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) Sr[j] = acc[j];
+            *reinterpret_cast<float4 *>(Sr + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            *reinterpret_cast<float4 *>(Sr + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            const size_t o = sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk;
             if (Sb) {  // operand of the tensor-core output pass
-                *reinterpret_cast<uint4 *>(Sb + o) = pack8(acc);
+                __nv_bfloat162 pa[2] = {__floats2bfloat162_rn(acc[0], acc[1]),
+                                        __floats2bfloat162_rn(acc[2], acc[3])};
+                __nv_bfloat162 pb[2] = {__floats2bfloat162_rn(acc[4], acc[5]),
+                                        __floats2bfloat162_rn(acc[6], acc[7])};
+                *reinterpret_cast<uint2 *>(Sb + o + ca) = *reinterpret_cast<uint2 *>(pa);
+                *reinterpret_cast<uint2 *>(Sb + o + cb) = *reinterpret_cast<uint2 *>(pb);
             } else {
-                float4 *o4 = reinterpret_cast<float4 *>(Sw + o);
-                o4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                o4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                *reinterpret_cast<float4 *>(Sw + o + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                *reinterpret_cast<float4 *>(Sw + o + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
             }
         }
         __syncthreads();
     }
     if (ok && S_final && mine) {
-        float4 *o4 = reinterpret_cast<float4 *>(S_final + soff + (size_t)(r0 + r) * dk + c0);
-        const float *Sr = S + r * dk + c0;
-        o4[0] = make_float4(Sr[0], Sr[1], Sr[2], Sr[3]);
-        o4[1] = make_float4(Sr[4], Sr[5], Sr[6], Sr[7]);
+        float *o = S_final + soff + (size_t)(r0 + r) * dk;
+        *reinterpret_cast<float4 *>(o + ca) = *reinterpret_cast<const float4 *>(Sr + ca);
+        *reinterpret_cast<float4 *>(o + cb) = *reinterpret_cast<const float4 *>(Sr + cb);
     }
     if (tid == 0)  // copies still in flight (error path) land before exit
         for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait_bounded(&bar[i & 1], (i >> 1) & 1, kSpinF, err);
@@ -615,7 +634,7 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
             return cudaErrorInvalidValue;
     }
     const size_t sm_gram = sizeof(float) * (size_t)(kTokTile * (d.dk + 1) + kTokTile * (d.dv + 1) + kTokTile);
-    const size_t sm_chain = sizeof(float) * (size_t)(2 * d.dk * d.dk + kChainRows * d.dk) + 64;
+    const size_t sm_chain = sizeof(float) * (size_t)(2 * d.dk * d.dk + kChainRows * (d.dk + 4)) + 64;
     const size_t sm_out = sizeof(float) * (size_t)(d.dv + kTokTile) * (d.dk + 1);
     if ((e = cudaFuncSetAttribute(frame_gram_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gram)) ||
         (e = cudaFuncSetAttribute(frame_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_chain)) ||
