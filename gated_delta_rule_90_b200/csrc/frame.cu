@@ -262,22 +262,33 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
         }
     bool ok = true;
     float *Sr = S + r * sst;
+    // C_t row entries and log-decays of this thread's columns, loaded one frame
+    // ahead so that their latency stays off the chain
+    float cv[8], gv[8];
+    auto fetch = [&](int f) {
+        const size_t sl = slot(d, b, f, h);
+        const float *crow = Cw + sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk;
+        const float4 x = *reinterpret_cast<const float4 *>(crow + ca);
+        const float4 y = *reinterpret_cast<const float4 *>(crow + cb);
+        cv[0] = x.x; cv[1] = x.y; cv[2] = x.z; cv[3] = x.w;
+        cv[4] = y.x; cv[5] = y.y; cv[6] = y.z; cv[7] = y.w;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            gv[j] = per_channel ? g[sl * dk + (j < 4 ? ca : cb - 4) + j] : g[sl];
+    };
+    if (mine) fetch(0);
     for (int f = 0; f < d.F; ++f) {
         const size_t sl = slot(d, b, f, h);
         const float *Mf = Mb + (f & 1) * dk * dk;
         float acc[8];
         if (mine) {  // S_{t-1} D_t + C_t, this thread's entries
-            const float *crow = Cw + sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk;
-            const float4 x = *reinterpret_cast<const float4 *>(crow + ca);
-            const float4 y = *reinterpret_cast<const float4 *>(crow + cb);
-            const float cv[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int c = (j < 4 ? ca : cb - 4) + j;
-                const float a = expf(per_channel ? g[sl * dk + c] : g[sl]);
-                Sr[c] = fmaf(Sr[c], a, cv[j]);
+                Sr[c] = fmaf(Sr[c], expf(gv[j]), cv[j]);
                 acc[j] = 0.f;
             }
+            if (f + 1 < d.F) fetch(f + 1);
         }
         const bool okw = mbar_wait_bounded(&bar[f & 1], (f >> 1) & 1, kSpinF, err);
         if (!__syncthreads_and(okw)) { ok = false; break; }
