@@ -332,11 +332,13 @@ class FrameRun:
 
 
 def frame_flops_per_token_head(dk, dv, n):
-    """G_t and C_t (2 d_k (d_k + d_v) per token), the output (2 d_k d_v per
-    token), and per frame the Cholesky (d_k^3 / 3), the substitutions for
-    M_t, N_t (2 d_k^2 (d_k + d_v)) and the chain product (2 d_v d_k^2), spread
-    over the frame's n tokens."""
-    per_frame = dk ** 3 / 3 + 2 * dk * dk * (dk + dv) + 2 * dv * dk * dk
+    """The method's own count: G_t and C_t (2 d_k (d_k + d_v) per token), the
+    output (2 d_k d_v per token), and per frame a Cholesky of I + G_t
+    (d_k^3 / 3) and the two triangular solves for the d_v rows of S_t
+    (2 d_v d_k^2), spread over the frame's n tokens.  The kernels form the
+    whole inverse instead (2 d_k^3 flops by the sweep) and multiply by it
+    (2 d_v d_k^2); the extra work is not counted."""
+    per_frame = dk ** 3 / 3 + 2 * dv * dk * dk
     return 2 * dk * (dk + dv) + 2 * dk * dv + per_frame / n
 
 
@@ -599,7 +601,7 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
         dk, dv = cfg.d_k, cfg.d_v
         tc_path = cfg.dtype == "bf16" and dk == 128 and dv == 128
         pflops = {"frame_gram": 2 * dk * (dk + dv) * th, "frame_out": 2 * dk * dv * th,
-                  "frame_solve": (dk ** 3 / 3 + 2 * dk * dk * (dk + dv)) * fh,
+                  "frame_solve": dk ** 3 / 3 * fh,
                   "frame_chain": 2 * dv * dk * dk * fh}
         flops = pflops.get(dom, 0)
         on_tc = tc_path and dom in ("frame_gram", "frame_out")
