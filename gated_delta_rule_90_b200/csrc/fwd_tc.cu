@@ -216,21 +216,12 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     const size_t slot = (size_t)gcid * geo.H + h;
     const int x0 = h * D, ytok = (int)tstart;
 
-    if (tid == 0) {
+    // The TMA thread initialises the barriers and issues the loads first, so
+    // that their latency overlaps the TMEM allocation and the gate loads.
+    if (tid == kWyTmaThread) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tslot, kWyTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tslot;
-
-    if (tid == kWyTmaThread) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
@@ -245,10 +236,17 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             tma_load_2d(sGt, &tm_g, &bars[0], x0, ytok);  // [64][128] fp32 per-channel gates
         }
     }
+    if (warp == 0) {
+        tmem_alloc(tslot, kWyTmemCols);
+        tmem_relinquish();
+    }
     // gates and beta (zero beyond the sequence end), cumulative log-decay G
     if (!CH && tid < C) sG[tid] = (tid < len) ? g[(size_t)(tstart + tid) * geo.H + h] : 0.f;
     if (tid < C) sB[tid] = (tid < len) ? (DEC ? 1.f : beta[(size_t)(tstart + tid) * geo.H + h]) : 0.f;
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
     if (!CH && warp == 0) {
         float a = sG[lane], b = sG[lane + 32];
 #pragma unroll
@@ -719,9 +717,41 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
     const int gc0 = geo.varlen ? ws.chunk_start[s] : s * geo.nc;
     const int nch = (int)((t1 - t0 + C - 1) / C);
 
-    if (tid == 0) {
+    auto issue = [&](int r) {  // stage r & 1 <- chunk r's operands and decay row
+        uint8_t *st = sm + (r & 1) * StSmem::STAGE;
+        uint64_t *bar = &full[r & 1];
+        const size_t sl = (size_t)(gc0 + r) * geo.H + h;
+        mbar_arrive_expect_tx(bar, StSmem::TX);
+        tma_load_2d(st + StSmem::WQ, &tm_W, bar, 0, (int)(sl * C));
+        tma_load_2d(st + StSmem::WQ + 16384, &tm_W, bar, 64, (int)(sl * C));
+        tma_load_2d(st + StSmem::UT, &tm_U, bar, 0, (int)(sl * D));
+        tma_load_2d(st + StSmem::WQ + 8192, &tm_Q, bar, 0, (int)(sl * C));
+        tma_load_2d(st + StSmem::WQ + 16384 + 8192, &tm_Q, bar, 64, (int)(sl * C));
+        tma_load_2d(st + StSmem::K, &tm_K, bar, 0, (int)(sl * C));
+        tma_load_2d(st + StSmem::K + 8192, &tm_K, bar, 64, (int)(sl * C));
+        tma_load_2d(st + StSmem::A, &tm_A, bar, 0, (int)(sl * C));
+        bulk_load(sm + StSmem::DEC + (r & 1) * kDecBytes, ws.dec + sl * D, kDecBytes, bar);
+    };
+    // The TMA thread initialises the stage barriers and issues the first two
+    // stages before the CTA barrier, overlapping the TMEM allocation and the
+    // S0 load.
+    constexpr int kStTmaThread = 13 * 32;
+    if (tid == kStTmaThread) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
+        fence_mbar_init();
+        if (nch > 0) {
+            prefetch_tmap(&tm_W);
+            prefetch_tmap(&tm_U);
+            prefetch_tmap(&tm_Q);
+            prefetch_tmap(&tm_K);
+            prefetch_tmap(&tm_A);
+            prefetch_tmap(&tm_out);
+            issue(0);
+            if (nch > 1) issue(1);
+        }
+    }
+    if (tid == 0) {
         mbar_init(barZ, 1);
         mbar_init(barS, 1);
         mbar_init(&barO[0], 1);
@@ -733,6 +763,14 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
     if (warp == 0) {
         tmem_alloc(tslot, kStTmemCols);
         tmem_relinquish();
+    }
+    // the chain warps' rows of S0 (or 0), loaded before the barrier as well
+    float s0v[64];
+    if (warp < 8) {
+        const int d = (warp & 3) * 32 + lane;
+        const size_t soff = ((size_t)s * geo.H + h) * (size_t)D * D + (size_t)d * D + (warp >> 2) * 64;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) s0v[i] = S0 ? S0[soff + i] : 0.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -748,12 +786,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
         const uint32_t lb = (uint32_t)(qd * 32) << 16;
         const size_t soff = ((size_t)s * geo.H + h) * (size_t)D * D + (size_t)d * D + hf * 64;
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {  // S <- S0 (or 0)
-            float v[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = S0 ? S0[soff + cb * 16 + i] : 0.f;
-            tmem_st16(tS + lb + hf * 64 + cb * 16, v);
-        }
+        for (int cb = 0; cb < 4; ++cb) tmem_st16(tS + lb + hf * 64 + cb * 16, s0v + cb * 16);  // S <- S0
         tmem_wait_st();
         for (int r = 0; r < nch; ++r) {
             const uint8_t *st = sm + (r & 1) * StSmem::STAGE;
@@ -873,38 +906,9 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             }
         }
         if (otid == 0) bulk_wait_group_read<0>();
-    } else if (warp == 13 && lane == 0) {
-        // ===================== TMA loads =====================
-        auto issue = [&](int r) {
-            uint8_t *st = sm + (r & 1) * StSmem::STAGE;
-            uint64_t *bar = &full[r & 1];
-            const size_t sl = (size_t)(gc0 + r) * geo.H + h;
-            mbar_arrive_expect_tx(bar, StSmem::TX);
-            tma_load_2d(st + StSmem::WQ, &tm_W, bar, 0, (int)(sl * C));
-            tma_load_2d(st + StSmem::WQ + 16384, &tm_W, bar, 64, (int)(sl * C));
-            tma_load_2d(st + StSmem::UT, &tm_U, bar, 0, (int)(sl * D));
-            tma_load_2d(st + StSmem::WQ + 8192, &tm_Q, bar, 0, (int)(sl * C));
-            tma_load_2d(st + StSmem::WQ + 16384 + 8192, &tm_Q, bar, 64, (int)(sl * C));
-            tma_load_2d(st + StSmem::K, &tm_K, bar, 0, (int)(sl * C));
-            tma_load_2d(st + StSmem::K + 8192, &tm_K, bar, 64, (int)(sl * C));
-            tma_load_2d(st + StSmem::A, &tm_A, bar, 0, (int)(sl * C));
-            bulk_load(sm + StSmem::DEC + (r & 1) * kDecBytes, ws.dec + sl * D, kDecBytes, bar);
-        };
-        int issued = 0;
-        if (nch > 0) {
-            prefetch_tmap(&tm_W);
-            prefetch_tmap(&tm_U);
-            prefetch_tmap(&tm_Q);
-            prefetch_tmap(&tm_K);
-            prefetch_tmap(&tm_A);
-            prefetch_tmap(&tm_out);
-            issue(0);
-            issued = 1;
-            if (nch > 1) {
-                issue(1);
-                issued = 2;
-            }
-        }
+    } else if (tid == kStTmaThread) {
+        // ===================== TMA loads (stages 0 and 1 are in flight) =====================
+        int issued = nch < 2 ? nch : 2;
         // stage r & 1 is free once chunk r - 2's MMAs (the last is O2) are done
         for (int r = 2; r < nch && ok; ++r) {
             ok = mbar_wait_bounded(&barO[r & 1], ((r - 2) >> 1) & 1, kSpin, err);
