@@ -41,11 +41,15 @@ SM_COUNT = 148
 # the sha256 of those sources in order.
 _TC_SRC = ('csrc/fwd_tc.cu', 'csrc/sm100.cuh', 'csrc/common.cuh')
 _DEC_SRC = ('csrc/decode.cu', 'csrc/common.cuh')
+_FR_SRC = ('csrc/frame.cu', 'csrc/sm100.cuh', 'csrc/tmap.cuh', 'csrc/common.cuh')
 NCU_TRAFFIC = {
-    ("tc_wy", "gdn_prefill"): (_TC_SRC, "ab41361bf6724bc7", 206.262272e6 + 256.316672e6),
-    ("tc_state", "gdn_prefill"): (_TC_SRC, "ab41361bf6724bc7", 308.345088e6 + 57.322240e6),
-    ("tc_wy", "kda_prefill"): (_TC_SRC, "ab41361bf6724bc7", 681.604608e6 + 565.627648e6),
+    ("tc_wy", "gdn_prefill"): (_TC_SRC, "b92518ad066f9472", 206.202112e6 + 255.384832e6),
+    ("tc_state", "gdn_prefill"): (_TC_SRC, "b92518ad066f9472", 308.424704e6 + 53.710848e6),
+    ("tc_wy", "kda_prefill"): (_TC_SRC, "b92518ad066f9472", 681.083648e6 + 565.622528e6),
     ("decode", "decode"): (_DEC_SRC, "82e1f5016f476188", 543.250944e6 + 482.361600e6),
+    ("decode", "kda_decode"): (_DEC_SRC, "82e1f5016f476188", 547.403264e6 + 482.458624e6),
+    ("frame_chain", "frame_prefill"): (_FR_SRC, "ebb311790167a782", 33.712128e6 + 0.0),
+    ("frame_solve", "frame_prefill"): (_FR_SRC, "ebb311790167a782", 16.801280e6 + 0.0),
 }
 
 
@@ -609,7 +613,7 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
         peak = peaks["bf16_tflops"] if on_tc else alu_peak
         ach = flops / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor" if on_tc else "alu", "kernel": dom, "achieved": ach,
-                "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "traffic": ncu_traffic(dom, name),
                 "peak_source": (peak_kind + " bf16_tflops (burst)") if on_tc else
                 "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
                 "algorithmic_flops_per_launch": flops,
