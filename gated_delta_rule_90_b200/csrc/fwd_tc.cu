@@ -176,7 +176,9 @@ struct WySmem {
 // section "What decoupling actually means here"): the Gram's reading rows are
 // e = b . k (so L = tril_-1(E K^T . Gamma) and W<- = T E<-), T solves
 // (I + L) T = I, and U = T (w . V).  The writing direction stays k (K->, A).
-template <bool CH, bool DEC = false>
+// BC (with CH): the decay is one scalar per token, broadcast over the key
+// channels of the gate tile in shared memory instead of loaded per channel.
+template <bool CH, bool DEC = false, bool BC = false>
 __global__ void __launch_bounds__(kWyThreads)
 wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -225,7 +227,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_arrive_expect_tx(&bars[0], 4 * kHalfBytes + (CH ? 2 * kHalfBytes + C * D * 4 : 0));
+        mbar_arrive_expect_tx(&bars[0], 4 * kHalfBytes + (CH ? 2 * kHalfBytes + (BC ? 0 : C * D * 4) : 0));
         tma_load_2d(sKQ, &tm_k, &bars[0], x0, ytok);
         tma_load_2d(sKQ + 16384, &tm_k, &bars[0], x0 + 64, ytok);
         tma_load_2d(sKQ + 8192, &tm_q, &bars[0], x0, ytok);
@@ -233,7 +235,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         if (CH) {
             tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
             tma_load_2d(sV + 8192, &tm_v, &bars[0], x0 + 64, ytok);
-            tma_load_2d(sGt, &tm_g, &bars[0], x0, ytok);  // [64][128] fp32 per-channel gates
+            if (!BC) tma_load_2d(sGt, &tm_g, &bars[0], x0, ytok);  // [64][128] fp32 per-channel gates
         }
     }
     if (warp == 0) {
@@ -243,6 +245,13 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     // gates and beta (zero beyond the sequence end), cumulative log-decay G
     if (!CH && tid < C) sG[tid] = (tid < len) ? g[(size_t)(tstart + tid) * geo.H + h] : 0.f;
     if (tid < C) sB[tid] = (tid < len) ? (DEC ? 1.f : beta[(size_t)(tstart + tid) * geo.H + h]) : 0.f;
+    if (BC) {  // the gate tile from one log-decay per token
+        for (int e = tid; e < C * D / 4; e += kWyThreads) {
+            const int l = e / (D / 4);
+            const float gl = (l < len) ? g[(size_t)(tstart + l) * geo.H + h] : 0.f;
+            reinterpret_cast<float4 *>(sGt)[e] = make_float4(gl, gl, gl, gl);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1074,10 +1083,11 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
     }
     const bool ch = gate == GDR_GATE_PER_KEY_CHANNEL;
     if (have_tokens && L.n_slots > 0) {
-        const size_t smem = wy_smem_bytes(ch);
         const bool dec = eg != nullptr;
-        if (dec && !ch) return cudaErrorInvalidValue;  // decoupled gates need the per-channel decay
-        auto kern = dec ? wy_kernel<true, true> : ch ? wy_kernel<true> : wy_kernel<false>;
+        // decoupled gates run the per-channel kernel; a scalar decay is broadcast
+        const size_t smem = wy_smem_bytes(ch || dec);
+        auto kern = dec ? (ch ? wy_kernel<true, true> : wy_kernel<true, true, true>)
+                        : ch ? wy_kernel<true> : wy_kernel<false>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem)) != cudaSuccess)
             return e;
@@ -1111,15 +1121,16 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
                        gate, workspace, ws_bytes, err, st);
 }
 
-// Gated DeltaNet-2 (per-channel decay): erase gate eg [.., d_k], write gate wg [.., d_v].
+// Gated DeltaNet-2: erase gate eg [.., d_k], write gate wg [.., d_v]; the decay
+// per key channel or one scalar per token.
 cudaError_t fwd_tc_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
                                  const float *eg, const float *wg, const float *S0, void *out,
                                  float *S_final, int B, int T, int H, const int32_t *cu, int n_seq,
-                                 void *workspace, size_t ws_bytes, unsigned int *err,
-                                 cudaStream_t st) {
+                                 gdr_gate gate, void *workspace, size_t ws_bytes,
+                                 unsigned int *err, cudaStream_t st) {
     if (!eg || !wg) return cudaErrorInvalidValue;
-    return tc_dispatch(q, k, v, g, nullptr, eg, wg, S0, out, S_final, B, T, H, cu, n_seq,
-                       GDR_GATE_PER_KEY_CHANNEL, workspace, ws_bytes, err, st);
+    return tc_dispatch(q, k, v, g, nullptr, eg, wg, S0, out, S_final, B, T, H, cu, n_seq, gate,
+                       workspace, ws_bytes, err, st);
 }
 
 }  // namespace gdr_host

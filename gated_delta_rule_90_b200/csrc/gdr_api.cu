@@ -27,8 +27,8 @@ cudaError_t fwd_simt_gdn2_dispatch(const void *q, const void *k, const void *v, 
 cudaError_t fwd_tc_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
                                  const float *eg, const float *wg, const float *S0, void *out,
                                  float *S_final, int B, int T, int H, const int32_t *cu, int n_seq,
-                                 void *workspace, size_t ws_bytes, unsigned int *err,
-                                 cudaStream_t st);
+                                 gdr_gate gate, void *workspace, size_t ws_bytes,
+                                 unsigned int *err, cudaStream_t st);
 cudaError_t decode_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
                                  const float *eg, const float *wg, float *S, void *out, int N,
                                  int H, int dk, int dv, gdr_dtype dtype, gdr_gate gate,
@@ -139,10 +139,10 @@ gdr_status resolve_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_path pat
     return GDR_OK;
 }
 
-// Gated DeltaNet-2 takes the tensor-core path only with the per-channel decay.
-gdr_status resolve_gdn2_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate gate,
+// Gated DeltaNet-2 takes the tensor-core path with either decay.
+gdr_status resolve_gdn2_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate,
                              gdr_path path, bool *use_tc) {
-    const bool tc = gdr_host::tc_applies(dk, dv, chunk, dtype) && gate == GDR_GATE_PER_KEY_CHANNEL;
+    const bool tc = gdr_host::tc_applies(dk, dv, chunk, dtype);
     switch (path) {
         case GDR_PATH_AUTO: *use_tc = tc; break;
         case GDR_PATH_SIMT: *use_tc = false; break;
@@ -284,7 +284,7 @@ gdr_status gdr_fwd_gdn2(const void *q, const void *k, const void *v, const float
         if (need && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
             return GDR_ERR_INVALID;
         e = gdr_host::fwd_tc_gdn2_dispatch(q, k, v, g, b, w, S0, out, S_final, B, T, H,
-                                           cu_seqlens, nseq, workspace, workspace_bytes,
+                                           cu_seqlens, nseq, gate, workspace, workspace_bytes,
                                            gdr_host::device_error_word(), s);
     } else {
         if (gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL, true) >

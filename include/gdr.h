@@ -194,9 +194,10 @@ gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const fl
  *  g        [B, T, H] or [B, T, H, d_k]  fp32 log-decay
  *  b        [B, T, H, d_k]   fp32 erase gate;  w [B, T, H, d_v] fp32 write gate
  *  S0, S_final, cu_seqlens, n_seq, chunk, path, workspace: as for gdr_fwd.  The
- *  tensor-core path takes bf16 with d_k = d_v = 128, chunk 64 and the
- *  per-channel decay (the page's setting); everything else (chunk 16, 32, 64
- *  or 128, d_k, d_v multiples of 16 up to 128) runs on the CUDA cores in fp32.
+ *  tensor-core path takes bf16 with d_k = d_v = 128 and chunk 64, with the
+ *  per-channel decay (the page's setting) or a scalar one (broadcast over the
+ *  key channels inside the kernel); everything else (chunk 16, 32, 64 or 128,
+ *  d_k, d_v multiples of 16 up to 128) runs on the CUDA cores in fp32.
  *  gdr_fwd_gdn2_workspace_size gives the workspace (0 on the CUDA-core path).
  * gdr_decode_step_gdn2: one token per sequence in place on S_inout, with
  *  b [N, H, d_k] and w [N, H, d_v]; otherwise as gdr_decode_step.

@@ -120,7 +120,9 @@ def test_product_rejects_on_host(kw, expect):
 
 def test_gdn2_workspace_only_on_the_tensor_core_path():
     assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 1, "auto") > 0
-    assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 0, "auto") == 0
+    # the scalar decay takes the tensor-core path too (broadcast in the kernel)
+    assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 0, "auto") > 0
+    assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 0, 0, "auto") == 0
     assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 1, "simt") == 0
     assert binding.fwd_gdn2_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 1, "auto") == \
         binding.fwd_workspace_size(2, 256, 4, 128, 128, 64, 2, False, 1, 1, "auto")

@@ -58,11 +58,25 @@ def test_gdn2_bf16_d128(cuda_device, gate, chunk):
     check(inputs.gdn2_inputs(cfg, seed=602), cuda_device, chunk)
 
 
+@pytest.mark.parametrize("gate", ["channel", "scalar"])
 @pytest.mark.parametrize("T", [64, 300, 1])
-def test_gdn2_tc_against_oracle(cuda_device, T):
-    """The tensor-core path (bf16, d = 128, C = 64, per-channel decay)."""
-    cfg = cfg_of(B=2, T=T, H=3, s0_var=0.01)
+def test_gdn2_tc_against_oracle(cuda_device, T, gate):
+    """The tensor-core path (bf16, d = 128, C = 64), per-channel decay or a
+    scalar one broadcast inside the WY kernel."""
+    cfg = cfg_of(B=2, T=T, H=3, s0_var=0.01, gate=gate,
+                 gate_scale=0.05 if gate == "channel" else 0.1)
     check(inputs.gdn2_inputs(cfg, seed=611), cuda_device, path="tc")
+
+
+def test_gdn2_tc_scalar_decay_matches_broadcast_channel_decay(cuda_device):
+    """A scalar decay on the tensor-core path equals the same decay given per
+    channel (broadcast on the host): the kernel's in-tile broadcast is exact."""
+    cfg = cfg_of(B=1, T=333, H=2, s0_var=0.01, gate="scalar", gate_scale=0.1)
+    inp = inputs.gdn2_inputs(cfg, seed=615)
+    O1, S1 = run_gpu(inp, cuda_device, path="tc")
+    inp.g = np.ascontiguousarray(np.broadcast_to(inp.g[..., None], inp.g.shape + (128,)))
+    O2, S2 = run_gpu(inp, cuda_device, path="tc")
+    assert np.array_equal(O1, O2) and np.array_equal(S1, S2)
 
 
 def test_gdn2_tc_varlen_with_empty_and_unit_sequences(cuda_device):
