@@ -146,28 +146,27 @@ constexpr uint32_t kWyTmemCols = 128;
 constexpr int kWyTmaThread = 128;
 
 // Shared-memory plan (byte offsets from a 1024-aligned base).  Regions are
-// reused once their first contents are dead, so a scalar-gate CTA needs
-// 74 KB and three fit on an SM:
+// reused once their first contents are dead, so a CTA needs 74 KB and three
+// fit on an SM, for either gate:
 //   KQ  [0, 32K)     raw K (rows 0-63) and Q (rows 64-127) in two 128-byte atom
-//                    columns.  Scalar gate: V replaces Q once Q is read; per-channel
-//                    gate: K^ and Q^ in place.  At the end: U^T / W^T staging.
-//   TT  [32K, 40K)   A staging for its TMA store, then T.
+//                    columns (per-channel gate: K^ and Q^ in place); V replaces Q
+//                    once the Gram has read it.  At the end: U^T staging.
+//   TT  [32K, 40K)   per-channel gate: the rows R, G_C and e^(G_C - R) until the
+//                    Gram; then A staging for its TMA store, then T.
 //   NT  [40K, 56K)   N^T fp32 [64][64]; after the solve, K<- (bf16, 2 atoms).
-//                    Per-channel gate: NT and XR first hold the gate tile G.
+//                    Per-channel gate: NT and XR first hold the gate tile G, then
+//                    NT holds K-check (the Gram's B operand).
 //   XR  [56K, 72.3K) X fp32 [64][65].
-//   per-channel gate only: V [73K, 89K) and K-check [89K, 105K).
+//   then the small region: scalar gate G and beta per row; per-channel gate beta
+//   and e^R per channel; two mbarriers and the TMEM slot.  The scalar gate's Gram
+//   factors e^(G - R), e^(R - G) and their flag live in XR, dead until the solve.
 struct WySmem {
     static constexpr uint32_t KQ = 0, TT = 32768, NT = 40960, XR = 57344;
     static constexpr int NTS = 64;                                   // N^T row stride (floats)
     static constexpr int XST = 65;                                   // X row stride (floats)
     static constexpr uint32_t XEND = XR + 64 * XST * 4;
-    static constexpr uint32_t VCH = 74752, KC = VCH + 16384;
-    static constexpr uint32_t small(bool ch) { return ch ? KC + 16384 : XEND; }
-    // scalar gate: G and beta per row; per-channel gate: R, G_C, beta, e^R and
-    // e^(G_C - R) per channel; then two mbarriers and the TMEM slot.  The
-    // scalar gate's Gram factors e^(G - R), e^(R - G) and their flag live in XR,
-    // which is dead until the solve.
-    static constexpr int small_floats(bool ch) { return ch ? 2 * D + 64 + 2 * D : 128; }
+    static constexpr uint32_t small(bool) { return XEND; }
+    static constexpr int small_floats(bool ch) { return ch ? 64 + D : 128; }
     static constexpr uint32_t small_bytes(bool ch) { return small_floats(ch) * 4 + 64; }
 };
 
@@ -179,7 +178,7 @@ struct WySmem {
 // BC (with CH): the decay is one scalar per token, broadcast over the key
 // channels of the gate tile in shared memory instead of loaded per channel.
 template <bool CH, bool DEC = false, bool BC = false>
-__global__ void __launch_bounds__(kWyThreads)
+__global__ void __launch_bounds__(kWyThreads, CH ? 3 : 0)
 wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
           const __grid_constant__ CUtensorMap tm_Ust,
@@ -192,20 +191,21 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     uint8_t *sm = align1024(smem_raw);
     uint8_t *sKQ = sm + WySmem::KQ, *sT = sm + WySmem::TT;
     uint8_t *sKL = sm + WySmem::NT;                                    // after the solve
-    uint8_t *sV = CH ? sm + WySmem::VCH : sKQ + 8192;                  // scalar gate: Q's place
-    uint8_t *sKC = sm + WySmem::KC;                                    // per-channel gate only
+    uint8_t *sV = sKQ + 8192;                                          // Q's place, after the Gram
+    uint8_t *sKC = sm + WySmem::NT;                                    // per-channel gate only
     float *sN = reinterpret_cast<float *>(sm + WySmem::NT);            // N^T [m][l]
     float *sX = reinterpret_cast<float *>(sm + WySmem::XR);            // X [row][col]
     float *sGt = reinterpret_cast<float *>(sm + WySmem::NT);           // per-channel G [64][128]
     float *sSm = reinterpret_cast<float *>(sm + WySmem::small(CH));
-    float *sG = sSm;                                                   // scalar: G [64]; channel: R row [128]
-    float *sGC = sSm + (CH ? D : 64);                                  // channel: G_C row [128]
-    float *sB = CH ? sGC + D : sSm + 64;                               // beta [64]
+    float *sTf = reinterpret_cast<float *>(sm + WySmem::TT);
+    float *sG = CH ? sTf : sSm;                                        // scalar: G [64]; channel: R row [128]
+    float *sGC = sTf + D;                                              // channel: G_C row [128]
+    float *sB = CH ? sSm : sSm + 64;                                   // beta [64]
     // exponential tables, so that no element-wise exp is needed below
-    float *eR = sB + 64, *eCR = sB + 64 + D;                           // channel: per channel
+    float *eR = sSm + 64, *eCR = sTf + 2 * D;                          // channel: per channel
     float *eA = sX, *eB = sX + 64;                                     // scalar: per row (XR)
     int *sFact = reinterpret_cast<int *>(sX + 128);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + 64 + (CH ? 2 * D : 0));  // [2]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sSm + WySmem::small_floats(CH));  // [2]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -227,16 +227,12 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_arrive_expect_tx(&bars[0], 4 * kHalfBytes + (CH ? 2 * kHalfBytes + (BC ? 0 : C * D * 4) : 0));
+        mbar_arrive_expect_tx(&bars[0], 4 * kHalfBytes + (CH && !BC ? C * D * 4 : 0));
         tma_load_2d(sKQ, &tm_k, &bars[0], x0, ytok);
         tma_load_2d(sKQ + 16384, &tm_k, &bars[0], x0 + 64, ytok);
         tma_load_2d(sKQ + 8192, &tm_q, &bars[0], x0, ytok);
         tma_load_2d(sKQ + 16384 + 8192, &tm_q, &bars[0], x0 + 64, ytok);
-        if (CH) {
-            tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
-            tma_load_2d(sV + 8192, &tm_v, &bars[0], x0 + 64, ytok);
-            if (!BC) tma_load_2d(sGt, &tm_g, &bars[0], x0, ytok);  // [64][128] fp32 per-channel gates
-        }
+        if (CH && !BC) tma_load_2d(sGt, &tm_g, &bars[0], x0, ytok);  // [64][128] fp32 per-channel gates
     }
     if (warp == 0) {
         tmem_alloc(tslot, kWyTmemCols);
@@ -335,6 +331,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         __nv_bfloat16 *Qg = ws.Q + slot * (C * D), *Kg = ws.K + slot * (C * D);
         const int cg = tid & 15, c0 = cg * 8, a = cg >> 3, l0 = tid >> 4;
         float R8[8], eR8[8], eCR8[8];
+        uint4 kcv[C / 16];  // per-channel gate: K-check, stored once G is read
         if (CH) {
             ld8(sG + c0, R8);
             ld8(eR + c0, eR8);
@@ -350,21 +347,14 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             if (CH) {
                 float kh[8], qh[8], kc[8], G8[8], b8[8];
                 ld8(sGt + l * D + c0, G8);
-                if (DEC) {  // erase gate of this row (reading side); write gate into V
+                if (DEC) {  // erase gate of this row (reading side)
                     const size_t gro = ((size_t)(tstart + l) * geo.H + h) * D + c0;
-                    float w8[8], vv[8];
                     if (l < len) {
                         ld8(eg + gro, b8);
-                        ld8(wg + gro, w8);
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) b8[i] = w8[i] = 0.f;
+                        for (int i = 0; i < 8; ++i) b8[i] = 0.f;
                     }
-                    uint4 *vp = reinterpret_cast<uint4 *>(sV + a * 8192 + l * 128 + j * 16);
-                    unpack8(*vp, vv);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) vv[i] *= w8[i];
-                    *vp = pack8(vv);
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -378,7 +368,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 }
                 *reinterpret_cast<uint4 *>(sKQ + off) = pack8(kh);
                 *reinterpret_cast<uint4 *>(sKQ + off + 8192) = pack8(qh);
-                *reinterpret_cast<uint4 *>(sKC + a * 8192 + l * 128 + j * 16) = pack8(kc);
+                kcv[k] = pack8(kc);
             } else {
                 const float eq = __expf(sG[l]), ek = __expf(sG[C - 1] - sG[l]);
 #pragma unroll
@@ -391,6 +381,14 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             *reinterpret_cast<uint4 *>(Kg + l * D + c0) = pack8(wk);
         }
         if (tid < D) ws.dec[slot * D + tid] = CH ? eCR[tid] * eR[tid] : __expf(sG[C - 1]);
+        if (CH) {  // the gate tile is read: K-check takes its first half
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < C / 16; ++k) {
+                const int l = l0 + 16 * k, j = (cg & 7) ^ (l & 7);
+                *reinterpret_cast<uint4 *>(sKC + a * 8192 + l * 128 + j * 16) = kcv[k];
+            }
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -464,11 +462,10 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     if (tid == kWyTmaThread) {  // A -> workspace
         tma_store_2d(&tm_Ast, sT, 0, (int)(slot * C));
         bulk_commit_group();
-        if (!CH) {  // Q is read: V takes its place (lands during the solve)
-            mbar_arrive_expect_tx(&bars[0], 2 * kHalfBytes);
-            tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
-            tma_load_2d(sV + 16384, &tm_v, &bars[0], x0 + 64, ytok);
-        }
+        // Q is read: V takes its place (lands during the solve)
+        mbar_arrive_expect_tx(&bars[0], 2 * kHalfBytes);
+        tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
+        tma_load_2d(sV + 16384, &tm_v, &bars[0], x0 + 64, ytok);
     }
     // T = (I + N)^{-1} diag(beta), N = diag(beta) L strictly lower, by 16 x 16
     // blocks: X_ii = (I + N_ii)^{-1} by forward substitution (one column per
@@ -598,9 +595,28 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             }
         }
     }
-    if (!CH) {  // V has landed in Q's place
+    {  // V has landed in Q's place
         const bool okv = mbar_wait_bounded(&bars[0], 1, kSpin, err);
         if (!__syncthreads_and(okv)) goto cleanup;
+    }
+    if (DEC) {  // the write gate: V <- w . V (zero beyond the sequence end)
+        const int cg = tid & 15, c0 = cg * 8, a = cg >> 3, l0 = tid >> 4;
+#pragma unroll
+        for (int k = 0; k < C / 16; ++k) {
+            const int l = l0 + 16 * k, j = (cg & 7) ^ (l & 7);
+            float w8[8], vv[8];
+            if (l < len) {
+                ld8(wg + ((size_t)(tstart + l) * geo.H + h) * D + c0, w8);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w8[i] = 0.f;
+            }
+            uint4 *vp = reinterpret_cast<uint4 *>(sV + a * 16384 + l * 128 + j * 16);
+            unpack8(*vp, vv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) vv[i] *= w8[i];
+            *vp = pack8(vv);
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -610,7 +626,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         tc_fence_after();
         const uint32_t id = idesc_bf16(128, 64, 1, 0);
         const uint64_t bd = sdesc_sw128(smem_u32(sT), 16, 1024);
-        const uint64_t av = sdesc_sw128(smem_u32(sV), CH ? 8192 : 16384, 1024);
+        const uint64_t av = sdesc_sw128(smem_u32(sV), 16384, 1024);
         const uint64_t ak = sdesc_sw128(smem_u32(sKL), 8192, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
