@@ -795,7 +795,11 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
         const int d = (warp & 3) * 32 + lane;
         const size_t soff = ((size_t)s * geo.H + h) * (size_t)D * D + (size_t)d * D + (warp >> 2) * 64;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) s0v[i] = S0 ? S0[soff + i] : 0.f;
+        for (int i4 = 0; i4 < 16; ++i4) {  // 16-byte loads (S0 rows are 16-byte aligned)
+            const float4 t = S0 ? reinterpret_cast<const float4 *>(S0 + soff)[i4]
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            s0v[4 * i4] = t.x; s0v[4 * i4 + 1] = t.y; s0v[4 * i4 + 2] = t.z; s0v[4 * i4 + 3] = t.w;
+        }
     }
     tc_fence_before();
     __syncthreads();
