@@ -220,8 +220,10 @@ static cudaError_t launch_inverse(float *GW, const Dims &d, unsigned int *err, c
 // S_t = (S_{t-1} D_t + C_t) W_t for kChainRows rows of S; every S_t is stored
 // for the output pass (fp32, or its bf16 copy for the tensor-core output pass),
 // the last one also as S_final.  W_t arrives by bulk copy into one of two
-// buffers, one frame ahead; thread (row r, 8 columns) first forms its 8 entries
-// of S_{t-1} D_t + C_t, then keeps 8 independent sums of the product with W_t.
+// buffers, one frame ahead.  Thread (row pair rp = warp, column group cg =
+// lane) owns rows 2 rp, 2 rp + 1 and columns 4 cg .. 4 cg + 3: each float4 read
+// of a W_t row serves both rows (the chain is bound by shared-memory reads),
+// and a warp's reads of S are broadcasts.
 __global__ void __launch_bounds__(kThreads)
 frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
                    const float *__restrict__ g, int per_channel,
@@ -236,11 +238,9 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
     // W_t double buffer (unpadded, as copied), then S rows [16][dk + 4]
     float *Mb = sm, *S = Mb + 2 * dk * dk;
     uint64_t *bar = reinterpret_cast<uint64_t *>(S + kChainRows * sst);  // [2]
-    // thread (row r, group cg): columns ca..ca+3 and cb..cb+3 of the row, so
-    // that each float4 read of a W_t row by 16 threads covers 256 contiguous bytes
-    const int tid = threadIdx.x, r = tid >> 4, cg = tid & 15;
-    const int ca = 4 * cg, cb = dk / 2 + 4 * cg;
-    const bool mine = r < nr && cg < dk / 8;
+    const int tid = threadIdx.x, rp = tid >> 5, cg = tid & 31, c4 = 4 * cg;
+    const bool colok = c4 < dk;
+    const bool mine0 = colok && 2 * rp < nr, mine1 = colok && 2 * rp + 1 < nr;
     const uint32_t mbytes = (uint32_t)(dk * dk * 4);
     const size_t soff = ((size_t)b * d.H + h) * (size_t)d.dv * dk;
     if (tid == 0) {
@@ -261,57 +261,55 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
                       &bar[issued]);
         }
     bool ok = true;
-    float *Sr = S + r * sst;
-    // C_t row entries and log-decays of this thread's columns, loaded one frame
+    float *Sr0 = S + (2 * rp) * sst, *Sr1 = Sr0 + sst;
+    // C_t entries and log-decays of this thread's columns, loaded one frame
     // ahead so that their latency stays off the chain
-    float cv[8], gv[8];
+    float4 cv0, cv1, gv;
     auto fetch = [&](int f) {
         const size_t sl = slot(d, b, f, h);
-        const float *crow = Cw + sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk;
-        const float4 x = *reinterpret_cast<const float4 *>(crow + ca);
-        const float4 y = *reinterpret_cast<const float4 *>(crow + cb);
-        cv[0] = x.x; cv[1] = x.y; cv[2] = x.z; cv[3] = x.w;
-        cv[4] = y.x; cv[5] = y.y; cv[6] = y.z; cv[7] = y.w;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            gv[j] = per_channel ? g[sl * dk + (j < 4 ? ca : cb - 4) + j] : g[sl];
+        const float *crow = Cw + sl * (size_t)d.dv * dk + (size_t)(r0 + 2 * rp) * dk + c4;
+        cv0 = mine0 ? *reinterpret_cast<const float4 *>(crow) : make_float4(0.f, 0.f, 0.f, 0.f);
+        cv1 = mine1 ? *reinterpret_cast<const float4 *>(crow + dk) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (per_channel) {
+            gv = *reinterpret_cast<const float4 *>(g + sl * dk + c4);
+        } else {
+            const float gs = g[sl];
+            gv = make_float4(gs, gs, gs, gs);
+        }
     };
-    if (mine) fetch(0);
+    if (colok) fetch(0);
     for (int f = 0; f < d.F; ++f) {
         const size_t sl = slot(d, b, f, h);
         const float *Mf = Mb + (f & 1) * dk * dk;
-        float acc[8];
-        if (mine) {  // S_{t-1} D_t + C_t, this thread's entries
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int c = (j < 4 ? ca : cb - 4) + j;
-                Sr[c] = fmaf(Sr[c], expf(gv[j]), cv[j]);
-                acc[j] = 0.f;
-            }
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        if (colok) {  // S_{t-1} D_t + C_t, this thread's entries
+            const float4 av = make_float4(expf(gv.x), expf(gv.y), expf(gv.z), expf(gv.w));
+            float4 *p0 = reinterpret_cast<float4 *>(Sr0 + c4), *p1 = reinterpret_cast<float4 *>(Sr1 + c4);
+            const float4 x0 = *p0, x1 = *p1;
+            *p0 = make_float4(fmaf(x0.x, av.x, cv0.x), fmaf(x0.y, av.y, cv0.y), fmaf(x0.z, av.z, cv0.z),
+                              fmaf(x0.w, av.w, cv0.w));
+            *p1 = make_float4(fmaf(x1.x, av.x, cv1.x), fmaf(x1.y, av.y, cv1.y), fmaf(x1.z, av.z, cv1.z),
+                              fmaf(x1.w, av.w, cv1.w));
             if (f + 1 < d.F) fetch(f + 1);
         }
         const bool okw = mbar_wait_bounded(&bar[f & 1], (f >> 1) & 1, kSpinF, err);
         if (!__syncthreads_and(okw)) { ok = false; break; }
-        if (mine) {  // 4 rows of W_t per round, every load issued before the FMAs
+        if (colok) {  // 4 rows of W_t per round, every load issued before the FMAs
             for (int m0 = 0; m0 < dk; m0 += 4) {
-                const float4 s4 = *reinterpret_cast<const float4 *>(Sr + m0);
-                const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-                float4 wa[4], wb[4];
+                const float4 s0 = *reinterpret_cast<const float4 *>(Sr0 + m0);
+                const float4 s1 = *reinterpret_cast<const float4 *>(Sr1 + m0);
+                const float sv0[4] = {s0.x, s0.y, s0.z, s0.w}, sv1[4] = {s1.x, s1.y, s1.z, s1.w};
+                float4 w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const float4 *>(Mf + (m0 + i) * dk + c4);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    wa[i] = *reinterpret_cast<const float4 *>(Mf + (m0 + i) * dk + ca);
-                    wb[i] = *reinterpret_cast<const float4 *>(Mf + (m0 + i) * dk + cb);
-                }
+                    const float wv[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    acc[0] = fmaf(sv[i], wa[i].x, acc[0]);
-                    acc[1] = fmaf(sv[i], wa[i].y, acc[1]);
-                    acc[2] = fmaf(sv[i], wa[i].z, acc[2]);
-                    acc[3] = fmaf(sv[i], wa[i].w, acc[3]);
-                    acc[4] = fmaf(sv[i], wb[i].x, acc[4]);
-                    acc[5] = fmaf(sv[i], wb[i].y, acc[5]);
-                    acc[6] = fmaf(sv[i], wb[i].z, acc[6]);
-                    acc[7] = fmaf(sv[i], wb[i].w, acc[7]);
+                    for (int j = 0; j < 4; ++j) {
+                        acc0[j] = fmaf(sv0[i], wv[j], acc0[j]);
+                        acc1[j] = fmaf(sv1[i], wv[j], acc1[j]);
+                    }
                 }
             }
         }
@@ -322,28 +320,28 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
                       &bar[f & 1]);
             issued = f + 3;
         }
-        if (mine) {
-            *reinterpret_cast<float4 *>(Sr + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            *reinterpret_cast<float4 *>(Sr + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-            const size_t o = sl * (size_t)d.dv * dk + (size_t)(r0 + r) * dk;
+        if (colok) {
+            *reinterpret_cast<float4 *>(Sr0 + c4) = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
+            *reinterpret_cast<float4 *>(Sr1 + c4) = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
+            const size_t o = sl * (size_t)d.dv * dk + (size_t)(r0 + 2 * rp) * dk + c4;
             if (Sb) {  // operand of the tensor-core output pass
-                __nv_bfloat162 pa[2] = {__floats2bfloat162_rn(acc[0], acc[1]),
-                                        __floats2bfloat162_rn(acc[2], acc[3])};
-                __nv_bfloat162 pb[2] = {__floats2bfloat162_rn(acc[4], acc[5]),
-                                        __floats2bfloat162_rn(acc[6], acc[7])};
-                *reinterpret_cast<uint2 *>(Sb + o + ca) = *reinterpret_cast<uint2 *>(pa);
-                *reinterpret_cast<uint2 *>(Sb + o + cb) = *reinterpret_cast<uint2 *>(pb);
+                __nv_bfloat162 p0[2] = {__floats2bfloat162_rn(acc0[0], acc0[1]),
+                                        __floats2bfloat162_rn(acc0[2], acc0[3])};
+                __nv_bfloat162 p1[2] = {__floats2bfloat162_rn(acc1[0], acc1[1]),
+                                        __floats2bfloat162_rn(acc1[2], acc1[3])};
+                if (mine0) *reinterpret_cast<uint2 *>(Sb + o) = *reinterpret_cast<uint2 *>(p0);
+                if (mine1) *reinterpret_cast<uint2 *>(Sb + o + dk) = *reinterpret_cast<uint2 *>(p1);
             } else {
-                *reinterpret_cast<float4 *>(Sw + o + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                *reinterpret_cast<float4 *>(Sw + o + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                if (mine0) *reinterpret_cast<float4 *>(Sw + o) = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
+                if (mine1) *reinterpret_cast<float4 *>(Sw + o + dk) = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
             }
         }
         __syncthreads();
     }
-    if (ok && S_final && mine) {
-        float *o = S_final + soff + (size_t)(r0 + r) * dk;
-        *reinterpret_cast<float4 *>(o + ca) = *reinterpret_cast<const float4 *>(Sr + ca);
-        *reinterpret_cast<float4 *>(o + cb) = *reinterpret_cast<const float4 *>(Sr + cb);
+    if (ok && S_final && colok) {
+        float *o = S_final + soff + (size_t)(r0 + 2 * rp) * dk + c4;
+        if (mine0) *reinterpret_cast<float4 *>(o) = *reinterpret_cast<const float4 *>(Sr0 + c4);
+        if (mine1) *reinterpret_cast<float4 *>(o + dk) = *reinterpret_cast<const float4 *>(Sr1 + c4);
     }
     if (tid == 0)  // copies still in flight (error path) land before exit
         for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait_bounded(&bar[i & 1], (i >> 1) & 1, kSpinF, err);
