@@ -122,84 +122,94 @@ frame_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
 // row's threads during the previous step: one barrier per pivot.  W_t
 // overwrites G_t.
 constexpr int kSwThreads = 512;  // (d_k / 4) x (d_k / 8) tiles of 4 x 8, d_k <= 128
+// Thread (row group rg, column group cg) holds rows 4 rg .. 4 rg + 3 and the
+// columns 4 cg .. 4 cg + 3 and d_k/2 + 4 cg .. + 3, so that the float4 reads of
+// a pivot row by the column groups cover contiguous bytes (no bank conflicts).
 template <int DK>
 __global__ void __launch_bounds__(kSwThreads, 2)
 frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
     __shared__ __align__(16) float buf[2][128];  // pivot rows
-    constexpr int NCG = DK / 8, NRG = DK / 4;     // column / row groups
+    constexpr int NCG = DK / 8, NRG = DK / 4, HALF = DK / 2;  // column / row groups
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, cg = tid % NCG, rg = tid / NCG;
     const bool act = rg < NRG;
-    const int r0 = 4 * rg, j0 = 8 * cg;
+    const int r0 = 4 * rg, jA = 4 * cg, jB = HALF + 4 * cg;
     const size_t sl = slot(d, b, f, h);
     float *Gp = GW + sl * (size_t)DK * DK;
+    auto col = [&](int u) { return u < 4 ? jA + u : jB + u - 4; };
     float a[4][8];
     if (act) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float4 x = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + j0);
-            const float4 y = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + j0 + 4);
+            const float4 x = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + jA);
+            const float4 y = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + jB);
             a[i][0] = x.x; a[i][1] = x.y; a[i][2] = x.z; a[i][3] = x.w;
             a[i][4] = y.x; a[i][5] = y.y; a[i][6] = y.z; a[i][7] = y.w;
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {  // G^T: column j0 + u, rows r0..r0+3
-            const float4 t = *reinterpret_cast<const float4 *>(Gp + (size_t)(j0 + u) * DK + r0);
+        for (int u = 0; u < 8; ++u) {  // G^T: column col(u), rows r0..r0+3
+            const float4 t = *reinterpret_cast<const float4 *>(Gp + (size_t)col(u) * DK + r0);
             const float tv[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                a[i][u] = 0.5f * (a[i][u] + tv[i]) + (r0 + i == j0 + u ? 1.f : 0.f);
+                a[i][u] = 0.5f * (a[i][u] + tv[i]) + (r0 + i == col(u) ? 1.f : 0.f);
         }
         if (rg == 0) {
-            *reinterpret_cast<float4 *>(&buf[0][j0]) = make_float4(a[0][0], a[0][1], a[0][2], a[0][3]);
-            *reinterpret_cast<float4 *>(&buf[0][j0 + 4]) = make_float4(a[0][4], a[0][5], a[0][6], a[0][7]);
+            *reinterpret_cast<float4 *>(&buf[0][jA]) = make_float4(a[0][0], a[0][1], a[0][2], a[0][3]);
+            *reinterpret_cast<float4 *>(&buf[0][jB]) = make_float4(a[0][4], a[0][5], a[0][6], a[0][7]);
         }
     }
     __syncthreads();
-    for (int k8 = 0; k8 < DK; k8 += 8) {
+    // pivot k: column k is local column (k >= d_k/2 ? 4 : 0) + k % 4 of column
+    // group (k % (d_k/2)) / 4; the two halves of the pivots are separate loops so
+    // that this index is a compile-time constant
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const int k = k8 + kk;
-            const float *bk = buf[kk & 1];
-            const float dkk = bk[k];
-            if (tid == 0 && !(dkk > 0.f)) atomicOr(err, kErrNumeric);
-            const float sq = rsqrtf(dkk);
-            if (act) {
-                const float4 br4 = *reinterpret_cast<const float4 *>(bk + r0);
-                const float4 bj0 = *reinterpret_cast<const float4 *>(bk + j0);
-                const float4 bj1 = *reinterpret_cast<const float4 *>(bk + j0 + 4);
-                const float cr[4] = {br4.x * sq, br4.y * sq, br4.z * sq, br4.w * sq};
-                const float cj[8] = {bj0.x * sq, bj0.y * sq, bj0.z * sq, bj0.w * sq,
-                                     bj1.x * sq, bj1.y * sq, bj1.z * sq, bj1.w * sq};
-                const bool krow = (k >> 2) == rg, kcol = (k >> 3) == cg;
-                const int ki = kk & 3;  // the pivot's row inside a tile (unrolled: a constant)
+    for (int hk = 0; hk < 2; ++hk) {
+        for (int k4 = 0; k4 < HALF; k4 += 4) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if (i == ki && krow) {  // row k
+            for (int kk = 0; kk < 4; ++kk) {
+                const int k = hk * HALF + k4 + kk;
+                const int uk = 4 * hk + kk;  // the pivot's local column
+                const float *bk = buf[k & 1];
+                const float dkk = bk[k];
+                if (tid == 0 && !(dkk > 0.f)) atomicOr(err, kErrNumeric);
+                const float sq = rsqrtf(dkk);
+                if (act) {
+                    const float4 br4 = *reinterpret_cast<const float4 *>(bk + r0);
+                    const float4 bj0 = *reinterpret_cast<const float4 *>(bk + jA);
+                    const float4 bj1 = *reinterpret_cast<const float4 *>(bk + jB);
+                    const float cr[4] = {br4.x * sq, br4.y * sq, br4.z * sq, br4.w * sq};
+                    const float cj[8] = {bj0.x * sq, bj0.y * sq, bj0.z * sq, bj0.w * sq,
+                                         bj1.x * sq, bj1.y * sq, bj1.z * sq, bj1.w * sq};
+                    const bool krow = (k >> 2) == rg, kcol = (k4 >> 2) == cg;
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) a[i][u] = (u == kk && kcol) ? -(sq * sq) : cj[u] * sq;
-                    } else {
+                    for (int i = 0; i < 4; ++i) {
+                        if (i == kk && krow) {  // row k
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) a[i][u] = fmaf(-cr[i], cj[u], a[i][u]);
-                        if (kcol) a[i][kk] = cr[i] * sq;  // column k
+                            for (int u = 0; u < 8; ++u) a[i][u] = (u == uk && kcol) ? -(sq * sq) : cj[u] * sq;
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) a[i][u] = fmaf(-cr[i], cj[u], a[i][u]);
+                            if (kcol) a[i][uk] = cr[i] * sq;  // column k
+                        }
+                    }
+                    if (((k + 1) >> 2) == rg && k + 1 < DK) {  // publish the next pivot row
+                        const int ni = (kk + 1) & 3;
+                        float *bn = buf[(k + 1) & 1];
+                        *reinterpret_cast<float4 *>(bn + jA) = make_float4(a[ni][0], a[ni][1], a[ni][2], a[ni][3]);
+                        *reinterpret_cast<float4 *>(bn + jB) = make_float4(a[ni][4], a[ni][5], a[ni][6], a[ni][7]);
                     }
                 }
-                const int ni = (kk + 1) & 3;  // the next pivot's row inside a tile
-                if (((k + 1) >> 2) == rg) {
-                    float *bn = buf[(kk + 1) & 1];
-                    *reinterpret_cast<float4 *>(bn + j0) = make_float4(a[ni][0], a[ni][1], a[ni][2], a[ni][3]);
-                    *reinterpret_cast<float4 *>(bn + j0 + 4) = make_float4(a[ni][4], a[ni][5], a[ni][6], a[ni][7]);
-                }
+                __syncthreads();
             }
-            __syncthreads();
         }
     }
     if (act) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float4 *o = reinterpret_cast<float4 *>(Gp + (size_t)(r0 + i) * DK + j0);
-            o[0] = make_float4(-a[i][0], -a[i][1], -a[i][2], -a[i][3]);
-            o[1] = make_float4(-a[i][4], -a[i][5], -a[i][6], -a[i][7]);
+            float *o = Gp + (size_t)(r0 + i) * DK;
+            *reinterpret_cast<float4 *>(o + jA) = make_float4(-a[i][0], -a[i][1], -a[i][2], -a[i][3]);
+            *reinterpret_cast<float4 *>(o + jB) = make_float4(-a[i][4], -a[i][5], -a[i][6], -a[i][7]);
         }
     }
 }
