@@ -48,8 +48,8 @@ NCU_TRAFFIC = {
     ("tc_wy", "kda_prefill"): (_TC_SRC, "c273c89937938c42", 681.130752e6 + 579.557120e6),
     ("decode", "decode"): (_DEC_SRC, "82e1f5016f476188", 543.250944e6 + 482.361600e6),
     ("decode", "kda_decode"): (_DEC_SRC, "82e1f5016f476188", 547.403264e6 + 482.458624e6),
-    ("frame_chain", "frame_prefill"): (_FR_SRC, "ebb311790167a782", 33.712128e6 + 0.0),
-    ("frame_solve", "frame_prefill"): (_FR_SRC, "ebb311790167a782", 16.801280e6 + 0.0),
+    ("frame_chain", "frame_prefill"): (_FR_SRC, "2984ca0634014dc4", 33.711104e6 + 0.0),
+    ("frame_solve", "frame_prefill"): (_FR_SRC, "2984ca0634014dc4", 16.795136e6 + 0.002048e6),
 }
 
 
