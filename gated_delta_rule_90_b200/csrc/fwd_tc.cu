@@ -59,6 +59,10 @@ constexpr uint32_t kDecBytes = D * 4;
 struct Geo {
     int B, T, H, n_seq, nc;  // nc: chunks per sequence (regular batches)
     int varlen, T_total, n_slots;
+    // > 1: the rows are a Gated DeltaProduct virtual sequence with keep
+    // substeps per token; out has one row per token and receives the last
+    // substep's output only
+    int keep;
 };
 
 struct Ws {
@@ -916,7 +920,47 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             if (lane == 0) mbar_arrive(&oFree[r & 1]);
             const long ts = t0 + (long)r * C;
             const int len = (int)min((long)C, t1 - ts);
-            if (len == C) {
+            const int kp = geo.keep;
+            if (kp > 1 && len == C && C % kp == 0 && ts % kp == 0) {
+                // the last substep of each token: C / kp rows staged, one TMA store
+                if (otid == 0) bulk_wait_group_read<0>();  // staging buffer free again
+                named_sync(1, kOutThreads);
+                if (kp == 2) {
+#pragma unroll
+                    for (int m = 0; m < 32; ++m) ost[m * D + d] = __float2bfloat16_rn(o[2 * m + 1]);
+                } else if (kp == 4) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) ost[m * D + d] = __float2bfloat16_rn(o[4 * m + 3]);
+                } else {
+                    int j = 0, m = 0;
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        if (j == kp - 1) {
+                            ost[m * D + d] = __float2bfloat16_rn(o[i]);
+                            ++m;
+                        }
+                        if (++j == kp) j = 0;
+                    }
+                }
+                fence_proxy_async_smem();
+                named_sync(1, kOutThreads);
+                if (otid == 0) {
+                    tma_store_2d(&tm_out, ost, h * D, (int)(ts / kp));
+                    bulk_commit_group();
+                }
+            } else if (kp > 1) {  // partial chunk, or kp not dividing C: plain stores
+                int j = (int)(ts % kp);
+                long t = ts / kp;
+                __nv_bfloat16 *og = out + (size_t)h * D + d;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    if (i < len && j == kp - 1) og[(size_t)t * geo.H * D] = __float2bfloat16_rn(o[i]);
+                    if (++j == kp) {
+                        j = 0;
+                        ++t;
+                    }
+                }
+            } else if (len == C) {
                 if (otid == 0) bulk_wait_group_read<0>();  // staging buffer free again
                 named_sync(1, kOutThreads);
 #pragma unroll
@@ -1052,7 +1096,8 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
                                const float *beta, const float *eg, const float *wg,
                                const float *S0, void *out, float *S_final, int B, int T, int H,
                                const int32_t *cu, int n_seq, gdr_gate gate, void *workspace,
-                               size_t ws_bytes, unsigned int *err, cudaStream_t st) {
+                               size_t ws_bytes, unsigned int *err, cudaStream_t st,
+                               int keep = 1) {
     const int varlen = cu != nullptr;
     const WsLayout L = ws_layout(B, T, H, n_seq, varlen);
     if (ws_bytes < L.total || !err) return cudaErrorInvalidValue;
@@ -1069,6 +1114,7 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
     Geo geo;
     geo.B = B; geo.T = T; geo.H = H; geo.n_seq = varlen ? n_seq : B;
     geo.nc = (T + C - 1) / C; geo.varlen = varlen; geo.T_total = B * T; geo.n_slots = L.n_slots;
+    geo.keep = keep;
 
     const size_t tiles = (size_t)L.n_slots * H;
     if (tiles * D >= ((size_t)1 << 31)) return cudaErrorInvalidValue;  // 32-bit TMA rows
@@ -1088,7 +1134,8 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
             !make_map(&mQ, kBF, ws.Q, D, tiles * C, D * 2, 64, 64, kSW) ||
             !make_map(&mK, kBF, ws.K, D, tiles * C, D * 2, 64, 64, kSW) ||
             !make_map(&mA, kBF, ws.A, C, tiles * C, C * 2, 64, 64, kSW) ||
-            !make_map(&mo, kBF, out, HD, tok_rows, HD * 2, D, 64, kNoSW))
+            !make_map(&mo, kBF, out, HD, tok_rows / keep, HD * 2, D,
+                      C % keep == 0 ? C / keep : 64, kNoSW))
             return cudaErrorInvalidValue;
     } else {
         memset(&mW, 0, sizeof(mW));
@@ -1139,6 +1186,19 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
                             cudaStream_t st) {
     return tc_dispatch(q, k, v, g, beta, nullptr, nullptr, S0, out, S_final, B, T, H, cu, n_seq,
                        gate, workspace, ws_bytes, err, st);
+}
+
+// Gated DeltaProduct: the prefill over the virtual sequence of keep substeps
+// per token (T virtual rows per sequence), out [B, T / keep, H, d_v] receiving
+// the last substep of each token.
+cudaError_t fwd_tc_keep_dispatch(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *S0, void *out, float *S_final,
+                                 int B, int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
+                                 int keep, void *workspace, size_t ws_bytes, unsigned int *err,
+                                 cudaStream_t st) {
+    if (keep < 1 || T % keep) return cudaErrorInvalidValue;
+    return tc_dispatch(q, k, v, g, beta, nullptr, nullptr, S0, out, S_final, B, T, H, cu, n_seq,
+                       gate, workspace, ws_bytes, err, st, keep);
 }
 
 // Gated DeltaNet-2: erase gate eg [.., d_k], write gate wg [.., d_v]; the decay

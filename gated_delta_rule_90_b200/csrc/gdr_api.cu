@@ -40,6 +40,11 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
                             const float *beta, const float *S0, void *out, float *S_final, int B,
                             int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
                             void *workspace, size_t ws_bytes, unsigned int *err, cudaStream_t st);
+cudaError_t fwd_tc_keep_dispatch(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *S0, void *out, float *S_final,
+                                 int B, int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
+                                 int keep, void *workspace, size_t ws_bytes, unsigned int *err,
+                                 cudaStream_t st);
 }  // namespace gdr_host
 
 // ------------------------------------------------------------ device error word
@@ -192,11 +197,17 @@ size_t gdr_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk, 
     return gdr_host::tc_workspace_bytes(B, T, H, n_seq, varlen, gate);
 }
 
-gdr_status gdr_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
-                   const float *S0, void *out, float *S_final, int B, int T, int H, int d_k,
-                   int d_v, int chunk, const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype,
-                   gdr_gate gate, gdr_path path, void *workspace, size_t workspace_bytes,
-                   void *stream) {
+// The prefill behind gdr_fwd.  keep > 1 (Gated DeltaProduct): the T rows of a
+// sequence are keep substeps per token and out holds one row per token, the
+// last substep's; only the tensor-core path does this, and where it does not
+// apply *ran is false and nothing is launched.
+static gdr_status fwd_common(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *S0, void *out, float *S_final, int B,
+                             int T, int H, int d_k, int d_v, int chunk,
+                             const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype, gdr_gate gate,
+                             gdr_path path, void *workspace, size_t workspace_bytes, void *stream,
+                             int keep, bool *ran) {
+    if (ran) *ran = false;
     // With no tokens (B*T == 0) the token tensors are empty and may be NULL.
     if ((long long)B * T > 0 && (!q || !k || !v || !g || !beta || !out)) return GDR_ERR_INVALID;
     if (!valid_enum(dtype, gate)) return GDR_ERR_INVALID;
@@ -209,6 +220,8 @@ gdr_status gdr_fwd(const void *q, const void *k, const void *v, const float *g, 
     bool use_tc = false;
     st = resolve_path(d_k, d_v, chunk, dtype, path, &use_tc);
     if (st != GDR_OK) return st;
+    if (keep > 1 && (!use_tc || T % keep)) return GDR_OK;  // the caller gathers
+    if (ran) *ran = true;
     const int nseq = varlen ? n_seq : B;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
@@ -216,9 +229,13 @@ gdr_status gdr_fwd(const void *q, const void *k, const void *v, const float *g, 
         const size_t need = gdr_host::tc_workspace_bytes(B, T, H, n_seq, varlen, gate);
         if (need && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
             return GDR_ERR_INVALID;
-        e = gdr_host::fwd_tc_dispatch(q, k, v, g, beta, S0, out, S_final, B, T, H, cu_seqlens,
-                                      nseq, gate, workspace, workspace_bytes,
-                                      gdr_host::device_error_word(), s);
+        e = keep > 1 ? gdr_host::fwd_tc_keep_dispatch(q, k, v, g, beta, S0, out, S_final, B, T, H,
+                                                      cu_seqlens, nseq, gate, keep, workspace,
+                                                      workspace_bytes,
+                                                      gdr_host::device_error_word(), s)
+                     : gdr_host::fwd_tc_dispatch(q, k, v, g, beta, S0, out, S_final, B, T, H,
+                                                 cu_seqlens, nseq, gate, workspace,
+                                                 workspace_bytes, gdr_host::device_error_word(), s);
     } else {
         if ((size_t)gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL,
                                               false) > 227u * 1024u)
@@ -229,6 +246,15 @@ gdr_status gdr_fwd(const void *q, const void *k, const void *v, const float *g, 
         gdr_host::prof_end(tk, s);
     }
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+gdr_status gdr_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                   const float *S0, void *out, float *S_final, int B, int T, int H, int d_k,
+                   int d_v, int chunk, const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype,
+                   gdr_gate gate, gdr_path path, void *workspace, size_t workspace_bytes,
+                   void *stream) {
+    return fwd_common(q, k, v, g, beta, S0, out, S_final, B, T, H, d_k, d_v, chunk, cu_seqlens,
+                      n_seq, dtype, gate, path, workspace, workspace_bytes, stream, 1, nullptr);
 }
 
 gdr_status gdr_decode_step(const void *q, const void *k, const void *v, const float *g,
@@ -318,6 +344,20 @@ gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, con
 }
 
 }  // extern "C"
+
+namespace gdr_host {
+// Gated DeltaProduct over its virtual sequence (T = n_h x tokens rows per
+// sequence), writing only the last substep of each token into out; *ran is
+// false where the tensor-core path does not apply and nothing was launched.
+gdr_status fwd_keep(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    const float *S0, void *out, float *S_final, int B, int T, int H, int d_k,
+                    int d_v, int chunk, const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype,
+                    gdr_gate gate, gdr_path path, void *workspace, size_t workspace_bytes,
+                    void *stream, int keep, bool *ran) {
+    return fwd_common(q, k, v, g, beta, S0, out, S_final, B, T, H, d_k, d_v, chunk, cu_seqlens,
+                      n_seq, dtype, gate, path, workspace, workspace_bytes, stream, keep, ran);
+}
+}  // namespace gdr_host
 
 // ------------------------------------------------------------ error-path self test
 static __global__ void wait_timeout_kernel(unsigned int spin_limit, unsigned int *err) {

@@ -13,9 +13,18 @@
 //
 // With k, v laid out [B, T, n_h, H, d] and beta [B, T, n_h, H], the virtual
 // k~, v~, beta~ are the same memory viewed as [B, T n_h, H, d]; only q~ and g~
-// are materialised (expand kernel) and the kept outputs gathered (gather
-// kernel).  The chunkwise kernels themselves run unchanged.
+// are materialised (expand kernel).  On the tensor-core path the state pass
+// writes the kept outputs straight into out; the CUDA-core path writes every
+// virtual row and a gather kernel keeps every n_h-th.
 #include "common.cuh"
+
+namespace gdr_host {
+gdr_status fwd_keep(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    const float *S0, void *out, float *S_final, int B, int T, int H, int d_k,
+                    int d_v, int chunk, const int32_t *cu_seqlens, int n_seq, gdr_dtype dtype,
+                    gdr_gate gate, gdr_path path, void *workspace, size_t workspace_bytes,
+                    void *stream, int keep, bool *ran);
+}  // namespace gdr_host
 
 namespace gdr {
 
@@ -188,9 +197,15 @@ gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const fl
         gdp_scale_offsets_kernel<<<1, 256, 0, st>>>(cu_seqlens, cuv, n_seq, n_h);
         if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     }
-    gdr_status s = gdr_fwd(qv, k, v, gv, beta, S0, ov, S_final, B, (int)((long)T * n_h), H, d_k,
-                           d_v, chunk, cuv, n_seq, dtype, gate, path, ws + L.inner,
-                           workspace_bytes - L.inner, stream);
+    // the tensor-core path writes the kept rows itself; otherwise gather them
+    bool ran = false;
+    gdr_status s = gdr_host::fwd_keep(qv, k, v, gv, beta, S0, out, S_final, B,
+                                      (int)((long)T * n_h), H, d_k, d_v, chunk, cuv, n_seq, dtype,
+                                      gate, path, ws + L.inner, workspace_bytes - L.inner, stream,
+                                      n_h, &ran);
+    if (s != GDR_OK || ran) return s;
+    s = gdr_fwd(qv, k, v, gv, beta, S0, ov, S_final, B, (int)((long)T * n_h), H, d_k, d_v, chunk,
+                cuv, n_seq, dtype, gate, path, ws + L.inner, workspace_bytes - L.inner, stream);
     if (s != GDR_OK) return s;
     if (ntok > 0) {
         const unsigned grid = copy_grid(ntok);

@@ -49,8 +49,11 @@ def test_gdp_simt_fp32(cuda_device, gate, n_h):
 
 
 @pytest.mark.parametrize("gate", ["scalar", "channel"])
-@pytest.mark.parametrize("n_h", [2, 3])
+@pytest.mark.parametrize("n_h", [2, 3, 4, 8])
 def test_gdp_tc_bf16(cuda_device, gate, n_h):
+    """The tensor-core path writes the kept rows itself: staged and stored by
+    TMA when n_h divides the chunk (2 and 4 by fixed strides, 8 by the general
+    loop), plain stores otherwise (3) and on a sequence's last, partial chunk."""
     cfg = cfg_of(B=2, T=150, H=3, gate=gate, n_h=n_h,
                  gate_scale=0.1 if gate == "scalar" else 0.05)
     check(inputs.product_inputs(cfg, seed=502), cuda_device, "tc")
