@@ -221,6 +221,28 @@ def test_decode_full_size_sampled(cuda_device, name):
     assert worst <= 1e-2 and es <= 1e-2, (worst, es)
 
 
+@pytest.mark.parametrize("name", ["decode", "kda_decode"])
+def test_decode_full_size_every_head_first_steps(cuda_device, name):
+    """The decode workloads at full size for their first 10 steps with the
+    oracle following all 256 x 32 heads: every output of every step and the
+    whole final state."""
+    cfg = inputs.DECODE[name]
+    dev = cuda_device
+    S = inputs.decode_state(cfg)
+    Sd = torch.from_numpy(S).to(dev)
+    Sr = S.astype(np.float64)
+    worst = 0.0
+    for step in range(10):
+        tok = inputs.decode_token(cfg, step)
+        out = binding.gdr_decode_step(*(to_dev(x, "bf16", dev) for x in (tok.q, tok.k, tok.v)),
+                                      to_dev(tok.g, "f32", dev), to_dev(tok.beta, "f32", dev), Sd)
+        o_ref, Sr = oracle.recurrence_decode_step(tok.q, tok.k, tok.v, tok.g, tok.beta, Sr)
+        worst = max(worst, max_rel_fro(to_np(out), o_ref, (0, 1)))
+    assert binding.device_status() == binding.GDR_OK
+    es = state_rel(to_np(Sd), Sr)
+    assert worst <= 1e-2 and es <= 1e-2, (worst, es)
+
+
 # ------------------------------------------------------------------ error path
 def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
     assert binding.selftest_wait_timeout(4096) == binding.GDR_OK
