@@ -56,3 +56,24 @@ def test_single_rank_aggregation_is_local():
     import bench
     value, ms = bench.aggregate(1000, 4.0, 1)
     assert ms == 4.0 and abs(value - 250000.0) < 1e-9
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """`bench.py --impl reference --gpus 2` launched the way the multi-GPU runs
+    are (torchrun, one process per rank, gloo here): rank 0 alone times the
+    oracle and prints one JSON line, the other rank exits 0 without work."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--ref-budget-s", "2"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
