@@ -38,7 +38,7 @@ constexpr int kSimtRows = 32;  // state rows (d_v) per CTA
 
 struct SimtSmem {
     // offsets in floats
-    int Kc, Qc, Gc, Kx, bt, Nm, Am, Tm, Pm, Zm, Ss, total;
+    int Kc, Qc, Gc, Kx, bt, kd, Nm, Am, Tm, Pm, Zm, Ss, total;
     int kst;  // padded row stride of the [C][d_k] buffers
 };
 
@@ -51,6 +51,7 @@ __host__ __device__ inline SimtSmem simt_layout(int C, int dk, bool channel, boo
     L.Gc = o; o += channel ? C * L.kst : C;
     L.Kx = o; o += (channel || dec) ? C * L.kst : 0;  // K<- / E<-, then K->
     L.bt = o; o += C;
+    L.kd = o; o += C;  // scalar gate: e^(G_C - G_l) per row
     L.Nm = o; o += C * C;
     L.Am = o; o += C * C;
     L.Tm = o; o += C * C;
@@ -71,6 +72,7 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     extern __shared__ float sm[];
     const SimtSmem L = simt_layout(C, dk, CH, DEC);
     float *Kc = sm + L.Kc, *Qc = sm + L.Qc, *Gc = sm + L.Gc, *Kx = sm + L.Kx, *bt = sm + L.bt;
+    float *kd = sm + L.kd;
     float *Nm = sm + L.Nm, *Am = sm + L.Am, *Tm = sm + L.Tm, *Pm = sm + L.Pm, *Zm = sm + L.Zm;
     float *Ss = sm + L.Ss;
     const int kst = L.kst;
@@ -215,6 +217,8 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                 const int l = e / dk, c = e % dk;
                 Kx[l * kst + c] = Kc[l * kst + c] * expf(Gc[last * kst + c] - Gc[l * kst + c]);
             }
+        } else {  // the scalar gate's write factors, once per row
+            for (int l = tid; l < C; l += kSimtThreads) kd[l] = expf(Gc[last] - Gc[l]);
         }
         __syncthreads();
         // ---- S <- S Diag(exp(G_C)) + Z^T K-> ----
@@ -226,8 +230,7 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                 for (int l = 0; l < C; ++l) acc = fmaf(Zm[l * kSimtRows + r], Kx[l * kst + c], acc);
             } else {
                 acc = Ss[r * kst + c] * expf(Gc[last]);
-                for (int l = 0; l < C; ++l)
-                    acc = fmaf(Zm[l * kSimtRows + r] * expf(Gc[last] - Gc[l]), Kc[l * kst + c], acc);
+                for (int l = 0; l < C; ++l) acc = fmaf(Zm[l * kSimtRows + r] * kd[l], Kc[l * kst + c], acc);
             }
             Ss[r * kst + c] = acc;
         }
