@@ -106,6 +106,31 @@ def _need_contig(*ts):
             raise ValueError("tensors must be contiguous")
 
 
+def _check(device, *specs):
+    """The memory the kernels will read or write, checked before the call:
+    each ``(name, tensor, dtype, numel)`` (tensor None = absent) must live on
+    ``device``, have ``dtype`` (None: not checked) and hold at least ``numel``
+    elements.  A tensor on another device, of a narrower type or too small
+    would otherwise be addressed out of bounds by the kernels."""
+    for name, t, dtype, numel in specs:
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}; expected {device}")
+        if dtype is not None and t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if t.numel() < numel:
+            raise ValueError(f"{name} holds {t.numel()} elements; needs {numel}")
+
+
+def _on_cuda(q):
+    if not isinstance(q, torch.Tensor) or q.device.type != "cuda":
+        raise ValueError("tensors must be CUDA tensors")
+    return q.device
+
+
 def fwd_workspace_size(B, T, H, d_k, d_v, chunk, n_seq, varlen, dtype, gate, path="auto") -> int:
     return int(lib().gdr_fwd_workspace_size(B, T, H, d_k, d_v, chunk, n_seq, int(bool(varlen)),
                                             dtype, gate, PATHS[path]))
@@ -127,6 +152,11 @@ def gdr_fwd(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, out=
     gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
     n_seq = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
     _need_contig(q, k, v, g, beta, S0, cu_seqlens)
+    dev, th = _on_cuda(q), B * T * H
+    _check(dev, ("k", k, q.dtype, th * d_k), ("v", v, q.dtype, th * d_v),
+           ("g", g, torch.float32, th * (d_k if gate else 1)), ("beta", beta, torch.float32, th),
+           ("S0", S0, torch.float32, n_seq * H * d_v * d_k), ("cu_seqlens", cu_seqlens, torch.int32, 1),
+           ("out", out, q.dtype, th * d_v), ("S_final", S_final, torch.float32, n_seq * H * d_v * d_k))
     if out is None:
         out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
     if S_final is None and want_final:
@@ -156,6 +186,12 @@ def gdr_fwd_product(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=No
     gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
     n_seq = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
     _need_contig(q, k, v, g, beta, S0, cu_seqlens)
+    dev, th = _on_cuda(q), B * T * H
+    _check(dev, ("k", k, q.dtype, th * n_h * d_k), ("v", v, q.dtype, th * n_h * d_v),
+           ("g", g, torch.float32, th * (d_k if gate else 1)),
+           ("beta", beta, torch.float32, th * n_h),
+           ("S0", S0, torch.float32, n_seq * H * d_v * d_k), ("cu_seqlens", cu_seqlens, torch.int32, 1),
+           ("out", out, q.dtype, th * d_v), ("S_final", S_final, torch.float32, n_seq * H * d_v * d_k))
     if out is None:
         out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
     if S_final is None and want_final:
@@ -192,6 +228,12 @@ def gdr_fwd_gdn2(q, k, v, g, b, w, S0=None, *, chunk: int = 64, cu_seqlens=None,
     gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
     n_seq = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
     _need_contig(q, k, v, g, b, w, S0, cu_seqlens)
+    dev, th = _on_cuda(q), B * T * H
+    _check(dev, ("k", k, q.dtype, th * d_k), ("v", v, q.dtype, th * d_v),
+           ("g", g, torch.float32, th * (d_k if gate else 1)), ("b", b, torch.float32, th * d_k),
+           ("w", w, torch.float32, th * d_v),
+           ("S0", S0, torch.float32, n_seq * H * d_v * d_k), ("cu_seqlens", cu_seqlens, torch.int32, 1),
+           ("out", out, q.dtype, th * d_v), ("S_final", S_final, torch.float32, n_seq * H * d_v * d_k))
     if out is None:
         out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
     if S_final is None and want_final:
@@ -217,6 +259,11 @@ def gdr_decode_step_gdn2(q, k, v, g, b, w, S, *, out=None, stream=None) -> torch
     dtype = _dtype_code(q)
     gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 3 else GDR_GATE_SCALAR
     _need_contig(q, k, v, g, b, w, S)
+    dev, nh = _on_cuda(q), N * H
+    _check(dev, ("k", k, q.dtype, nh * d_k), ("v", v, q.dtype, nh * d_v),
+           ("g", g, torch.float32, nh * (d_k if gate else 1)), ("b", b, torch.float32, nh * d_k),
+           ("w", w, torch.float32, nh * d_v), ("S", S, torch.float32, nh * d_v * d_k),
+           ("out", out, q.dtype, nh * d_v))
     if out is None:
         out = torch.empty((N, H, d_v), dtype=q.dtype, device=q.device)
     st = lib().gdr_decode_step_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S),
@@ -240,6 +287,11 @@ def gdr_fwd_frame(q, k, v, g, gamma, n: int, S0=None, *, out=None, S_final=None,
     dtype = _dtype_code(q)
     gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
     _need_contig(q, k, v, g, gamma, S0)
+    dev, th, F = _on_cuda(q), B * T * H, (T + n - 1) // max(n, 1)
+    _check(dev, ("k", k, q.dtype, th * d_k), ("v", v, q.dtype, th * d_v),
+           ("g", g, torch.float32, B * F * H * (d_k if gate else 1)),
+           ("gamma", gamma, torch.float32, th), ("S0", S0, torch.float32, B * H * d_v * d_k),
+           ("out", out, q.dtype, th * d_v), ("S_final", S_final, torch.float32, B * H * d_v * d_k))
     if out is None:
         out = torch.empty((B, T, H, d_v), dtype=q.dtype, device=q.device)
     if S_final is None and want_final:
@@ -263,6 +315,10 @@ def gdr_decode_step(q, k, v, g, beta, S, *, out=None, stream=None) -> torch.Tens
     dtype = _dtype_code(q)
     gate = GDR_GATE_PER_KEY_CHANNEL if g.dim() == 3 else GDR_GATE_SCALAR
     _need_contig(q, k, v, g, beta, S)
+    dev, nh = _on_cuda(q), N * H
+    _check(dev, ("k", k, q.dtype, nh * d_k), ("v", v, q.dtype, nh * d_v),
+           ("g", g, torch.float32, nh * (d_k if gate else 1)), ("beta", beta, torch.float32, nh),
+           ("S", S, torch.float32, nh * d_v * d_k), ("out", out, q.dtype, nh * d_v))
     if out is None:
         out = torch.empty((N, H, d_v), dtype=q.dtype, device=q.device)
     st = lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),

@@ -156,8 +156,8 @@ def test_ncu_traffic_is_tied_to_the_sources(monkeypatch):
     """A recorded traffic figure is reported only while the kernel sources
     still hash to the digest it was taken on."""
     assert bench.ncu_traffic("tc_wy", "no_such_workload") is None
-    for key in bench.NCU_TRAFFIC:
-        assert bench.ncu_traffic(*key) is not None, key
+    for key, (_, _, val) in bench.NCU_TRAFFIC.items():
+        assert bench.ncu_traffic(*key) in (None, val), key  # current, or null once stale
     files, _, val = bench.NCU_TRAFFIC[("decode", "decode")]
     monkeypatch.setitem(bench.NCU_TRAFFIC, ("decode", "decode"), (files, "0" * 16, val))
     assert bench.ncu_traffic("decode", "decode") is None
@@ -177,3 +177,30 @@ def test_kernel_ids_match_the_header():
            for m in re.finditer(r"GDR_K_([A-Z0-9_]+)\s*=\s*(\d+)", hdr) if m.group(1) != "COUNT"}
     assert sorted(ids.values()) == sorted(binding.KERNELS.values())
     assert len(ids) == len(binding.KERNELS)
+
+
+def test_binding_rejects_host_tensors_before_any_launch():
+    """Host tensors never reach the library: their addresses would be device
+    faults in the kernels."""
+    q = torch.zeros(1, 4, 2, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.gdr_fwd(q, q, q, torch.zeros(1, 4, 2), torch.zeros(1, 4, 2))
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.gdr_decode_step(q[0], q[0], q[0], torch.zeros(4, 2), torch.zeros(4, 2),
+                                torch.zeros(4, 2, 16, 16))
+
+
+def test_binding_checks_device_dtype_and_size():
+    """The tensor checks the binding applies before a call (shown on the CPU
+    device): a narrower dtype, a too-small tensor or another device is refused."""
+    dev = torch.device("cpu")
+    ok = ("g", torch.zeros(6, dtype=torch.float32), torch.float32, 6)
+    binding._check(dev, ok, ("absent", None, torch.float32, 10))
+    with pytest.raises(TypeError):
+        binding._check(dev, ("g", torch.zeros(6, dtype=torch.bfloat16), torch.float32, 6))
+    with pytest.raises(ValueError, match="elements"):
+        binding._check(dev, ("beta", torch.zeros(5), torch.float32, 6))
+    with pytest.raises(ValueError, match="expected"):
+        binding._check(dev, ("S0", torch.zeros(6, device="meta"), torch.float32, 6))
+    with pytest.raises(TypeError):
+        binding._check(dev, ("k", [0.0] * 6, None, 6))
