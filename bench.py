@@ -480,6 +480,24 @@ def workload_config(name):
                "dtype_io": c.dtype, "steps_per_sequence": c.steps}
 
 
+L2_NOTE_FLUSHED = (f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then a "
+                   f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer, outside the per-step "
+                   "CUDA-event intervals)")
+L2_NOTE_DECODE = "no flush: the 512 MiB state is larger than L2 and is streamed every step"
+
+
+def full_config(name, path, world):
+    """The workload's config as both arms print it: its shapes plus the L2
+    treatment, the kernel path and the replica count."""
+    cfg, conf = workload_config(name)
+    is_decode = isinstance(cfg, inputs.DecodeConfig)
+    conf["l2"] = L2_NOTE_DECODE if is_decode else L2_NOTE_FLUSHED
+    if not is_decode and not isinstance(cfg, inputs.FrameConfig):
+        conf["path"] = path
+    conf["parallelism"] = f"replicas x{world}"
+    return cfg, conf
+
+
 class L2Flush:
     """Leaves L2 cold and clean between steps: writes one buffer larger than L2,
     then reads a second one, so the dirty lines of the write are written back
@@ -515,7 +533,7 @@ def run_reference(args, rank, world):
     """Reference arm: the fp64 CPU oracle, timed as it stands on the host cores."""
     if rank != 0:
         return
-    cfg, conf = workload_config(args.workload)
+    cfg, conf = full_config(args.workload, args.path, world)
     budget = max(0.5, args.ref_budget_s / max(1, args.steps + args.warmup))
     vals = []
     if isinstance(cfg, inputs.DecodeConfig):
@@ -551,7 +569,7 @@ def run_reference(args, rank, world):
 
 def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warmup,
             with_cpu, with_e2e, sampler=None):
-    cfg, conf = workload_config(name)
+    cfg, conf = full_config(name, path, world)
     seed = (inputs.BASE_SEED + cfg.seed_index) * 1000 + rank
     is_decode = isinstance(cfg, inputs.DecodeConfig)
     is_frame = isinstance(cfg, inputs.FrameConfig)
@@ -595,7 +613,6 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                 "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": ncu_traffic(dom, name),
                 "peak_source": peak_kind + " hbm_gbs", "algorithmic_bytes_per_launch": B_,
                 "frac_of_8TBps_spec": ach / 8000.0}
-        conf["l2"] = "no flush: the 512 MiB state is larger than L2 and is streamed every step"
     elif is_frame:
         # the dominant pass against its own roof: the token contractions (Gram,
         # output) run on the tensor cores for bf16 d = 128, the factorisation and
@@ -618,9 +635,6 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                 "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
                 "algorithmic_flops_per_launch": flops,
                 "step": {"tflops": frame_flops_per_token_head(dk, dv, cfg.n) * th / (ms * 1e-3) / 1e12}}
-        conf["l2"] = (f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then a "
-                      f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer, outside the "
-                      "per-step CUDA-event intervals)")
     else:
         th = cfg.B * cfg.T * cfg.H * cfg.n_h  # virtual steps when a token has substeps
         f_all = prefill_flops_per_token_head(cfg.chunk, cfg.d_k, cfg.d_v)
@@ -663,10 +677,13 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                         "hbm_gbs_min_bytes": min_bytes / (ms * 1e-3) / 1e9,
                         "hbm_frac": min_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                         "flops_per_step": f_all * th, "min_bytes_per_step": min_bytes}
-        conf["l2"] = (f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then a "
-                      f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer, outside the "
-                      "per-step CUDA-event intervals)")
-        conf["path"] = path
+        # the whole step against the bf16 tensor-core peak (the end-to-end
+        # fraction the prefill target is stated in), next to the dominant
+        # kernel's own fraction above
+        roof["frac_is"] = f"dominant kernel {dom}: {roof['bound']} roof of its algorithmic share"
+        roof["step_tc_frac"] = roof["step"]["tc_frac"]
+        roof["step_hbm_frac"] = roof["step"]["hbm_frac"]
+        roof["step_tflops"] = roof["step"]["tflops"]
     res = {"value": value, "ms_per_step": ms, "wall_s_incl_flush": wall, "roofline": roof,
            "kernels": kernels, "gpu_launches": launches, "clocks": clocks, "config": conf,
            "cfg": cfg, "run": run}
@@ -696,8 +713,9 @@ def main():
     ap.add_argument("--workload", default="gdn_prefill",
                     choices=list(inputs.PREFILL) + list(inputs.DECODE) + list(inputs.FRAME))
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
-    ap.add_argument("--extra", default=("decode,kda_decode,kda_prefill,varlen_prefill,gdp_prefill,"
-                                        "gdn2_prefill,frame_prefill,gdn_prefill_c16,gdn_prefill_c128"),
+    ap.add_argument("--extra", default=("kda_prefill,varlen_prefill,gdp_prefill,gdn2_prefill,"
+                                        "frame_prefill,gdn_prefill_c16,gdn_prefill_c128,decode,"
+                                        "kda_decode"),
                     help="comma-separated workloads measured after the main one ('' for none)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -730,9 +748,15 @@ def main():
             steps = 200 if name in inputs.DECODE else 20
             r = measure(args, name, device, rank, world, peaks, peak_kind, args.path, steps, 3,
                         False, False, None)
-            extra[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
-                           "steps": steps, "config": r["config"], "roofline": r["roofline"],
-                           "kernels": r["kernels"]}
+            # compact, so that the line's tail holds every extra workload
+            rf = r["roofline"]
+            extra[name] = {"ms_per_step": round(r["ms_per_step"], 5),
+                           "tokens_per_s": round(r["value"], 1), "steps": steps,
+                           "roofline": {"kernel": rf["kernel"], "bound": rf["bound"],
+                                        "frac": round(rf["frac"], 4),
+                                        **({"step_tc_frac": round(rf["step_tc_frac"], 4)}
+                                           if "step_tc_frac" in rf else {})},
+                           "kernel_ms": {k: round(v["avg_ms"], 5) for k, v in r["kernels"].items()}}
             del r
             torch.cuda.empty_cache()
         if rank == 0:
@@ -743,7 +767,7 @@ def main():
                     "scaling": "weak", "vs_baseline": None,
                     "dtype": "bf16" if getattr(cfg, "dtype", "bf16") == "bf16" else "f32",
                     "data": "synthetic (seeded; shapes and distributions of the workload)",
-                    "config": {**main_res["config"], "parallelism": f"replicas x{world}"},
+                    "config": main_res["config"],
                     "roofline": main_res["roofline"], "e2e": main_res.get("e2e"),
                     "gpu_launches": main_res["gpu_launches"], "clocks": main_res["clocks"],
                     "kernels": main_res["kernels"], "cpu_baseline": main_res.get("cpu_baseline"),

@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_profile_read.restype = i
         L.gdr_profile_read.argtypes = [i, ctypes.POINTER(ctypes.c_longlong),
                                        ctypes.POINTER(ctypes.c_double)]
+        L.gdr_set_gram_spread_limit.restype = ctypes.c_float
+        L.gdr_set_gram_spread_limit.argtypes = [ctypes.c_float]
         _lib = L
     return _lib
 
@@ -86,10 +88,24 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, device=None) -> ctypes.c_void_p:
+    """The cudaStream_t handle of ``stream`` (None: the current stream of
+    ``device``).  A torch stream must belong to ``device``: the library
+    launches on the current device, which the calls below set to it."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    sdev = getattr(stream, "device", None)
+    if device is not None and sdev is not None and torch.device(sdev) != torch.device(device):
+        raise ValueError(f"stream belongs to {sdev}; the tensors are on {device}")
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _call_on(device, fn):
+    """Run ``fn`` with ``device`` as the current CUDA device.  libgdr launches
+    on the current device (its tensor maps, error word and scratch lookup are
+    per device), so every call is made with the tensors' device current."""
+    with torch.cuda.device(device):
+        return fn()
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -166,9 +182,11 @@ def gdr_fwd(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, out=
     if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     ws_avail = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().gdr_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out),
-                       _ptr(S_final), B, T, H, d_k, d_v, chunk, _ptr(cu_seqlens), n_seq, dtype,
-                       gate, PATHS[path], _ptr(workspace), ws_avail, _stream(stream))
+    _check(dev, ("workspace", workspace, None, 0))
+    st = _call_on(dev, lambda: lib().gdr_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out), _ptr(S_final), B, T,
+        H, d_k, d_v, chunk, _ptr(cu_seqlens), n_seq, dtype, gate, PATHS[path], _ptr(workspace),
+        ws_avail, _stream(stream, dev)))
     if st != GDR_OK:
         raise GdrError(st, "gdr_fwd")
     return out, S_final
@@ -202,10 +220,11 @@ def gdr_fwd_product(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=No
     if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     ws_avail = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().gdr_fwd_product(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
-                               _ptr(out), _ptr(S_final), B, T, H, n_h, d_k, d_v, chunk,
-                               _ptr(cu_seqlens), n_seq, dtype, gate, PATHS[path],
-                               _ptr(workspace), ws_avail, _stream(stream))
+    _check(dev, ("workspace", workspace, None, 0))
+    st = _call_on(dev, lambda: lib().gdr_fwd_product(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out), _ptr(S_final), B, T,
+        H, n_h, d_k, d_v, chunk, _ptr(cu_seqlens), n_seq, dtype, gate, PATHS[path],
+        _ptr(workspace), ws_avail, _stream(stream, dev)))
     if st != GDR_OK:
         raise GdrError(st, "gdr_fwd_product")
     return out, S_final
@@ -243,10 +262,11 @@ def gdr_fwd_gdn2(q, k, v, g, b, w, S0=None, *, chunk: int = 64, cu_seqlens=None,
     if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     ws_avail = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().gdr_fwd_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
-                            _ptr(out), _ptr(S_final), B, T, H, d_k, d_v, chunk, _ptr(cu_seqlens),
-                            n_seq, dtype, gate, PATHS[path], _ptr(workspace), ws_avail,
-                            _stream(stream))
+    _check(dev, ("workspace", workspace, None, 0))
+    st = _call_on(dev, lambda: lib().gdr_fwd_gdn2(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(out), _ptr(S_final),
+        B, T, H, d_k, d_v, chunk, _ptr(cu_seqlens), n_seq, dtype, gate, PATHS[path],
+        _ptr(workspace), ws_avail, _stream(stream, dev)))
     if st != GDR_OK:
         raise GdrError(st, "gdr_fwd_gdn2")
     return out, S_final
@@ -266,8 +286,9 @@ def gdr_decode_step_gdn2(q, k, v, g, b, w, S, *, out=None, stream=None) -> torch
            ("out", out, q.dtype, nh * d_v))
     if out is None:
         out = torch.empty((N, H, d_v), dtype=q.dtype, device=q.device)
-    st = lib().gdr_decode_step_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S),
-                                    _ptr(out), N, H, d_k, d_v, dtype, gate, _stream(stream))
+    st = _call_on(dev, lambda: lib().gdr_decode_step_gdn2(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S), _ptr(out), N, H, d_k, d_v,
+        dtype, gate, _stream(stream, dev)))
     if st != GDR_OK:
         raise GdrError(st, "gdr_decode_step_gdn2")
     return out
@@ -300,9 +321,10 @@ def gdr_fwd_frame(q, k, v, g, gamma, n: int, S0=None, *, out=None, S_final=None,
     if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     ws_avail = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().gdr_fwd_frame(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma), _ptr(S0), _ptr(out),
-                             _ptr(S_final), B, T, H, d_k, d_v, n, dtype, gate, _ptr(workspace),
-                             ws_avail, _stream(stream))
+    _check(dev, ("workspace", workspace, None, 0))
+    st = _call_on(dev, lambda: lib().gdr_fwd_frame(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma), _ptr(S0), _ptr(out), _ptr(S_final), B, T,
+        H, d_k, d_v, n, dtype, gate, _ptr(workspace), ws_avail, _stream(stream, dev)))
     if st != GDR_OK:
         raise GdrError(st, "gdr_fwd_frame")
     return out, S_final
@@ -321,8 +343,9 @@ def gdr_decode_step(q, k, v, g, beta, S, *, out=None, stream=None) -> torch.Tens
            ("S", S, torch.float32, nh * d_v * d_k), ("out", out, q.dtype, nh * d_v))
     if out is None:
         out = torch.empty((N, H, d_v), dtype=q.dtype, device=q.device)
-    st = lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
-                               _ptr(out), N, H, d_k, d_v, dtype, gate, _stream(stream))
+    st = _call_on(dev, lambda: lib().gdr_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(out), N, H, d_k, d_v, dtype,
+        gate, _stream(stream, dev)))
     if st != GDR_OK:
         raise GdrError(st, "gdr_decode_step")
     return out
@@ -334,6 +357,12 @@ def device_status(stream=None) -> int:
 
 def selftest_wait_timeout(spin_limit: int, stream=None) -> int:
     return int(lib().gdr_selftest_wait_timeout(spin_limit, _stream(stream)))
+
+
+def set_gram_spread_limit(limit: float) -> float:
+    """Set the tensor-core prefill's Gram range limit (gdr.h,
+    gdr_set_gram_spread_limit); returns the previous one."""
+    return float(lib().gdr_set_gram_spread_limit(float(limit)))
 
 
 def profile_enable(on: bool = True) -> None:

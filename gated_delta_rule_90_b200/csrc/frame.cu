@@ -488,6 +488,7 @@ frame_gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     }
     // the last tile's MMAs cover all earlier ones
     if (ok && ntiles > 0) ok = mbar_wait_bounded(&done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, kSpinF, err);
+    ok = __syncthreads_and(ok);  // the TMEM loads below are warp-wide: decide for all threads
     tc_fence_after();
     if (ok) {
         const int qd = warp & 3, hf = warp >> 2, row = qd * 32 + lane;
@@ -576,6 +577,7 @@ frame_out_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mma_commit(&bar[1]);
     }
     ok = ok && mbar_wait_bounded(&bar[1], 0, kSpinF, err);
+    ok = __syncthreads_and(ok);  // the TMEM loads below are warp-wide: decide for all threads
     tc_fence_after();
     if (ok) {  // thread = token row
         const int r = warp * 32 + lane;

@@ -9,6 +9,8 @@
 //
 // The scratch is one file-scope device array of kNoAllocScratchBytes bytes.
 // Every device that loads this library holds it until the process exits.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace gdr_host {
@@ -30,23 +32,25 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of the scratch on the current device, looked up once per
 // device (the first gdr_fwd_noalloc call on that device does the lookup).
+// Host threads may race on a device's first call: each entry is atomic, and
+// two concurrent lookups store the same address.
 void *scratch_address(int *status) {
-    static void *addr[64] = {nullptr};
+    static std::atomic<void *> addr[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         *status = GDR_ERR_CUDA;
         return nullptr;
     }
-    if (!addr[dev]) {
-        void *p = nullptr;
+    void *p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
             *status = GDR_ERR_CUDA;
             return nullptr;
         }
-        addr[dev] = p;
+        addr[dev].store(p, std::memory_order_release);
     }
     *status = GDR_OK;
-    return addr[dev];
+    return p;
 }
 
 bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }

@@ -28,8 +28,11 @@
 // Per-channel gates (KDA) enter the Gram GEMM factorised around the middle
 // row r = 31 of the chunk: (k_l . e^(G_l - G_r)) . (k_m . e^(G_r - G_m)), so
 // every factor stays within e^(|G_l - G_r|) of 1 -- never a ratio of products.
-// This needs |G_l - G_r| < ~80 per channel inside a chunk (bf16/fp32 range);
-// the SIMT path has no such limit.
+// That needs |G_l - G_r| well inside the fp32/bf16 exponent range.  A chunk in
+// which some channel's spread max_l |G_l - G_r| reaches the limit (60 by
+// default) takes the exact route instead: L and A are summed on the CUDA cores
+// with e^(G_lc - G_mc) exponentiated per element (never above 1 for a decay),
+// and Q<-, K->, K<- use e^(G), e^(G_C - G) directly.
 //
 // Tokens of a chunk that runs past the end of its sequence are zeroed in
 // shared memory (k = q = v = 0, beta = 0, g = 0), which leaves every valid row
@@ -38,6 +41,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <string.h>
+
+#include <atomic>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -63,6 +68,10 @@ struct Geo {
     // substeps per token; out has one row per token and receives the last
     // substep's output only
     int keep;
+    // largest within-chunk |G_l - G_31| (cumulative log-decay, any channel)
+    // for which the Gram weights e^(G_l - G_m) are taken as the product of two
+    // per-row factors; a chunk beyond it exponentiates every difference
+    float spread_limit;
 };
 
 struct Ws {
@@ -137,6 +146,32 @@ __global__ void plan_kernel(const int32_t *cu, int n_seq, int T_total, int *chun
         }
         order[rank] = s;
     }
+}
+
+// Sums each of v[0..7] over the 32 lanes of a warp in 9 shuffles (each step
+// halves the values a lane keeps); lane L returns the total of v[(L >> 2) & 7].
+__device__ __forceinline__ float warp_sum8(const float (&v)[8], int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float w[4], x[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = (b4 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, b4 ? v[i] : v[i + 4], 16);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        x[i] = (b3 ? w[i + 2] : w[i]) + __shfl_xor_sync(0xffffffffu, b3 ? w[i] : w[i + 2], 8);
+    float y = (b2 ? x[1] : x[0]) + __shfl_xor_sync(0xffffffffu, b2 ? x[0] : x[1], 4);
+    y += __shfl_xor_sync(0xffffffffu, y, 1);
+    y += __shfl_xor_sync(0xffffffffu, y, 2);
+    return y;
+}
+// Four consecutive bf16 of a 128-byte-swizzled [rows][64] atom: row r,
+// columns 4 q .. 4 q + 3 (q = 0..15).
+__device__ __forceinline__ void ld4_sw128(const uint8_t *atom, int r, int q, float *f) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(atom + r * 128 + (((q >> 1) ^ (r & 7)) << 4) +
+                                                     (q & 1) * 8);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
 }
 
 // ------------------------------------------------------------------ WY kernel
@@ -256,6 +291,8 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
+    // per-channel gate: this chunk takes the exact route (see the file header)
+    int fb = 0;
     if (!CH && warp == 0) {
         float a = sG[lane], b = sG[lane + 32];
 #pragma unroll
@@ -283,7 +320,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         eA[lane + 32] = __expf(b - R);
         eB[lane] = __expf(R - a);
         eB[lane + 32] = __expf(R - b);
-        if (lane == 0) *sFact = spread < 60.f;
+        if (lane == 0) *sFact = spread < geo.spread_limit;
     }
     {
         const bool ok_ld = mbar_wait_bounded(&bars[0], 0, kSpin, err);
@@ -298,17 +335,25 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         for (int i = 0; i < 32; ++i) v[i] = (r0 + i < len) ? sGt[(r0 + i) * D + c] : 0.f;
 #pragma unroll
         for (int i = 1; i < 32; ++i) v[i] += v[i - 1];
+        // spread = max_l |G_l - R| of this channel (R = G_31)
+        float spread = 0.f;
         if (!r0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sGt[i * D + c] = v[i];
+            for (int i = 0; i < 32; ++i) {
+                sGt[i * D + c] = v[i];
+                spread = fmaxf(spread, fabsf(v[i] - v[31]));
+            }
         }
         __syncthreads();
         if (r0) {
             const float base = sGt[31 * D + c];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sGt[(32 + i) * D + c] = v[i] + base;
+            for (int i = 0; i < 32; ++i) {
+                sGt[(32 + i) * D + c] = v[i] + base;
+                spread = fmaxf(spread, fabsf(v[i]));
+            }
         }
-        __syncthreads();
+        fb = __syncthreads_or(!(spread < geo.spread_limit));
         if (tid < D) {
             const float R = sGt[31 * D + tid], GC = sGt[(C - 1) * D + tid];
             sG[tid] = R;    // reference row R of the Gram factorisation
@@ -360,19 +405,29 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                         for (int i = 0; i < 8; ++i) b8[i] = 0.f;
                     }
                 }
+                if (fb) {  // exact route: e^G and e^(G_C - G) themselves (at most 1)
+                    float GC8[8];
+                    ld8(sGC + c0, GC8);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    // e^G = e^(G - R) e^R and e^(G_C - G) = e^(R - G) e^(G_C - R)
-                    const float e1 = __expf(G8[i] - R8[i]), e2 = __expf(R8[i] - G8[i]);
-                    wq[i] = qv[i] * (e1 * eR8[i]);
-                    wk[i] = kv[i] * (e2 * eCR8[i]);
-                    kh[i] = (DEC ? kv[i] * b8[i] : kv[i]) * e1;
-                    qh[i] = qv[i] * e1;
-                    kc[i] = kv[i] * e2;
+                    for (int i = 0; i < 8; ++i) {
+                        wq[i] = qv[i] * __expf(G8[i]);
+                        wk[i] = kv[i] * __expf(GC8[i] - G8[i]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        // e^G = e^(G - R) e^R and e^(G_C - G) = e^(R - G) e^(G_C - R)
+                        const float e1 = __expf(G8[i] - R8[i]), e2 = __expf(R8[i] - G8[i]);
+                        wq[i] = qv[i] * (e1 * eR8[i]);
+                        wk[i] = kv[i] * (e2 * eCR8[i]);
+                        kh[i] = (DEC ? kv[i] * b8[i] : kv[i]) * e1;
+                        qh[i] = qv[i] * e1;
+                        kc[i] = kv[i] * e2;
+                    }
+                    *reinterpret_cast<uint4 *>(sKQ + off) = pack8(kh);
+                    *reinterpret_cast<uint4 *>(sKQ + off + 8192) = pack8(qh);
+                    kcv[k] = pack8(kc);
                 }
-                *reinterpret_cast<uint4 *>(sKQ + off) = pack8(kh);
-                *reinterpret_cast<uint4 *>(sKQ + off + 8192) = pack8(qh);
-                kcv[k] = pack8(kc);
             } else {
                 const float eq = __expf(sG[l]), ek = __expf(sG[C - 1] - sG[l]);
 #pragma unroll
@@ -384,8 +439,10 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             *reinterpret_cast<uint4 *>(Qg + l * D + c0) = pack8(wq);
             *reinterpret_cast<uint4 *>(Kg + l * D + c0) = pack8(wk);
         }
-        if (tid < D) ws.dec[slot * D + tid] = CH ? eCR[tid] * eR[tid] : __expf(sG[C - 1]);
-        if (CH) {  // the gate tile is read: K-check takes its first half
+        if (tid < D)
+            ws.dec[slot * D + tid] = CH ? (fb ? __expf(sGC[tid]) : eCR[tid] * eR[tid])
+                                        : __expf(sG[C - 1]);
+        if (CH && !fb) {  // the gate tile is read: K-check takes its first half
             __syncthreads();
 #pragma unroll
             for (int k = 0; k < C / 16; ++k) {
@@ -398,74 +455,161 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     tc_fence_before();
     __syncthreads();
 
-    // Gram: TMEM[0:64) = [K;Q] (128 x 128) * Kc^T (64 x 128)^T
-    if (tid == 0) {
-        tc_fence_after();
-        const uint8_t *Bb = CH ? sKC : sKQ;
-        const uint32_t bstride = CH ? 8192 : 16384;
-        const uint32_t id = idesc_bf16(128, 64, 0, 0);
-        const uint64_t ad = sdesc_sw128(smem_u32(sKQ), 16, 1024);
-        const uint64_t bd = sdesc_sw128(smem_u32(Bb), 16, 1024);
+    if (!fb) {
+        // Gram: TMEM[0:64) = [K;Q] (128 x 128) * Kc^T (64 x 128)^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint8_t *Bb = CH ? sKC : sKQ;
+            const uint32_t bstride = CH ? 8192 : 16384;
+            const uint32_t id = idesc_bf16(128, 64, 0, 0);
+            const uint64_t ad = sdesc_sw128(smem_u32(sKQ), 16, 1024);
+            const uint64_t bd = sdesc_sw128(smem_u32(Bb), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (kk & 3) * 32;
-            mma_bf16_ss(tmem, sdesc_add(ad, (kk >> 2) * 16384 + koff),
-                        sdesc_add(bd, (kk >> 2) * bstride + koff), id, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t koff = (kk & 3) * 32;
+                mma_bf16_ss(tmem, sdesc_add(ad, (kk >> 2) * 16384 + koff),
+                            sdesc_add(bd, (kk >> 2) * bstride + koff), id, kk > 0);
+            }
+            mma_commit(&bars[1]);
         }
-        mma_commit(&bars[1]);
-    }
-    {
-        const bool ok = mbar_wait_bounded(&bars[1], 0, kSpin, err);
-        if (!__syncthreads_and(ok)) goto cleanup;
-    }
-    tc_fence_after();
-    {
-        // accumulator rows 0..63: K K^T -> N = diag(beta) tril_-1(. Gamma), stored
-        // transposed; rows 64..127: Q K^T -> A = tril_0(. Gamma), bf16, staged in TT
-        const int l = (qd & 1) * 32 + lane, m0 = hf * 32;
-        float gr[32];
-        tmem_ld16(tmem + lb + m0, gr);
-        tmem_ld16(tmem + lb + m0 + 16, gr + 16);
-        tmem_wait_ld();
-        // gam(m) = Gamma[l][m] (scalar gate; the per-channel gate is inside the operands)
-        auto epilogue = [&](auto gam) {
-            if (qd < 2) {
-                const float bl = sB[l];
+        {
+            const bool ok = mbar_wait_bounded(&bars[1], 0, kSpin, err);
+            if (!__syncthreads_and(ok)) goto cleanup;
+        }
+        tc_fence_after();
+        {
+            // accumulator rows 0..63: K K^T -> N = diag(beta) tril_-1(. Gamma), stored
+            // transposed; rows 64..127: Q K^T -> A = tril_0(. Gamma), bf16, staged in TT
+            const int l = (qd & 1) * 32 + lane, m0 = hf * 32;
+            float gr[32];
+            tmem_ld16(tmem + lb + m0, gr);
+            tmem_ld16(tmem + lb + m0 + 16, gr + 16);
+            tmem_wait_ld();
+            // gam(m) = Gamma[l][m] (scalar gate; the per-channel gate is inside the operands)
+            auto epilogue = [&](auto gam) {
+                if (qd < 2) {
+                    const float bl = sB[l];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int m = m0 + i;
-                    sN[m * NTS + l] = (m < l) ? bl * gr[i] * gam(m) : 0.f;
-                }
-            } else {
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    float o[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int m = m0 + jj * 8 + i;
-                        o[i] = (m <= l) ? gr[jj * 8 + i] * gam(m) : 0.f;
+                    for (int i = 0; i < 32; ++i) {
+                        const int m = m0 + i;
+                        sN[m * NTS + l] = (m < l) ? bl * gr[i] * gam(m) : 0.f;
                     }
-                    const int j = hf * 4 + jj;
-                    *reinterpret_cast<uint4 *>(sT + l * 128 + ((j ^ (l & 7)) << 4)) = pack8(o);
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        float o[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int m = m0 + jj * 8 + i;
+                            o[i] = (m <= l) ? gr[jj * 8 + i] * gam(m) : 0.f;
+                        }
+                        const int j = hf * 4 + jj;
+                        *reinterpret_cast<uint4 *>(sT + l * 128 + ((j ^ (l & 7)) << 4)) = pack8(o);
+                    }
+                }
+            };
+            if (CH) {
+                epilogue([](int) { return 1.f; });
+            } else if (*sFact) {
+                const float eAl = eA[l];
+                epilogue([&](int m) { return eAl * eB[m]; });
+            } else {
+                const float Gl = sG[l];
+                epilogue([&](int m) { return __expf(Gl - sG[m]); });
+            }
+        }
+    } else {
+        // Exact route (per-channel gate, a chunk beyond the spread limit): L and
+        // A on the CUDA cores with every weight e^(G_lc - G_mc) exponentiated.
+        // A warp takes (row l, columns m0..m0+3) at a time, its lanes four
+        // channels each; beta L goes to the W tile of the workspace (fp32,
+        // N^T order) until the gate tile is dead, A straight to its workspace
+        // tile.
+        float *Nsc = reinterpret_cast<float *>(ws.W + slot * (C * D));
+        __nv_bfloat16 *Ag = ws.A + slot * (C * C);
+        for (int e = tid; e < C * C; e += kWyThreads)
+            if (e % C > e / C) Ag[e] = __float2bfloat16_rn(0.f);
+        const int qa = lane >> 4, qc = lane & 15;  // atom, 4-channel group
+        int gi = 0;
+        for (int l = 0; l < C; ++l) {
+            for (int m0 = 0; m0 <= l; m0 += 4, ++gi) {
+                if ((gi & 7) != warp) continue;
+                const float4 gl = *reinterpret_cast<const float4 *>(sGt + l * D + 4 * lane);
+                float el[4], ql[4], acc[8];
+                ld4_sw128(sKQ + qa * 16384, l, qc, el);
+                ld4_sw128(sKQ + qa * 16384 + 8192, l, qc, ql);
+                if (DEC) {  // reading row e = b . k (zero beyond the sequence end)
+                    const float4 bb = (l < len)
+                        ? *reinterpret_cast<const float4 *>(
+                              eg + ((size_t)(tstart + l) * geo.H + h) * D + 4 * lane)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    el[0] *= bb.x; el[1] *= bb.y; el[2] *= bb.z; el[3] *= bb.w;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int m = min(m0 + u, C - 1);  // m > l: computed, never stored
+                    const float4 gm = *reinterpret_cast<const float4 *>(sGt + m * D + 4 * lane);
+                    float km[4];
+                    ld4_sw128(sKQ + qa * 16384, m, qc, km);
+                    const float w0 = __expf(gl.x - gm.x) * km[0], w1 = __expf(gl.y - gm.y) * km[1];
+                    const float w2 = __expf(gl.z - gm.z) * km[2], w3 = __expf(gl.w - gm.w) * km[3];
+                    acc[u] = el[0] * w0 + el[1] * w1 + el[2] * w2 + el[3] * w3;
+                    acc[4 + u] = ql[0] * w0 + ql[1] * w1 + ql[2] * w2 + ql[3] * w3;
+                }
+                const float tot = warp_sum8(acc, lane);
+                if ((lane & 3) == 0) {
+                    const int vi = lane >> 2;
+                    if (vi < 4) {
+                        const int m = m0 + vi;
+                        if (m < l) Nsc[m * C + l] = sB[l] * tot;
+                    } else {
+                        const int m = m0 + vi - 4;
+                        if (m <= l) Ag[l * C + m] = __float2bfloat16_rn(tot);
+                    }
                 }
             }
-        };
-        if (CH) {
-            epilogue([](int) { return 1.f; });
-        } else if (*sFact) {
-            const float eAl = eA[l];
-            epilogue([&](int m) { return eAl * eB[m]; });
-        } else {
-            const float Gl = sG[l];
-            epilogue([&](int m) { return __expf(Gl - sG[m]); });
+        }
+        __syncthreads();
+        // K<- = e^G . k (. b) over the raw K rows, while the gate tile lives
+        {
+            const int cg = tid & 15, c0 = cg * 8, a = cg >> 3, l0 = tid >> 4;
+#pragma unroll
+            for (int k = 0; k < C / 16; ++k) {
+                const int l = l0 + 16 * k, j = (cg & 7) ^ (l & 7);
+                const uint32_t off = a * 16384 + l * 128 + j * 16;
+                float kv[8], G8[8], o[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sKQ + off), kv);
+                ld8(sGt + l * D + c0, G8);
+                if (DEC) {
+                    float b8[8];
+                    if (l < len) {
+                        ld8(eg + ((size_t)(tstart + l) * geo.H + h) * D + c0, b8);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) b8[i] = 0.f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) kv[i] *= b8[i];
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[i] = kv[i] * __expf(G8[i]);
+                *reinterpret_cast<uint4 *>(sKQ + off) = pack8(o);
+            }
+        }
+        __syncthreads();  // the gate tile is dead: N^T into its place
+        for (int e = tid; e < C * C; e += kWyThreads) {
+            const int m = e / C, l = e % C;
+            sN[m * NTS + l] = (m < l) ? Nsc[e] : 0.f;
         }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == kWyTmaThread) {  // A -> workspace
-        tma_store_2d(&tm_Ast, sT, 0, (int)(slot * C));
-        bulk_commit_group();
+    if (tid == kWyTmaThread) {  // A -> workspace (the exact route stored it already)
+        if (!fb) {
+            tma_store_2d(&tm_Ast, sT, 0, (int)(slot * C));
+            bulk_commit_group();
+        }
         // Q is read: V takes its place (lands during the solve)
         mbar_arrive_expect_tx(&bars[0], 2 * kHalfBytes);
         tma_load_2d(sV, &tm_v, &bars[0], x0, ytok);
@@ -582,7 +726,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             *reinterpret_cast<uint4 *>(sT + i * 128 + ((j8 ^ (i & 7)) << 4)) = pack8(o);
         }
         // K<- into the dead N^T area: scalar gate e^G . k from raw K, per-channel
-        // gate K^ . e^R
+        // gate K^ . e^R (exact route: K<- is already in place)
         {
             const int cg = tid & 15, c0 = cg * 8, a = cg >> 3, l0 = tid >> 4;
             float eR8[8];
@@ -594,7 +738,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 unpack8(*reinterpret_cast<const uint4 *>(sKQ + a * 16384 + l * 128 + jj * 16), kv);
                 const float el = CH ? 0.f : __expf(sG[l]);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = kv[i] * (CH ? eR8[i] : el);
+                for (int i = 0; i < 8; ++i) o[i] = kv[i] * (CH ? (fb ? 1.f : eR8[i]) : el);
                 *reinterpret_cast<uint4 *>(sKL + a * 8192 + l * 128 + jj * 16) = pack8(o);
             }
         }
@@ -640,7 +784,8 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         mma_commit(&bars[1]);
     }
     {
-        const bool ok = mbar_wait_bounded(&bars[1], 1, kSpin, err);
+        // the second commit on this barrier, or the first on the exact route
+        const bool ok = mbar_wait_bounded(&bars[1], fb ? 0 : 1, kSpin, err);
         if (!__syncthreads_and(ok)) goto cleanup;  // V and K<- are no longer read
     }
     tc_fence_after();
@@ -715,6 +860,20 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 }
 __device__ __forceinline__ void named_arrive(int id, int n) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Named barrier that also ANDs a predicate over its n threads, so that a
+// decision taken after a bounded wait is the same in every thread of a role.
+__device__ __forceinline__ bool named_sync_and(int id, int n, bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)p), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
 }
 // Chain -> MMA-warp hand-offs on hardware named barriers (the chain warps
 // arrive, the MMA warp syncs).  Both sides pass each barrier exactly twice per
@@ -825,6 +984,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             const uint8_t *st = sm + (r & 1) * StSmem::STAGE;
             if (ok) ok = mbar_wait_bounded(&full[r & 1], (r >> 1) & 1, kSpin, err);
             if (ok && r > 0) ok = mbar_wait_bounded(barS, (r - 1) & 1, kSpin, err);
+            ok = __all_sync(0xffffffffu, ok);  // the TMEM accesses below are warp-wide
             float v[64];
             if (ok) {  // S (fp32) -> bf16 operand in TMEM
                 tc_fence_after();
@@ -857,6 +1017,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
                 tmem_wait_st();
             }
             if (ok) ok = mbar_wait_bounded(barZ, r & 1, kSpin, err);
+            ok = __all_sync(0xffffffffu, ok);
             if (ok) {  // Z^T = U^T - S W<-^T -> bf16 A operand in TMEM (this thread: 32 tokens)
                 tc_fence_after();
                 float z[32];
@@ -886,6 +1047,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             named_arrive(kBarOpsZ, kOpsThreads);
         }
         if (ok && nch > 0) ok = mbar_wait_bounded(barS, (nch - 1) & 1, kSpin, err);
+        ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         if (ok && S_final) {
 #pragma unroll
@@ -906,8 +1068,11 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
         const int otid = tid - kChainThreads;
         const uint32_t lb = (uint32_t)(qd * 32) << 16;
         __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(sm + StSmem::OST);
-        for (int r = 0; r < nch && ok; ++r) {
-            ok = mbar_wait_bounded(&barO[r & 1], (r >> 1) & 1, kSpin, err);
+        for (int r = 0; r < nch; ++r) {
+            // every output thread goes on, or all stop: the named barriers
+            // below need all of them
+            ok = named_sync_and(1, kOutThreads,
+                                mbar_wait_bounded(&barO[r & 1], (r >> 1) & 1, kSpin, err));
             if (!ok) break;
             tc_fence_after();
             float o[64];
@@ -1076,6 +1241,10 @@ WsLayout ws_layout(int B, int T, int H, int n_seq, int varlen) {
 
 using namespace gdr_host::tmap;
 
+// Spread limit of the factorised Gram weights (Geo::spread_limit).
+std::atomic<float> g_spread_limit{60.f};
+constexpr float kSpreadLimitMax = 80.f;  // e^80 and e^-80 stay normal fp32 / bf16
+
 size_t wy_smem_bytes(bool ch) {  // + 1024 for the in-kernel alignment
     return 1024 + WySmem::small(ch) + WySmem::small_bytes(ch);
 }
@@ -1115,6 +1284,7 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
     geo.B = B; geo.T = T; geo.H = H; geo.n_seq = varlen ? n_seq : B;
     geo.nc = (T + C - 1) / C; geo.varlen = varlen; geo.T_total = B * T; geo.n_slots = L.n_slots;
     geo.keep = keep;
+    geo.spread_limit = g_spread_limit.load(std::memory_order_relaxed);
 
     const size_t tiles = (size_t)L.n_slots * H;
     if (tiles * D >= ((size_t)1 << 31)) return cudaErrorInvalidValue;  // 32-bit TMA rows
@@ -1214,3 +1384,12 @@ cudaError_t fwd_tc_gdn2_dispatch(const void *q, const void *k, const void *v, co
 }
 
 }  // namespace gdr_host
+
+extern "C" float gdr_set_gram_spread_limit(float limit) {
+    float prev = g_spread_limit.load();
+    if (limit == limit) {  // NaN leaves the limit as it is
+        limit = limit < 0.f ? 0.f : (limit > kSpreadLimitMax ? kSpreadLimitMax : limit);
+        prev = g_spread_limit.exchange(limit);
+    }
+    return prev;
+}

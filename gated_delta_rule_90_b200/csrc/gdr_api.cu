@@ -51,16 +51,20 @@ cudaError_t fwd_tc_keep_dispatch(const void *q, const void *k, const void *v, co
 static __device__ unsigned int g_gdr_device_error;
 
 namespace gdr_host {
+// Cached per device; entries are atomic because host threads may make their
+// first call on a device at the same time (both store the same address).
 unsigned int *device_error_word() {
-    static unsigned int *cache[64] = {nullptr};
+    static std::atomic<unsigned int *> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!cache[dev]) {
+    unsigned int *w = cache[dev].load(std::memory_order_acquire);
+    if (!w) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_gdr_device_error) != cudaSuccess) return nullptr;
-        cache[dev] = (unsigned int *)p;
+        w = (unsigned int *)p;
+        cache[dev].store(w, std::memory_order_release);
     }
-    return cache[dev];
+    return w;
 }
 }  // namespace gdr_host
 

@@ -275,6 +275,23 @@ gdr_status gdr_fwd_noalloc(const void *q, const void *k, const void *v, const fl
 size_t gdr_fwd_noalloc_scratch_bytes(void);
 
 /*
+ * Range control of the tensor-core prefill's Gram weights.  Inside a chunk the
+ * weights e^(G_l - G_m) of L and A (G = cumulative log-decay from the chunk
+ * start; "Linear Attention, Visualized", sections "Gated DeltaNet (GDN) /
+ * Complete per-chunk algorithm" and "Kimi Delta Attention (KDA) / Complete
+ * per-chunk algorithm") are taken as e^(G_l - G_r) e^(G_r - G_m) around the
+ * chunk's row r = 31, which keeps the Gram on the tensor cores.  A chunk in
+ * which max_l |G_l - G_r| (any channel) reaches `limit` exponentiates every
+ * difference instead (scalar gate: in the Gram epilogue; per-channel gate: L
+ * and A summed on the CUDA cores); both give the same result up to rounding.
+ * The default is 60; `limit` is clamped into [0, 80] (beyond 80 the factors
+ * leave the normal fp32 / bf16 range) and 0 sends every chunk the exact way.
+ * NaN leaves the setting unchanged.  Returns the previous limit.  Process-wide;
+ * applies to calls made after it returns.
+ */
+float gdr_set_gram_spread_limit(float limit);
+
+/*
  * Per-kernel launch accounting and timing (a small built-in profiler).
  * Kernel ids: GDR_K_DECODE, GDR_K_FWD_SIMT, GDR_K_TC_PLAN, GDR_K_TC_WY,
  * GDR_K_TC_STATE, GDR_K_GDP_REMAP (the Gated DeltaProduct expand/gather),

@@ -189,3 +189,16 @@ def test_frame_workspace_size():
     F = -(-T // n)
     assert binding.fwd_frame_workspace_size(B, T, H, d, d, n) >= 3 * B * F * H * d * d * 4
     assert binding.fwd_frame_workspace_size(B, T, H, 12, d, n) == 0
+
+
+def test_gram_spread_limit_is_clamped_and_restored():
+    """gdr_set_gram_spread_limit returns the previous limit, clamps into
+    [0, 80] and ignores NaN (host state only; no launch)."""
+    prev = binding.set_gram_spread_limit(60.0)
+    try:
+        assert binding.set_gram_spread_limit(1000.0) == 60.0
+        assert binding.set_gram_spread_limit(-5.0) == 80.0
+        assert binding.set_gram_spread_limit(float("nan")) == 0.0
+        assert binding.set_gram_spread_limit(60.0) == 0.0
+    finally:
+        binding.set_gram_spread_limit(prev)

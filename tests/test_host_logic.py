@@ -204,3 +204,46 @@ def test_binding_checks_device_dtype_and_size():
         binding._check(dev, ("S0", torch.zeros(6, device="meta"), torch.float32, 6))
     with pytest.raises(TypeError):
         binding._check(dev, ("k", [0.0] * 6, None, 6))
+
+
+# ------------------------------------------------------------------ binding device rules
+def test_binding_calls_run_with_the_tensors_device_current(monkeypatch):
+    """libgdr launches on the current CUDA device, so the binding makes the
+    tensors' device current around every call (a mocked device guard records
+    which device it was given)."""
+    import contextlib
+
+    from gated_delta_rule_90_b200 import binding
+
+    seen = []
+
+    @contextlib.contextmanager
+    def fake_device(d):
+        seen.append(torch.device(d))
+        yield
+
+    monkeypatch.setattr(binding.torch.cuda, "device", fake_device)
+    assert binding._call_on(torch.device("cuda", 3), lambda: 17) == 17
+    assert seen == [torch.device("cuda", 3)]
+
+
+def test_binding_rejects_a_stream_of_another_device():
+    from gated_delta_rule_90_b200 import binding
+
+    class FakeStream:
+        device = torch.device("cuda", 1)
+        cuda_stream = 1234
+
+    with pytest.raises(ValueError):
+        binding._stream(FakeStream(), torch.device("cuda", 0))
+    assert binding._stream(FakeStream(), torch.device("cuda", 1)).value == 1234
+    assert binding._stream(5678, torch.device("cuda", 0)).value == 5678  # raw handle: unchecked
+
+
+def test_binding_rejects_a_workspace_on_another_device():
+    from gated_delta_rule_90_b200 import binding
+
+    ws = torch.empty(16, dtype=torch.uint8)  # host memory
+    with pytest.raises(ValueError):
+        binding._check(torch.device("cuda", 0), ("workspace", ws, None, 0))
+    binding._check(torch.device("cpu"), ("workspace", ws, None, 0))
