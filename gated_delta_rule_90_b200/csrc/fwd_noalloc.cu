@@ -19,7 +19,8 @@ size_t tc_workspace_bytes(int B, int T, int H, int n_seq, int varlen, gdr_gate g
 cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const float *S0, void *out, float *S_final, int B,
                             int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
-                            void *workspace, size_t ws_bytes, unsigned int *err, cudaStream_t st);
+                            void *workspace, size_t ws_bytes, unsigned int *err, cudaStream_t st,
+                            int chunk);
 }  // namespace gdr_host
 
 namespace {
@@ -87,7 +88,7 @@ gdr_status gdr_fwd_noalloc(const void *q, const void *k, const void *v, const fl
     cudaError_t e = gdr_host::fwd_tc_dispatch(q, k, v, g, beta, S0, out, S_final, B, T, H,
                                               cu_seqlens, varlen ? n_seq : B, gate, scratch,
                                               kNoAllocScratchBytes, gdr_host::device_error_word(),
-                                              (cudaStream_t)stream);
+                                              (cudaStream_t)stream, 64);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -209,6 +209,10 @@ struct WySmem {
     static constexpr uint32_t small_bytes(bool ch) { return small_floats(ch) * 4 + 64; }
 };
 
+// SUB (scalar gate): the chunk size of the method, 64 or 16.  With 16 a
+// 64-token tile holds four chunks: G restarts every 16 rows, L, A and T are
+// block diagonal (the 16 x 16 diagonal blocks of the 64 x 64 solve), K->
+// decays to each chunk's own end, and four decay rows are written.
 // DEC (per-channel decay only): Gated DeltaNet-2's erase gate b and write gate
 // w replace beta ("Gated DeltaNet-2, and the gate that was doing two jobs",
 // section "What decoupling actually means here"): the Gram's reading rows are
@@ -216,7 +220,7 @@ struct WySmem {
 // (I + L) T = I, and U = T (w . V).  The writing direction stays k (K->, A).
 // BC (with CH): the decay is one scalar per token, broadcast over the key
 // channels of the gate tile in shared memory instead of loaded per channel.
-template <bool CH, bool DEC = false, bool BC = false>
+template <bool CH, bool DEC = false, bool BC = false, int SUB = C>
 __global__ void __launch_bounds__(kWyThreads, CH ? 3 : 0)
 wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -226,6 +230,10 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           const float *__restrict__ wg, const int32_t *__restrict__ cu, Geo geo, Ws ws,
           unsigned int *err) {
     constexpr int NTS = WySmem::NTS, XST = WySmem::XST;
+    constexpr bool SUB16 = SUB == 16;
+    static_assert(SUB == C || (SUB == 16 && !CH), "16-token chunks: scalar gate only");
+    // same method chunk: m and l in one SUB-row block
+    auto same = [](int m, int l) { return !SUB16 || (m >> 4) == (l >> 4); };
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint8_t *sKQ = sm + WySmem::KQ, *sT = sm + WySmem::TT;
@@ -294,32 +302,34 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     // per-channel gate: this chunk takes the exact route (see the file header)
     int fb = 0;
     if (!CH && warp == 0) {
+        // rows 0-31 in a, 32-63 in b; 16-token chunks scan each 16-row block
         float a = sG[lane], b = sG[lane + 32];
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
+        for (int off = 1; off < (SUB16 ? 16 : 32); off <<= 1) {
             const float ya = __shfl_up_sync(0xffffffffu, a, off);
             const float yb = __shfl_up_sync(0xffffffffu, b, off);
-            if (lane >= off) {
+            if ((SUB16 ? (lane & 15) : lane) >= off) {
                 a += ya;
                 b += yb;
             }
         }
-        b += __shfl_sync(0xffffffffu, a, 31);
+        if (!SUB16) b += __shfl_sync(0xffffffffu, a, 31);
         sG[lane] = a;
         sG[lane + 32] = b;
-        // Gamma[l][m] = e^(G_l - G_m) factorised around the middle row R = G_31 as
-        // e^(G_l - R) e^(R - G_m) -- exact up to rounding while every |G_l - R|
-        // stays far from the fp32 exp range; otherwise the Gram epilogue takes
-        // the exp of each difference (flag 0)
-        const float R = __shfl_sync(0xffffffffu, a, 31);
-        float spread = fmaxf(fabsf(a - R), fabsf(b - R));
+        // Gamma[l][m] = e^(G_l - G_m) factorised around a middle row R (row 31,
+        // or row 7 of each 16-row chunk) as e^(G_l - R) e^(R - G_m) -- exact up
+        // to rounding while every |G_l - R| stays far from the fp32 exp range;
+        // otherwise the Gram epilogue takes the exp of each difference (flag 0)
+        const float Ra = __shfl_sync(0xffffffffu, a, SUB16 ? ((lane & 16) | 7) : 31);
+        const float Rb = SUB16 ? __shfl_sync(0xffffffffu, b, (lane & 16) | 7) : Ra;
+        float spread = fmaxf(fabsf(a - Ra), fabsf(b - Rb));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
             spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, off));
-        eA[lane] = __expf(a - R);
-        eA[lane + 32] = __expf(b - R);
-        eB[lane] = __expf(R - a);
-        eB[lane + 32] = __expf(R - b);
+        eA[lane] = __expf(a - Ra);
+        eA[lane + 32] = __expf(b - Rb);
+        eB[lane] = __expf(Ra - a);
+        eB[lane + 32] = __expf(Rb - b);
         if (lane == 0) *sFact = spread < geo.spread_limit;
     }
     {
@@ -429,7 +439,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                     kcv[k] = pack8(kc);
                 }
             } else {
-                const float eq = __expf(sG[l]), ek = __expf(sG[C - 1] - sG[l]);
+                const float eq = __expf(sG[l]), ek = __expf(sG[SUB16 ? (l | 15) : C - 1] - sG[l]);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     wq[i] = qv[i] * eq;
@@ -439,9 +449,13 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             *reinterpret_cast<uint4 *>(Qg + l * D + c0) = pack8(wq);
             *reinterpret_cast<uint4 *>(Kg + l * D + c0) = pack8(wk);
         }
-        if (tid < D)
+        if (SUB16) {  // one decay row per 16-token chunk
+            for (int e = tid; e < (C / 16) * D; e += kWyThreads)
+                ws.dec[slot * (C / 16) * D + e] = __expf(sG[(e / D) * 16 + 15]);
+        } else if (tid < D) {
             ws.dec[slot * D + tid] = CH ? (fb ? __expf(sGC[tid]) : eCR[tid] * eR[tid])
                                         : __expf(sG[C - 1]);
+        }
         if (CH && !fb) {  // the gate tile is read: K-check takes its first half
             __syncthreads();
 #pragma unroll
@@ -492,7 +506,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int m = m0 + i;
-                        sN[m * NTS + l] = (m < l) ? bl * gr[i] * gam(m) : 0.f;
+                        sN[m * NTS + l] = (m < l && same(m, l)) ? bl * gr[i] * gam(m) : 0.f;
                     }
                 } else {
 #pragma unroll
@@ -501,7 +515,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const int m = m0 + jj * 8 + i;
-                            o[i] = (m <= l) ? gr[jj * 8 + i] * gam(m) : 0.f;
+                            o[i] = (m <= l && same(m, l)) ? gr[jj * 8 + i] * gam(m) : 0.f;
                         }
                         const int j = hf * 4 + jj;
                         *reinterpret_cast<uint4 *>(sT + l * 128 + ((j ^ (l & 7)) << 4)) = pack8(o);
@@ -637,82 +651,87 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             for (int i = 0; i < 16; ++i) sX[(16 * b + i) * XST + 16 * b + j] = x[i];
         }
         __syncthreads();
-        // tasks: strips of 4 rows x 1 column of a 16 x 16 block (float4 over N^T rows)
-        const int c = tid & 15, r0 = ((tid >> 4) & 3) * 4, blk = tid >> 6;
-        {   // level A: X_10 = -X_11 (N_10 X_00), X_32 = -X_33 (N_32 X_22)
-            const int j = blk * 2, i = j + 1;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            if (tid < 128) {
+        if (SUB16) {  // block diagonal: the diagonal blocks are the whole inverse
+            if (tid == kWyTmaThread) bulk_wait_group_read<0>();  // the A staging is read
+            __syncthreads();
+        } else {
+            // tasks: strips of 4 rows x 1 column of a 16 x 16 block (float4 over N^T rows)
+            const int c = tid & 15, r0 = ((tid >> 4) & 3) * 4, blk = tid >> 6;
+            {   // level A: X_10 = -X_11 (N_10 X_00), X_32 = -X_33 (N_32 X_22)
+                const int j = blk * 2, i = j + 1;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                if (tid < 128) {
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float xv = sX[(16 * j + m) * XST + 16 * j + c];
-                    const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * j + m) * NTS + 16 * i + r0);
-                    acc[0] = fmaf(nv.x, xv, acc[0]);
-                    acc[1] = fmaf(nv.y, xv, acc[1]);
-                    acc[2] = fmaf(nv.z, xv, acc[2]);
-                    acc[3] = fmaf(nv.w, xv, acc[3]);
+                    for (int m = 0; m < 16; ++m) {
+                        const float xv = sX[(16 * j + m) * XST + 16 * j + c];
+                        const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * j + m) * NTS + 16 * i + r0);
+                        acc[0] = fmaf(nv.x, xv, acc[0]);
+                        acc[1] = fmaf(nv.y, xv, acc[1]);
+                        acc[2] = fmaf(nv.z, xv, acc[2]);
+                        acc[3] = fmaf(nv.w, xv, acc[3]);
+                    }
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = acc[t];
+                }
+                __syncthreads();
+                float res[4] = {0.f, 0.f, 0.f, 0.f};
+                if (tid < 128) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        const float pv = sX[(16 * i + m) * XST + 16 * j + c];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            res[t] = fmaf(sX[(16 * i + r0 + t) * XST + 16 * i + m], pv, res[t]);
+                    }
+                }
+                __syncthreads();
+                if (tid < 128) {
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = -res[t];
+                }
+                __syncthreads();
+            }
+            {   // level B: P_ij = N_i0 X_0j + N_i1 X_1j (i in {2,3}, j in {0,1});
+                // X_2j = -X_22 P_2j,  X_3j = -(X_32 P_2j + X_33 P_3j)
+                const int i = 2 + (blk >> 1), j = blk & 1;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int kb = j; kb < 2; ++kb) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        const float xv = sX[(16 * kb + m) * XST + 16 * j + c];
+                        const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * kb + m) * NTS + 16 * i + r0);
+                        acc[0] = fmaf(nv.x, xv, acc[0]);
+                        acc[1] = fmaf(nv.y, xv, acc[1]);
+                        acc[2] = fmaf(nv.z, xv, acc[2]);
+                        acc[3] = fmaf(nv.w, xv, acc[3]);
+                    }
                 }
 #pragma unroll
                 for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = acc[t];
-            }
-            __syncthreads();
-            float res[4] = {0.f, 0.f, 0.f, 0.f};
-            if (tid < 128) {
+                __syncthreads();  // N^T is dead from here on
+                float res[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
+                for (int m = 0; m < 16; ++m) {  // X_ii P_ij
                     const float pv = sX[(16 * i + m) * XST + 16 * j + c];
 #pragma unroll
                     for (int t = 0; t < 4; ++t)
                         res[t] = fmaf(sX[(16 * i + r0 + t) * XST + 16 * i + m], pv, res[t]);
                 }
-            }
-            __syncthreads();
-            if (tid < 128) {
+                if (i == 3) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {  // + X_32 P_2j
+                        const float pv = sX[(32 + m) * XST + 16 * j + c];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            res[t] = fmaf(sX[(48 + r0 + t) * XST + 32 + m], pv, res[t]);
+                    }
+                }
+                if (tid == kWyTmaThread) bulk_wait_group_read<0>();  // the A staging is read
+                __syncthreads();
 #pragma unroll
                 for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = -res[t];
+                __syncthreads();
             }
-            __syncthreads();
-        }
-        {   // level B: P_ij = N_i0 X_0j + N_i1 X_1j (i in {2,3}, j in {0,1});
-            // X_2j = -X_22 P_2j,  X_3j = -(X_32 P_2j + X_33 P_3j)
-            const int i = 2 + (blk >> 1), j = blk & 1;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int kb = j; kb < 2; ++kb) {
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float xv = sX[(16 * kb + m) * XST + 16 * j + c];
-                    const float4 nv = *reinterpret_cast<const float4 *>(sN + (16 * kb + m) * NTS + 16 * i + r0);
-                    acc[0] = fmaf(nv.x, xv, acc[0]);
-                    acc[1] = fmaf(nv.y, xv, acc[1]);
-                    acc[2] = fmaf(nv.z, xv, acc[2]);
-                    acc[3] = fmaf(nv.w, xv, acc[3]);
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = acc[t];
-            __syncthreads();  // N^T is dead from here on
-            float res[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {  // X_ii P_ij
-                const float pv = sX[(16 * i + m) * XST + 16 * j + c];
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-                    res[t] = fmaf(sX[(16 * i + r0 + t) * XST + 16 * i + m], pv, res[t]);
-            }
-            if (i == 3) {
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {  // + X_32 P_2j
-                    const float pv = sX[(32 + m) * XST + 16 * j + c];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        res[t] = fmaf(sX[(48 + r0 + t) * XST + 32 + m], pv, res[t]);
-                }
-            }
-            if (tid == kWyTmaThread) bulk_wait_group_read<0>();  // the A staging is read
-            __syncthreads();
-#pragma unroll
-            for (int t = 0; t < 4; ++t) sX[(16 * i + r0 + t) * XST + 16 * j + c] = -res[t];
-            __syncthreads();
         }
         // T[i][j] = X[i][j] beta_j (lower triangle) -> bf16, K-major SW128 tile
         for (int e = tid; e < C * 8; e += kWyThreads) {
@@ -721,7 +740,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int j = j8 * 8 + u;
-                o[u] = (j <= i) ? sX[i * XST + j] * sB[j] : 0.f;
+                o[u] = (j <= i && same(j, i)) ? sX[i * XST + j] * sB[j] : 0.f;
             }
             *reinterpret_cast<uint4 *>(sT + i * 128 + ((j8 ^ (i & 7)) << 4)) = pack8(o);
         }
@@ -845,11 +864,12 @@ struct StSmem {
     // K-> (64 x 128, MN-major B), U^T (128 x 64), A (64 x 64, K-major B)
     static constexpr uint32_t WQ = 0, K = 32768, UT = 49152, A = 65536;
     static constexpr uint32_t STAGE = 73728;
-    static constexpr uint32_t DEC = 2 * STAGE;      // decay [2][128] fp32
-    static constexpr uint32_t OST = DEC + 1024;     // O staging for the TMA store [64][128]
+    static constexpr uint32_t DEC = 2 * STAGE;      // decay rows [2][up to 4][128] fp32
+    static constexpr uint32_t OST = DEC + 4096;     // O staging for the TMA store [64][128]
     static constexpr uint32_t BARS = OST + 16384;
     static constexpr uint32_t TOTAL = BARS + 256;
-    static constexpr uint32_t TX = 4 * kTileBytes + kHalfBytes + kDecBytes;
+    // bytes one stage's loads deliver, with nd decay rows
+    static constexpr uint32_t tx(int nd) { return 4 * kTileBytes + kHalfBytes + nd * kDecBytes; }
 };
 constexpr int kChainThreads = 256, kOutThreads = 128;
 constexpr int kStThreads = kChainThreads + kOutThreads + 64;
@@ -877,10 +897,20 @@ __device__ __forceinline__ bool named_sync_and(int id, int n, bool p) {
 }
 // Chain -> MMA-warp hand-offs on hardware named barriers (the chain warps
 // arrive, the MMA warp syncs).  Both sides pass each barrier exactly twice per
-// chunk on every path, error paths included, so neither can be left waiting.
+// chain step on every path, error paths included, so neither can be left
+// waiting.
+//
+// SUB (the method's chunk, 64 or 16): a stage holds one 64-token tile; with
+// 16-token chunks the chain takes four steps per stage.  Step j uses rows
+// 16j.. of the tile: [Z_j^T | O_j^T] = S [W<-_j; Q<-_j]^T (N = 32, the -W<- and
+// Q<- rows loaded as alternating 16-row blocks so that each step's pair is
+// contiguous), S <- S Diag(decay_j) + Z_j^T K->_j and O_j^T += Z_j^T A_jj^T
+// with the diagonal 16 x 16 block of A; the TMEM buffer holds
+// [Z_0 O_0 Z_1 O_1 ...] in 16-column blocks.
 constexpr int kBarOpsS = 2, kBarOpsZ = 3;
 constexpr int kOpsThreads = 256 + 32;
 
+template <int SUB>
 __global__ void __launch_bounds__(kStThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ CUtensorMap tm_U,
              const __grid_constant__ CUtensorMap tm_Q, const __grid_constant__ CUtensorMap tm_K,
@@ -888,6 +918,8 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
              const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
              float *__restrict__ S_final, const int32_t *__restrict__ cu, Geo geo, Ws ws,
              unsigned int *err) {
+    static_assert(SUB == C || SUB == 16, "method chunk of 64 or 16 tokens");
+    constexpr int NSUB = C / SUB;  // chain steps per stage
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + StSmem::BARS);  // [2] TMA stage loaded
@@ -905,20 +937,27 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
     const int gc0 = geo.varlen ? ws.chunk_start[s] : s * geo.nc;
     const int nch = (int)((t1 - t0 + C - 1) / C);
 
-    auto issue = [&](int r) {  // stage r & 1 <- chunk r's operands and decay row
+    // stage r & 1 <- chunk r's operands and decay rows; -W<- and Q<- arrive as
+    // alternating SUB-row blocks (their maps have SUB-row boxes)
+    auto issue = [&](int r) {
         uint8_t *st = sm + (r & 1) * StSmem::STAGE;
         uint64_t *bar = &full[r & 1];
         const size_t sl = (size_t)(gc0 + r) * geo.H + h;
-        mbar_arrive_expect_tx(bar, StSmem::TX);
-        tma_load_2d(st + StSmem::WQ, &tm_W, bar, 0, (int)(sl * C));
-        tma_load_2d(st + StSmem::WQ + 16384, &tm_W, bar, 64, (int)(sl * C));
+        mbar_arrive_expect_tx(bar, StSmem::tx(NSUB));
+#pragma unroll
+        for (int b = 0; b < NSUB; ++b) {
+            const int y = (int)(sl * C) + b * SUB;
+            tma_load_2d(st + StSmem::WQ + 2 * b * SUB * 128, &tm_W, bar, 0, y);
+            tma_load_2d(st + StSmem::WQ + 16384 + 2 * b * SUB * 128, &tm_W, bar, 64, y);
+            tma_load_2d(st + StSmem::WQ + (2 * b + 1) * SUB * 128, &tm_Q, bar, 0, y);
+            tma_load_2d(st + StSmem::WQ + 16384 + (2 * b + 1) * SUB * 128, &tm_Q, bar, 64, y);
+        }
         tma_load_2d(st + StSmem::UT, &tm_U, bar, 0, (int)(sl * D));
-        tma_load_2d(st + StSmem::WQ + 8192, &tm_Q, bar, 0, (int)(sl * C));
-        tma_load_2d(st + StSmem::WQ + 16384 + 8192, &tm_Q, bar, 64, (int)(sl * C));
         tma_load_2d(st + StSmem::K, &tm_K, bar, 0, (int)(sl * C));
         tma_load_2d(st + StSmem::K + 8192, &tm_K, bar, 64, (int)(sl * C));
         tma_load_2d(st + StSmem::A, &tm_A, bar, 0, (int)(sl * C));
-        bulk_load(sm + StSmem::DEC + (r & 1) * kDecBytes, ws.dec + sl * D, kDecBytes, bar);
+        bulk_load(sm + StSmem::DEC + (r & 1) * NSUB * kDecBytes, ws.dec + sl * NSUB * D,
+                  NSUB * kDecBytes, bar);
     };
     // The TMA thread initialises the stage barriers and issues the first two
     // stages before the CTA barrier, overlapping the TMEM allocation and the
@@ -983,7 +1022,9 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
         for (int r = 0; r < nch; ++r) {
             const uint8_t *st = sm + (r & 1) * StSmem::STAGE;
             if (ok) ok = mbar_wait_bounded(&full[r & 1], (r >> 1) & 1, kSpin, err);
-            if (ok && r > 0) ok = mbar_wait_bounded(barS, (r - 1) & 1, kSpin, err);
+            for (int j = 0; j < NSUB; ++j) {
+            const int q = r * NSUB + j;  // chain step
+            if (ok && q > 0) ok = mbar_wait_bounded(barS, (q - 1) & 1, kSpin, err);
             ok = __all_sync(0xffffffffu, ok);  // the TMEM accesses below are warp-wide
             float v[64];
             if (ok) {  // S (fp32) -> bf16 operand in TMEM
@@ -993,12 +1034,12 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
                 tmem_wait_ld();
                 float p[32];  // bf16 pairs
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 w = pack8(v + j * 8);
-                    p[4 * j] = __uint_as_float(w.x);
-                    p[4 * j + 1] = __uint_as_float(w.y);
-                    p[4 * j + 2] = __uint_as_float(w.z);
-                    p[4 * j + 3] = __uint_as_float(w.w);
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 w = pack8(v + i * 8);
+                    p[4 * i] = __uint_as_float(w.x);
+                    p[4 * i + 1] = __uint_as_float(w.y);
+                    p[4 * i + 2] = __uint_as_float(w.z);
+                    p[4 * i + 3] = __uint_as_float(w.w);
                 }
                 tmem_st16(tS16 + lb + hf * 32, p);
                 tmem_st16(tS16 + lb + hf * 32 + 16, p + 16);
@@ -1009,16 +1050,16 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             named_arrive(kBarOpsS, kOpsThreads);
             if (ok) {  // S <- S Diag(decay), needed by the S-update MMA (after opsZ)
                 const float *dec = reinterpret_cast<const float *>(sm + StSmem::DEC) +
-                                   (r & 1) * D + hf * 64;
+                                   ((r & 1) * NSUB + j) * D + hf * 64;
 #pragma unroll
                 for (int i = 0; i < 64; ++i) v[i] *= dec[i];
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) tmem_st16(tS + lb + hf * 64 + cb * 16, v + cb * 16);
                 tmem_wait_st();
             }
-            if (ok) ok = mbar_wait_bounded(barZ, r & 1, kSpin, err);
+            if (ok) ok = mbar_wait_bounded(barZ, q & 1, kSpin, err);
             ok = __all_sync(0xffffffffu, ok);
-            if (ok) {  // Z^T = U^T - S W<-^T -> bf16 A operand in TMEM (this thread: 32 tokens)
+            if (ok && SUB == C) {  // Z^T = U^T - S W<-^T -> bf16 A operand in TMEM (this thread: 32 tokens)
                 tc_fence_after();
                 float z[32];
                 const uint32_t tZ = tZO0 + (r & 1) * 128;
@@ -1029,9 +1070,9 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
                 float p[16];
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const int j = hf * 4 + jj;
+                    const int c16 = hf * 4 + jj;
                     float u[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(urow + ((j ^ (d & 7)) << 4)), u);
+                    unpack8(*reinterpret_cast<const uint4 *>(urow + ((c16 ^ (d & 7)) << 4)), u);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) u[i] -= z[jj * 8 + i];
                     const uint4 w = pack8(u);
@@ -1043,10 +1084,27 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
                 tmem_st16(tZ16 + lb + hf * 16, p);
                 tmem_wait_st();
                 tc_fence_before();
+            } else if (ok) {  // 16-token chunk j: this thread 8 of its tokens
+                tc_fence_after();
+                float z[8];
+                tmem_ld8(tZO0 + (r & 1) * 128 + 32 * j + hf * 8 + lb, z);
+                tmem_wait_ld();
+                const uint8_t *urow = st + StSmem::UT + d * 128;
+                float u[8];
+                unpack8(*reinterpret_cast<const uint4 *>(urow + (((2 * j + hf) ^ (d & 7)) << 4)), u);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) u[i] -= z[i];
+                const uint4 w = pack8(u);
+                const float p[4] = {__uint_as_float(w.x), __uint_as_float(w.y),
+                                    __uint_as_float(w.z), __uint_as_float(w.w)};
+                tmem_st4(tZ16 + lb + hf * 4, p);
+                tmem_wait_st();
+                tc_fence_before();
             }
             named_arrive(kBarOpsZ, kOpsThreads);
+            }  // chain steps
         }
-        if (ok && nch > 0) ok = mbar_wait_bounded(barS, (nch - 1) & 1, kSpin, err);
+        if (ok && nch > 0) ok = mbar_wait_bounded(barS, (nch * NSUB - 1) & 1, kSpin, err);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         if (ok && S_final) {
@@ -1075,10 +1133,11 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
                                 mbar_wait_bounded(&barO[r & 1], (r >> 1) & 1, kSpin, err));
             if (!ok) break;
             tc_fence_after();
-            float o[64];
+            float o[64];  // token order: O sits after Z in each SUB-column block
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb)
-                tmem_ld16(tZO0 + (r & 1) * 128 + 64 + lb + cb * 16, o + cb * 16);
+                tmem_ld16(tZO0 + (r & 1) * 128 + (SUB == C ? 64 + cb * 16 : 32 * cb + 16) + lb,
+                          o + cb * 16);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -1159,8 +1218,8 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
             if (i >= 0) mbar_wait_bounded(&full[i & 1], (i >> 1) & 1, kSpin, err);
     } else if (warp == 12) {
         // ===================== MMA issue (lane 0; the warp syncs) =====================
-        const uint32_t idZO = idesc_bf16(128, 128, 0, 0);
-        const uint32_t idO = idesc_bf16(128, 64, 0, 0);
+        const uint32_t idZO = idesc_bf16(128, 2 * SUB, 0, 0);
+        const uint32_t idO = idesc_bf16(128, SUB, 0, 0);
         const uint32_t idS = idesc_bf16(128, 128, 0, 1);
         // operand descriptors, built once; k-steps only advance the start address
         const uint64_t dWQ0 = sdesc_sw128(smem_u32(sm + StSmem::WQ), 16, 1024);
@@ -1168,35 +1227,42 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
         const uint64_t dA0 = sdesc_sw128(smem_u32(sm + StSmem::A), 16, 1024);
         const uint32_t stage16 = StSmem::STAGE >> 4;  // stage stride in descriptor units
         for (int r = 0; r < nch; ++r) {
-            const uint32_t tZr = tZO0 + (r & 1) * 128, tO = tZr + 64;
+            const uint32_t tZr = tZO0 + (r & 1) * 128;
             const uint64_t so = (r & 1) ? stage16 : 0;
             const uint64_t dwq = dWQ0 + so, dk = dK0 + so, da = dA0 + so;
             // this buffer's O half must have been read out (chunk r - 2)
             if (ok && lane == 0 && r >= 2)
                 ok = mbar_wait_bounded(&oFree[r & 1], ((r - 2) >> 1) & 1, kSpin, err);
-            __syncwarp();
-            // the chain has written S(r) in bf16 (and so has seen chunk r's stage land)
-            named_sync(kBarOpsS, kOpsThreads);
-            if (ok && lane == 0) {
-                tc_fence_after();
+            for (int j = 0; j < NSUB; ++j) {
+                __syncwarp();
+                // the chain has written S in bf16 (and so has seen chunk r's stage land)
+                named_sync(kBarOpsS, kOpsThreads);
+                const uint32_t tZj = tZr + 2 * SUB * j;  // [Z_j | O_j]
+                if (ok && lane == 0) {
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // [Z^T | O^T] = S [W<-; Q<-]^T
-                    mma_bf16_ts(tZr, tS16 + kk * 8,
-                                sdesc_add(dwq, (kk >> 2) * 16384 + (kk & 3) * 32), idZO, kk > 0);
-                mma_commit(barZ);
-            }
-            __syncwarp();
-            named_sync(kBarOpsZ, kOpsThreads);
-            if (ok && lane == 0) {
-                tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk)  // [Z_j^T | O_j^T] = S [W<-_j; Q<-_j]^T
+                        mma_bf16_ts(tZj, tS16 + kk * 8,
+                                    sdesc_add(dwq, 2 * SUB * j * 128 + (kk >> 2) * 16384 +
+                                                       (kk & 3) * 32),
+                                    idZO, kk > 0);
+                    mma_commit(barZ);
+                }
+                __syncwarp();
+                named_sync(kBarOpsZ, kOpsThreads);
+                if (ok && lane == 0) {
+                    tc_fence_after();
+                    constexpr int KS = SUB / 16;  // k-steps over the chunk's tokens
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // S += Z^T K->
-                    mma_bf16_ts(tS, tZ16 + kk * 8, sdesc_add(dk, kk * 2048), idS, 1);
-                mma_commit(barS);
+                    for (int kk = 0; kk < KS; ++kk)  // S += Z_j^T K->_j
+                        mma_bf16_ts(tS, tZ16 + kk * 8, sdesc_add(dk, (j * KS + kk) * 2048), idS, 1);
+                    mma_commit(barS);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // O^T += Z^T A^T
-                    mma_bf16_ts(tO, tZ16 + kk * 8, sdesc_add(da, kk * 32), idO, 1);
-                mma_commit(&barO[r & 1]);
+                    for (int kk = 0; kk < KS; ++kk)  // O_j^T += Z_j^T A_jj^T
+                        mma_bf16_ts(tZj + SUB, tZ16 + kk * 8,
+                                    sdesc_add(da, j * SUB * 128 + (j * KS + kk) * 32), idO, 1);
+                    if (j == NSUB - 1) mma_commit(&barO[r & 1]);
+                }
             }
         }
     }
@@ -1223,13 +1289,14 @@ struct WsLayout {
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-WsLayout ws_layout(int B, int T, int H, int n_seq, int varlen) {
+// nsub: decay rows per tile (one per method chunk: 1 at 64 tokens, 4 at 16)
+WsLayout ws_layout(int B, int T, int H, int n_seq, int varlen, int nsub = 1) {
     WsLayout L;
     L.n_slots = varlen ? (T + C - 1) / C + n_seq : B * ((T + C - 1) / C);
     const size_t tiles = (size_t)L.n_slots * H;
     size_t o = 0;
     L.plan = o; o += up256(sizeof(int) * (size_t)(2 * (varlen ? n_seq : 0) + 1));
-    L.dec = o;  o += up256(tiles * D * 4);
+    L.dec = o;  o += up256(tiles * nsub * D * 4);
     L.W = o;    o += up256(tiles * C * D * 2);
     L.U = o;    o += up256(tiles * C * D * 2);
     L.Q = o;    o += up256(tiles * C * D * 2);
@@ -1257,8 +1324,21 @@ bool tc_applies(int dk, int dv, int chunk, gdr_dtype dtype) {
     return dtype == GDR_BF16 && dk == D && dv == D && chunk == C;
 }
 
+// gdr_fwd also runs 16-token chunks on the tensor cores (scalar gate, one
+// substep per token)
+bool tc_applies_fwd(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate gate, int keep) {
+    return tc_applies(dk, dv, chunk, dtype) ||
+           (dtype == GDR_BF16 && dk == D && dv == D && chunk == 16 &&
+            gate == GDR_GATE_SCALAR && keep == 1);
+}
+
 size_t tc_workspace_bytes(int B, int T, int H, int n_seq, int varlen, gdr_gate) {
     return ws_layout(B, T, H, n_seq, varlen).total;
+}
+
+size_t tc_workspace_bytes_chunk(int B, int T, int H, int n_seq, int varlen, gdr_gate,
+                                int chunk) {
+    return ws_layout(B, T, H, n_seq, varlen, chunk == 16 ? C / 16 : 1).total;
 }
 
 static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, const float *g,
@@ -1266,9 +1346,13 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
                                const float *S0, void *out, float *S_final, int B, int T, int H,
                                const int32_t *cu, int n_seq, gdr_gate gate, void *workspace,
                                size_t ws_bytes, unsigned int *err, cudaStream_t st,
-                               int keep = 1) {
+                               int keep = 1, int chunk = C) {
     const int varlen = cu != nullptr;
-    const WsLayout L = ws_layout(B, T, H, n_seq, varlen);
+    const bool c16 = chunk == 16;
+    if (!(chunk == C || (c16 && gate == GDR_GATE_SCALAR && !eg && keep == 1)))
+        return cudaErrorInvalidValue;
+    const int sub = c16 ? 16 : C;
+    const WsLayout L = ws_layout(B, T, H, n_seq, varlen, C / sub);
     if (ws_bytes < L.total || !err) return cudaErrorInvalidValue;
     uint8_t *wsb = (uint8_t *)workspace;
     Ws ws;
@@ -1299,9 +1383,9 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
             !make_map(&mv, kBF, v, HD, tok_rows, HD * 2, 64, 64, kSW) ||
             (gate == GDR_GATE_PER_KEY_CHANNEL &&
              !make_map(&mg, kF32, g, HD, tok_rows, HD * 4, D, 64, kNoSW)) ||
-            !make_map(&mW, kBF, ws.W, D, tiles * C, D * 2, 64, 64, kSW) ||
+            !make_map(&mW, kBF, ws.W, D, tiles * C, D * 2, 64, sub, kSW) ||
             !make_map(&mU, kBF, ws.U, C, tiles * D, C * 2, 64, 128, kSW) ||
-            !make_map(&mQ, kBF, ws.Q, D, tiles * C, D * 2, 64, 64, kSW) ||
+            !make_map(&mQ, kBF, ws.Q, D, tiles * C, D * 2, 64, sub, kSW) ||
             !make_map(&mK, kBF, ws.K, D, tiles * C, D * 2, 64, 64, kSW) ||
             !make_map(&mA, kBF, ws.A, C, tiles * C, C * 2, 64, 64, kSW) ||
             !make_map(&mo, kBF, out, HD, tok_rows / keep, HD * 2, D,
@@ -1324,7 +1408,8 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
         // decoupled gates run the per-channel kernel; a scalar decay is broadcast
         const size_t smem = wy_smem_bytes(ch || dec);
         auto kern = dec ? (ch ? wy_kernel<true, true> : wy_kernel<true, true, true>)
-                        : ch ? wy_kernel<true> : wy_kernel<false>;
+                        : ch ? wy_kernel<true> : c16 ? wy_kernel<false, false, false, 16>
+                                                     : wy_kernel<false>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem)) != cudaSuccess)
             return e;
@@ -1337,11 +1422,12 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
     }
     {
         const size_t smem = 1024 + StSmem::TOTAL;
-        if ((e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        auto skern = c16 ? state_kernel<16> : state_kernel<C>;
+        if ((e = cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem)) != cudaSuccess)
             return e;
         ProfToken tk = prof_begin(GDR_K_TC_STATE, st);
-        state_kernel<<<(unsigned)(geo.n_seq * H), kStThreads, smem, st>>>(
+        skern<<<(unsigned)(geo.n_seq * H), kStThreads, smem, st>>>(
             mW, mU, mQ, mK, mA, mo, S0, (__nv_bfloat16 *)out, S_final, cu, geo, ws, err);
         prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1353,9 +1439,9 @@ cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const f
                             const float *beta, const float *S0, void *out, float *S_final, int B,
                             int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
                             void *workspace, size_t ws_bytes, unsigned int *err,
-                            cudaStream_t st) {
+                            cudaStream_t st, int chunk) {
     return tc_dispatch(q, k, v, g, beta, nullptr, nullptr, S0, out, S_final, B, T, H, cu, n_seq,
-                       gate, workspace, ws_bytes, err, st);
+                       gate, workspace, ws_bytes, err, st, 1, chunk);
 }
 
 // Gated DeltaProduct: the prefill over the virtual sequence of keep substeps

@@ -35,11 +35,15 @@ cudaError_t decode_gdn2_dispatch(const void *q, const void *k, const void *v, co
                                  cudaStream_t st);
 // tensor-core path (fwd_tc.cu)
 bool tc_applies(int dk, int dv, int chunk, gdr_dtype dtype);
+bool tc_applies_fwd(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate gate, int keep);
 size_t tc_workspace_bytes(int B, int T, int H, int n_seq, int varlen, gdr_gate gate);
+size_t tc_workspace_bytes_chunk(int B, int T, int H, int n_seq, int varlen, gdr_gate gate,
+                                int chunk);
 cudaError_t fwd_tc_dispatch(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const float *S0, void *out, float *S_final, int B,
                             int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
-                            void *workspace, size_t ws_bytes, unsigned int *err, cudaStream_t st);
+                            void *workspace, size_t ws_bytes, unsigned int *err, cudaStream_t st,
+                            int chunk);
 cudaError_t fwd_tc_keep_dispatch(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const float *S0, void *out, float *S_final,
                                  int B, int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
@@ -128,8 +132,9 @@ bool simt_shape_ok(int dk, int dv, int chunk) {
 }
 
 // Resolve the path; returns GDR_OK and sets *use_tc, or an error.
-gdr_status resolve_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_path path, bool *use_tc) {
-    const bool tc = gdr_host::tc_applies(dk, dv, chunk, dtype);
+gdr_status resolve_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate gate, int keep,
+                        gdr_path path, bool *use_tc) {
+    const bool tc = gdr_host::tc_applies_fwd(dk, dv, chunk, dtype, gate, keep);
     switch (path) {
         case GDR_PATH_AUTO:
             *use_tc = tc;
@@ -196,9 +201,9 @@ size_t gdr_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk, 
     if (!valid_enum(dtype, gate)) return 0;
     if (check_fwd_shapes(B, T, H, d_k, d_v, chunk, n_seq, varlen != 0) != GDR_OK) return 0;
     bool use_tc = false;
-    if (resolve_path(d_k, d_v, chunk, dtype, path, &use_tc) != GDR_OK) return 0;
+    if (resolve_path(d_k, d_v, chunk, dtype, gate, 1, path, &use_tc) != GDR_OK) return 0;
     if (!use_tc) return 0;
-    return gdr_host::tc_workspace_bytes(B, T, H, n_seq, varlen, gate);
+    return gdr_host::tc_workspace_bytes_chunk(B, T, H, n_seq, varlen, gate, chunk);
 }
 
 // The prefill behind gdr_fwd.  keep > 1 (Gated DeltaProduct): the T rows of a
@@ -222,7 +227,7 @@ static gdr_status fwd_common(const void *q, const void *k, const void *v, const 
     gdr_status st = check_fwd_shapes(B, T, H, d_k, d_v, chunk, n_seq, varlen);
     if (st != GDR_OK) return st;
     bool use_tc = false;
-    st = resolve_path(d_k, d_v, chunk, dtype, path, &use_tc);
+    st = resolve_path(d_k, d_v, chunk, dtype, gate, keep, path, &use_tc);
     if (st != GDR_OK) return st;
     if (keep > 1 && (!use_tc || T % keep)) return GDR_OK;  // the caller gathers
     if (ran) *ran = true;
@@ -230,7 +235,7 @@ static gdr_status fwd_common(const void *q, const void *k, const void *v, const 
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     if (use_tc) {  // the dispatcher accounts for its own launches
-        const size_t need = gdr_host::tc_workspace_bytes(B, T, H, n_seq, varlen, gate);
+        const size_t need = gdr_host::tc_workspace_bytes_chunk(B, T, H, n_seq, varlen, gate, chunk);
         if (need && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
             return GDR_ERR_INVALID;
         e = keep > 1 ? gdr_host::fwd_tc_keep_dispatch(q, k, v, g, beta, S0, out, S_final, B, T, H,
@@ -239,7 +244,8 @@ static gdr_status fwd_common(const void *q, const void *k, const void *v, const 
                                                       gdr_host::device_error_word(), s)
                      : gdr_host::fwd_tc_dispatch(q, k, v, g, beta, S0, out, S_final, B, T, H,
                                                  cu_seqlens, nseq, gate, workspace,
-                                                 workspace_bytes, gdr_host::device_error_word(), s);
+                                                 workspace_bytes, gdr_host::device_error_word(), s,
+                                                 chunk);
     } else {
         if ((size_t)gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL,
                                               false) > 227u * 1024u)

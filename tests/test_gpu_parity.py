@@ -346,3 +346,40 @@ def test_tc_varlen_prefill_full_size_sampled(cuda_device):
 def test_tc_varlen_nonzero_state_sampled(cuda_device):
     inp = inputs.prefill_inputs(inputs.PREFILL["varlen_prefill"], s0_var=0.01)
     check_sampled(inp, cuda_device, heads=[1])
+
+
+# ------------------------------------------------------------------ tensor cores, 16-token chunks
+@pytest.mark.parametrize("T", [16, 64, 300, 1])
+def test_tc_chunk16_against_oracle(cuda_device, T):
+    """16-token chunks on the tensor cores (scalar gate): each 64-token tile is
+    four chunks of the method, so sequences of 1, 16, 64 and 300 tokens cover
+    a partial chunk, whole tiles and a partial tile."""
+    cfg = small_cfg(B=2, T=T, H=3, chunk=16)
+    check(inputs.prefill_inputs(cfg, seed=311), cuda_device, path="tc", chunk=16)
+
+
+@pytest.mark.parametrize("gate_scale", [0.1, 4.0])
+def test_tc_chunk16_matches_simt(cuda_device, gate_scale):
+    """The same 16-token chunk algorithm on the tensor cores and on the CUDA
+    cores; with scale 4 the per-chunk spread passes the factorisation's limit."""
+    cfg = small_cfg(B=1, T=515, H=4, chunk=16, gate_scale=gate_scale)
+    inp = inputs.prefill_inputs(cfg, seed=312)
+    O1, S1 = run_fwd(inp, cuda_device, path="tc", chunk=16)
+    O2, S2 = run_fwd(inp, cuda_device, path="simt", chunk=16)
+    assert prefill_out_rel(O1, O2) < 1e-2 and state_rel(S1, S2) < 1e-2
+    check(inp, cuda_device, path="tc", chunk=16)
+
+
+def test_tc_chunk16_varlen_with_empty_and_unit_sequences(cuda_device):
+    cfg = inputs.PREFILL["varlen_prefill"].replace(T=600, H=2, n_seq=0, s0_var=0.01, chunk=16)
+    inp = inputs.prefill_inputs(cfg, seed=313)
+    inp.cu_seqlens = np.array([0, 0, 1, 17, 65, 200, 200, 600], dtype=np.int32)
+    inp.S0 = np.random.default_rng(7).standard_normal((7, 2, 128, 128)).astype(np.float32) * 0.1
+    check(inp, cuda_device, path="tc", chunk=16)
+
+
+def test_tc_gdn_prefill_chunk16_full_size_sampled(cuda_device):
+    """The Gated DeltaNet prefill workload at 16-token chunks, full size, as
+    the benchmark's chunk-16 line runs it; oracle on 2 heads x 4 sequences."""
+    inp = inputs.prefill_inputs(inputs.PREFILL["gdn_prefill_c16"])
+    check_sampled(inp, cuda_device, heads=[2, 13])
