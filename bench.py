@@ -714,8 +714,8 @@ def main():
                     choices=list(inputs.PREFILL) + list(inputs.DECODE) + list(inputs.FRAME))
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--extra", default=("kda_prefill,varlen_prefill,gdp_prefill,gdn2_prefill,"
-                                        "frame_prefill,gdn_prefill_c16,gdn_prefill_c128,decode,"
-                                        "kda_decode"),
+                                        "frame_prefill,gdn_prefill_c16,kda_prefill_c16,"
+                                        "gdn_prefill_c128,decode,kda_decode"),
                     help="comma-separated workloads measured after the main one ('' for none)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

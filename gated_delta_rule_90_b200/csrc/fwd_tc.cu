@@ -209,10 +209,12 @@ struct WySmem {
     static constexpr uint32_t small_bytes(bool ch) { return small_floats(ch) * 4 + 64; }
 };
 
-// SUB (scalar gate): the chunk size of the method, 64 or 16.  With 16 a
+// SUB: the chunk size of the method, 64 or 16 (not with DEC).  With 16 a
 // 64-token tile holds four chunks: G restarts every 16 rows, L, A and T are
 // block diagonal (the 16 x 16 diagonal blocks of the 64 x 64 solve), K->
-// decays to each chunk's own end, and four decay rows are written.
+// decays to each chunk's own end, and four decay rows are written.  The
+// per-channel Gram then factorises around each chunk's start (G = 0), so the
+// reading factor e^G is K<-'s own and only the chunk ends G_C are tabulated.
 // DEC (per-channel decay only): Gated DeltaNet-2's erase gate b and write gate
 // w replace beta ("Gated DeltaNet-2, and the gate that was doing two jobs",
 // section "What decoupling actually means here"): the Gram's reading rows are
@@ -231,7 +233,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           unsigned int *err) {
     constexpr int NTS = WySmem::NTS, XST = WySmem::XST;
     constexpr bool SUB16 = SUB == 16;
-    static_assert(SUB == C || (SUB == 16 && !CH), "16-token chunks: scalar gate only");
+    static_assert(SUB == C || (SUB == 16 && !DEC && !BC), "16-token chunks: not with DEC");
     // same method chunk: m and l in one SUB-row block
     auto same = [](int m, int l) { return !SUB16 || (m >> 4) == (l >> 4); };
     extern __shared__ uint8_t smem_raw[];
@@ -250,6 +252,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     float *sB = CH ? sSm : sSm + 64;                                   // beta [64]
     // exponential tables, so that no element-wise exp is needed below
     float *eR = sSm + 64, *eCR = sTf + 2 * D;                          // channel: per channel
+    float *sGC4 = sTf, *eCR4 = sTf + 4 * D;  // channel, 16-token chunks: G_C, e^(G_C) [4][128]
     float *eA = sX, *eB = sX + 64;                                     // scalar: per row (XR)
     int *sFact = reinterpret_cast<int *>(sX + 128);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sSm + WySmem::small_floats(CH));  // [2]
@@ -344,19 +347,21 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = (r0 + i < len) ? sGt[(r0 + i) * D + c] : 0.f;
 #pragma unroll
-        for (int i = 1; i < 32; ++i) v[i] += v[i - 1];
-        // spread = max_l |G_l - R| of this channel (R = G_31)
+        for (int i = 1; i < 32; ++i)
+            if (!SUB16 || i != 16) v[i] += v[i - 1];  // 16-token chunks restart at row 16
+        // spread = max_l |G_l - R| of this channel (R = G_31; for 16-token
+        // chunks R = 0, the chunk's start)
         float spread = 0.f;
         if (!r0) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 sGt[i * D + c] = v[i];
-                spread = fmaxf(spread, fabsf(v[i] - v[31]));
+                spread = fmaxf(spread, fabsf(v[i] - (SUB16 ? 0.f : v[31])));
             }
         }
         __syncthreads();
         if (r0) {
-            const float base = sGt[31 * D + c];
+            const float base = SUB16 ? 0.f : sGt[31 * D + c];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 sGt[(32 + i) * D + c] = v[i] + base;
@@ -364,7 +369,13 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             }
         }
         fb = __syncthreads_or(!(spread < geo.spread_limit));
-        if (tid < D) {
+        if (SUB16) {  // each chunk's G_C and decay e^(G_C)
+            for (int e = tid; e < (C / 16) * D; e += kWyThreads) {
+                const float GC = sGt[((e / D) * 16 + 15) * D + (e % D)];
+                sGC4[e] = GC;
+                eCR4[e] = __expf(GC);
+            }
+        } else if (tid < D) {
             const float R = sGt[31 * D + tid], GC = sGt[(C - 1) * D + tid];
             sG[tid] = R;    // reference row R of the Gram factorisation
             sGC[tid] = GC;  // G_C
@@ -391,13 +402,20 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         const int cg = tid & 15, c0 = cg * 8, a = cg >> 3, l0 = tid >> 4;
         float R8[8], eR8[8], eCR8[8];
         uint4 kcv[C / 16];  // per-channel gate: K-check, stored once G is read
-        if (CH) {
+        if (CH && SUB16) {  // R = 0: e^R = 1; e^(G_C - R) per chunk, below
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                R8[i] = 0.f;
+                eR8[i] = 1.f;
+            }
+        } else if (CH) {
             ld8(sG + c0, R8);
             ld8(eR + c0, eR8);
             ld8(eCR + c0, eCR8);
         }
 #pragma unroll
         for (int k = 0; k < C / 16; ++k) {
+            if (CH && SUB16) ld8(eCR4 + k * D + c0, eCR8);  // row l is in chunk k
             const int l = l0 + 16 * k, j = (cg & 7) ^ (l & 7);  // physical 16-byte chunk
             const uint32_t off = a * 16384 + l * 128 + j * 16;
             float kv[8], qv[8], wq[8], wk[8];
@@ -417,7 +435,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 }
                 if (fb) {  // exact route: e^G and e^(G_C - G) themselves (at most 1)
                     float GC8[8];
-                    ld8(sGC + c0, GC8);
+                    ld8(SUB16 ? sGC4 + k * D + c0 : sGC + c0, GC8);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         wq[i] = qv[i] * __expf(G8[i]);
@@ -451,7 +469,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         }
         if (SUB16) {  // one decay row per 16-token chunk
             for (int e = tid; e < (C / 16) * D; e += kWyThreads)
-                ws.dec[slot * (C / 16) * D + e] = __expf(sG[(e / D) * 16 + 15]);
+                ws.dec[slot * (C / 16) * D + e] = CH ? eCR4[e] : __expf(sG[(e / D) * 16 + 15]);
         } else if (tid < D) {
             ws.dec[slot * D + tid] = CH ? (fb ? __expf(sGC[tid]) : eCR[tid] * eR[tid])
                                         : __expf(sG[C - 1]);
@@ -542,11 +560,11 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         float *Nsc = reinterpret_cast<float *>(ws.W + slot * (C * D));
         __nv_bfloat16 *Ag = ws.A + slot * (C * C);
         for (int e = tid; e < C * C; e += kWyThreads)
-            if (e % C > e / C) Ag[e] = __float2bfloat16_rn(0.f);
+            if (e % C > e / C || !same(e % C, e / C)) Ag[e] = __float2bfloat16_rn(0.f);
         const int qa = lane >> 4, qc = lane & 15;  // atom, 4-channel group
         int gi = 0;
         for (int l = 0; l < C; ++l) {
-            for (int m0 = 0; m0 <= l; m0 += 4, ++gi) {
+            for (int m0 = SUB16 ? (l & ~15) : 0; m0 <= l; m0 += 4, ++gi) {
                 if ((gi & 7) != warp) continue;
                 const float4 gl = *reinterpret_cast<const float4 *>(sGt + l * D + 4 * lane);
                 float el[4], ql[4], acc[8];
@@ -613,7 +631,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         __syncthreads();  // the gate tile is dead: N^T into its place
         for (int e = tid; e < C * C; e += kWyThreads) {
             const int m = e / C, l = e % C;
-            sN[m * NTS + l] = (m < l) ? Nsc[e] : 0.f;
+            sN[m * NTS + l] = (m < l && same(m, l)) ? Nsc[e] : 0.f;
         }
     }
     fence_proxy_async_smem();
@@ -749,7 +767,12 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         {
             const int cg = tid & 15, c0 = cg * 8, a = cg >> 3, l0 = tid >> 4;
             float eR8[8];
-            if (CH) ld8(eR + c0, eR8);
+            if (CH && SUB16) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) eR8[i] = 1.f;  // K^ is K<- when R = 0
+            } else if (CH) {
+                ld8(eR + c0, eR8);
+            }
 #pragma unroll
             for (int k = 0; k < C / 16; ++k) {
                 const int l = l0 + 16 * k, jj = (cg & 7) ^ (l & 7);
@@ -1324,12 +1347,11 @@ bool tc_applies(int dk, int dv, int chunk, gdr_dtype dtype) {
     return dtype == GDR_BF16 && dk == D && dv == D && chunk == C;
 }
 
-// gdr_fwd also runs 16-token chunks on the tensor cores (scalar gate, one
+// gdr_fwd also runs 16-token chunks on the tensor cores (either gate, one
 // substep per token)
-bool tc_applies_fwd(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate gate, int keep) {
+bool tc_applies_fwd(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate, int keep) {
     return tc_applies(dk, dv, chunk, dtype) ||
-           (dtype == GDR_BF16 && dk == D && dv == D && chunk == 16 &&
-            gate == GDR_GATE_SCALAR && keep == 1);
+           (dtype == GDR_BF16 && dk == D && dv == D && chunk == 16 && keep == 1);
 }
 
 size_t tc_workspace_bytes(int B, int T, int H, int n_seq, int varlen, gdr_gate) {
@@ -1349,8 +1371,7 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
                                int keep = 1, int chunk = C) {
     const int varlen = cu != nullptr;
     const bool c16 = chunk == 16;
-    if (!(chunk == C || (c16 && gate == GDR_GATE_SCALAR && !eg && keep == 1)))
-        return cudaErrorInvalidValue;
+    if (!(chunk == C || (c16 && !eg && keep == 1))) return cudaErrorInvalidValue;
     const int sub = c16 ? 16 : C;
     const WsLayout L = ws_layout(B, T, H, n_seq, varlen, C / sub);
     if (ws_bytes < L.total || !err) return cudaErrorInvalidValue;
@@ -1408,8 +1429,9 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
         // decoupled gates run the per-channel kernel; a scalar decay is broadcast
         const size_t smem = wy_smem_bytes(ch || dec);
         auto kern = dec ? (ch ? wy_kernel<true, true> : wy_kernel<true, true, true>)
-                        : ch ? wy_kernel<true> : c16 ? wy_kernel<false, false, false, 16>
-                                                     : wy_kernel<false>;
+                        : ch ? (c16 ? wy_kernel<true, false, false, 16> : wy_kernel<true>)
+                             : c16 ? wy_kernel<false, false, false, 16>
+                                   : wy_kernel<false>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem)) != cudaSuccess)
             return e;

@@ -101,9 +101,12 @@ PREFILL = {
                                  0.01, seed_index=5, n_h=2),
     "gdn2_prefill": PrefillConfig("gdn2_prefill", 2, 4096, 16, 128, 128, 64, "bf16", "channel", 0.05,
                                   0.0, seed_index=6, variant="gdn2"),
-    # the Gated DeltaNet workload at the other chunk sizes (CUDA-core path)
+    # the Gated DeltaNet and per-channel workloads at the other chunk sizes
+    # (16: tensor cores; 128: CUDA cores)
     "gdn_prefill_c16": PrefillConfig("gdn_prefill_c16", 4, 4096, 16, 128, 128, 16, "bf16",
                                      "scalar", 0.1, 0.01, seed_index=1),
+    "kda_prefill_c16": PrefillConfig("kda_prefill_c16", 2, 8192, 32, 128, 128, 16, "bf16",
+                                     "channel", 0.05, 0.0, seed_index=2),
     "gdn_prefill_c128": PrefillConfig("gdn_prefill_c128", 4, 4096, 16, 128, 128, 128, "bf16",
                                       "scalar", 0.1, 0.01, seed_index=1),
 }

@@ -54,8 +54,8 @@ typedef enum { GDR_GATE_SCALAR = 0, GDR_GATE_PER_KEY_CHANNEL = 1 } gdr_gate;
 
 /* Which kernels run the prefill.
  *  GDR_PATH_AUTO        tensor-core path when it applies (bf16, d_k = d_v = 128,
- *                       chunk = 64, or chunk = 16 with the scalar gate in
- *                       gdr_fwd), else the SIMT path.
+ *                       chunk = 64, or chunk = 16 in gdr_fwd), else the SIMT
+ *                       path.
  *  GDR_PATH_SIMT        fp32 CUDA-core kernels (any supported shape; the only
  *                       path for fp32 inputs).
  *  GDR_PATH_TENSORCORE  tcgen05/TMEM + TMA kernels; GDR_ERR_UNSUPPORTED where
@@ -89,8 +89,8 @@ size_t gdr_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk, 
  *  out      [B, T, H, d_v]   dtype, written for every token
  *           (with B*T == 0 the token tensors may be NULL; S_final = S0)
  *  S_final  [N, H, d_v, d_k] fp32 final states, or NULL to skip
- *  chunk    16, 32, 64 or 128 (SIMT); 64, and 16 with the scalar gate
- *           (tensor-core path: a 64-token tile then holds four 16-token chunks,
+ *  chunk    16, 32, 64 or 128 (SIMT); 64 or 16 (tensor-core path; at 16 a
+ *           64-token tile holds four 16-token chunks,
  *           with block-diagonal L, A and T and four chain steps per tile).
  *           Every chunk size gives the token recurrence's result up to
  *           rounding.  At 128 the SIMT path streams the chunk's key channels

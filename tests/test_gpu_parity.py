@@ -349,20 +349,24 @@ def test_tc_varlen_nonzero_state_sampled(cuda_device):
 
 
 # ------------------------------------------------------------------ tensor cores, 16-token chunks
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
 @pytest.mark.parametrize("T", [16, 64, 300, 1])
-def test_tc_chunk16_against_oracle(cuda_device, T):
-    """16-token chunks on the tensor cores (scalar gate): each 64-token tile is
-    four chunks of the method, so sequences of 1, 16, 64 and 300 tokens cover
-    a partial chunk, whole tiles and a partial tile."""
-    cfg = small_cfg(B=2, T=T, H=3, chunk=16)
+def test_tc_chunk16_against_oracle(cuda_device, T, gate):
+    """16-token chunks on the tensor cores: each 64-token tile is four chunks
+    of the method, so sequences of 1, 16, 64 and 300 tokens cover a partial
+    chunk, whole tiles and a partial tile."""
+    cfg = small_cfg(B=2, T=T, H=3, chunk=16, gate=gate,
+                    gate_scale=0.1 if gate == "scalar" else 0.05, s0_var=0.01)
     check(inputs.prefill_inputs(cfg, seed=311), cuda_device, path="tc", chunk=16)
 
 
-@pytest.mark.parametrize("gate_scale", [0.1, 4.0])
-def test_tc_chunk16_matches_simt(cuda_device, gate_scale):
+@pytest.mark.parametrize("gate,gate_scale", [("scalar", 0.1), ("scalar", 4.0),
+                                             ("channel", 0.05), ("channel", 12.0)])
+def test_tc_chunk16_matches_simt(cuda_device, gate, gate_scale):
     """The same 16-token chunk algorithm on the tensor cores and on the CUDA
-    cores; with scale 4 the per-chunk spread passes the factorisation's limit."""
-    cfg = small_cfg(B=1, T=515, H=4, chunk=16, gate_scale=gate_scale)
+    cores; with the large scales the per-chunk spread passes the
+    factorisation's limit and the chunks take the exact route."""
+    cfg = small_cfg(B=1, T=515, H=4, chunk=16, gate=gate, gate_scale=gate_scale)
     inp = inputs.prefill_inputs(cfg, seed=312)
     O1, S1 = run_fwd(inp, cuda_device, path="tc", chunk=16)
     O2, S2 = run_fwd(inp, cuda_device, path="simt", chunk=16)
@@ -383,3 +387,9 @@ def test_tc_gdn_prefill_chunk16_full_size_sampled(cuda_device):
     the benchmark's chunk-16 line runs it; oracle on 2 heads x 4 sequences."""
     inp = inputs.prefill_inputs(inputs.PREFILL["gdn_prefill_c16"])
     check_sampled(inp, cuda_device, heads=[2, 13])
+
+
+def test_tc_kda_prefill_chunk16_full_size_sampled(cuda_device):
+    """The per-channel-gate workload (B=2, H=32, T=8192) at 16-token chunks."""
+    inp = inputs.prefill_inputs(inputs.PREFILL["kda_prefill"].replace(chunk=16))
+    check_sampled(inp, cuda_device, heads=[4, 27])
