@@ -209,7 +209,7 @@ struct WySmem {
     static constexpr uint32_t small_bytes(bool ch) { return small_floats(ch) * 4 + 64; }
 };
 
-// SUB: the chunk size of the method, 64 or 16 (not with DEC).  With 16 a
+// SUB: the chunk size of the method, 64 or 16.  With 16 a
 // 64-token tile holds four chunks: G restarts every 16 rows, L, A and T are
 // block diagonal (the 16 x 16 diagonal blocks of the 64 x 64 solve), K->
 // decays to each chunk's own end, and four decay rows are written.  The
@@ -233,7 +233,7 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           unsigned int *err) {
     constexpr int NTS = WySmem::NTS, XST = WySmem::XST;
     constexpr bool SUB16 = SUB == 16;
-    static_assert(SUB == C || (SUB == 16 && !DEC && !BC), "16-token chunks: not with DEC");
+    static_assert(SUB == C || SUB == 16, "method chunk of 64 or 16 tokens");
     // same method chunk: m and l in one SUB-row block
     auto same = [](int m, int l) { return !SUB16 || (m >> 4) == (l >> 4); };
     extern __shared__ uint8_t smem_raw[];
@@ -1347,11 +1347,10 @@ bool tc_applies(int dk, int dv, int chunk, gdr_dtype dtype) {
     return dtype == GDR_BF16 && dk == D && dv == D && chunk == C;
 }
 
-// gdr_fwd also runs 16-token chunks on the tensor cores (either gate, one
-// substep per token)
-bool tc_applies_fwd(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate, int keep) {
-    return tc_applies(dk, dv, chunk, dtype) ||
-           (dtype == GDR_BF16 && dk == D && dv == D && chunk == 16 && keep == 1);
+// The prefill entry points also run 16-token chunks on the tensor cores
+// (gdr_fwd_noalloc keeps to 64)
+bool tc_applies_fwd(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate, int) {
+    return dtype == GDR_BF16 && dk == D && dv == D && (chunk == C || chunk == 16);
 }
 
 size_t tc_workspace_bytes(int B, int T, int H, int n_seq, int varlen, gdr_gate) {
@@ -1363,6 +1362,10 @@ size_t tc_workspace_bytes_chunk(int B, int T, int H, int n_seq, int varlen, gdr_
     return ws_layout(B, T, H, n_seq, varlen, chunk == 16 ? C / 16 : 1).total;
 }
 
+size_t tc_workspace_bytes_gdn2_chunk(int B, int T, int H, int n_seq, int varlen, int chunk) {
+    return ws_layout(B, T, H, n_seq, varlen, chunk == 16 ? C / 16 : 1).total;
+}
+
 static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, const float *g,
                                const float *beta, const float *eg, const float *wg,
                                const float *S0, void *out, float *S_final, int B, int T, int H,
@@ -1371,7 +1374,7 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
                                int keep = 1, int chunk = C) {
     const int varlen = cu != nullptr;
     const bool c16 = chunk == 16;
-    if (!(chunk == C || (c16 && !eg && keep == 1))) return cudaErrorInvalidValue;
+    if (!(chunk == C || c16)) return cudaErrorInvalidValue;
     const int sub = c16 ? 16 : C;
     const WsLayout L = ws_layout(B, T, H, n_seq, varlen, C / sub);
     if (ws_bytes < L.total || !err) return cudaErrorInvalidValue;
@@ -1428,7 +1431,8 @@ static cudaError_t tc_dispatch(const void *q, const void *k, const void *v, cons
         const bool dec = eg != nullptr;
         // decoupled gates run the per-channel kernel; a scalar decay is broadcast
         const size_t smem = wy_smem_bytes(ch || dec);
-        auto kern = dec ? (ch ? wy_kernel<true, true> : wy_kernel<true, true, true>)
+        auto kern = dec ? (ch ? (c16 ? wy_kernel<true, true, false, 16> : wy_kernel<true, true>)
+                              : (c16 ? wy_kernel<true, true, true, 16> : wy_kernel<true, true, true>))
                         : ch ? (c16 ? wy_kernel<true, false, false, 16> : wy_kernel<true>)
                              : c16 ? wy_kernel<false, false, false, 16>
                                    : wy_kernel<false>;
@@ -1473,10 +1477,10 @@ cudaError_t fwd_tc_keep_dispatch(const void *q, const void *k, const void *v, co
                                  const float *beta, const float *S0, void *out, float *S_final,
                                  int B, int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
                                  int keep, void *workspace, size_t ws_bytes, unsigned int *err,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, int chunk) {
     if (keep < 1 || T % keep) return cudaErrorInvalidValue;
     return tc_dispatch(q, k, v, g, beta, nullptr, nullptr, S0, out, S_final, B, T, H, cu, n_seq,
-                       gate, workspace, ws_bytes, err, st, keep);
+                       gate, workspace, ws_bytes, err, st, keep, chunk);
 }
 
 // Gated DeltaNet-2: erase gate eg [.., d_k], write gate wg [.., d_v]; the decay
@@ -1485,10 +1489,10 @@ cudaError_t fwd_tc_gdn2_dispatch(const void *q, const void *k, const void *v, co
                                  const float *eg, const float *wg, const float *S0, void *out,
                                  float *S_final, int B, int T, int H, const int32_t *cu, int n_seq,
                                  gdr_gate gate, void *workspace, size_t ws_bytes,
-                                 unsigned int *err, cudaStream_t st) {
+                                 unsigned int *err, cudaStream_t st, int chunk) {
     if (!eg || !wg) return cudaErrorInvalidValue;
     return tc_dispatch(q, k, v, g, nullptr, eg, wg, S0, out, S_final, B, T, H, cu, n_seq, gate,
-                       workspace, ws_bytes, err, st);
+                       workspace, ws_bytes, err, st, 1, chunk);
 }
 
 }  // namespace gdr_host

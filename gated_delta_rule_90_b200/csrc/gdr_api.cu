@@ -28,7 +28,8 @@ cudaError_t fwd_tc_gdn2_dispatch(const void *q, const void *k, const void *v, co
                                  const float *eg, const float *wg, const float *S0, void *out,
                                  float *S_final, int B, int T, int H, const int32_t *cu, int n_seq,
                                  gdr_gate gate, void *workspace, size_t ws_bytes,
-                                 unsigned int *err, cudaStream_t st);
+                                 unsigned int *err, cudaStream_t st, int chunk);
+size_t tc_workspace_bytes_gdn2_chunk(int B, int T, int H, int n_seq, int varlen, int chunk);
 cudaError_t decode_gdn2_dispatch(const void *q, const void *k, const void *v, const float *g,
                                  const float *eg, const float *wg, float *S, void *out, int N,
                                  int H, int dk, int dv, gdr_dtype dtype, gdr_gate gate,
@@ -48,7 +49,7 @@ cudaError_t fwd_tc_keep_dispatch(const void *q, const void *k, const void *v, co
                                  const float *beta, const float *S0, void *out, float *S_final,
                                  int B, int T, int H, const int32_t *cu, int n_seq, gdr_gate gate,
                                  int keep, void *workspace, size_t ws_bytes, unsigned int *err,
-                                 cudaStream_t st);
+                                 cudaStream_t st, int chunk);
 }  // namespace gdr_host
 
 // ------------------------------------------------------------ device error word
@@ -154,9 +155,9 @@ gdr_status resolve_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate gat
 }
 
 // Gated DeltaNet-2 takes the tensor-core path with either decay.
-gdr_status resolve_gdn2_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate,
+gdr_status resolve_gdn2_path(int dk, int dv, int chunk, gdr_dtype dtype, gdr_gate gate,
                              gdr_path path, bool *use_tc) {
-    const bool tc = gdr_host::tc_applies(dk, dv, chunk, dtype);
+    const bool tc = gdr_host::tc_applies_fwd(dk, dv, chunk, dtype, gate, 1);
     switch (path) {
         case GDR_PATH_AUTO: *use_tc = tc; break;
         case GDR_PATH_SIMT: *use_tc = false; break;
@@ -241,7 +242,7 @@ static gdr_status fwd_common(const void *q, const void *k, const void *v, const 
         e = keep > 1 ? gdr_host::fwd_tc_keep_dispatch(q, k, v, g, beta, S0, out, S_final, B, T, H,
                                                       cu_seqlens, nseq, gate, keep, workspace,
                                                       workspace_bytes,
-                                                      gdr_host::device_error_word(), s)
+                                                      gdr_host::device_error_word(), s, chunk)
                      : gdr_host::fwd_tc_dispatch(q, k, v, g, beta, S0, out, S_final, B, T, H,
                                                  cu_seqlens, nseq, gate, workspace,
                                                  workspace_bytes, gdr_host::device_error_word(), s,
@@ -292,7 +293,7 @@ size_t gdr_fwd_gdn2_workspace_size(int B, int T, int H, int d_k, int d_v, int ch
     bool use_tc = false;
     if (resolve_gdn2_path(d_k, d_v, chunk, dtype, gate, path, &use_tc) != GDR_OK) return 0;
     if (!use_tc) return 0;
-    return gdr_host::tc_workspace_bytes(B, T, H, n_seq, varlen, gate);
+    return gdr_host::tc_workspace_bytes_gdn2_chunk(B, T, H, n_seq, varlen, chunk);
 }
 
 gdr_status gdr_fwd_gdn2(const void *q, const void *k, const void *v, const float *g,
@@ -316,12 +317,12 @@ gdr_status gdr_fwd_gdn2(const void *q, const void *k, const void *v, const float
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     if (use_tc) {  // the dispatcher accounts for its own launches
-        const size_t need = gdr_host::tc_workspace_bytes(B, T, H, n_seq, varlen, gate);
+        const size_t need = gdr_host::tc_workspace_bytes_gdn2_chunk(B, T, H, n_seq, varlen, chunk);
         if (need && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
             return GDR_ERR_INVALID;
         e = gdr_host::fwd_tc_gdn2_dispatch(q, k, v, g, b, w, S0, out, S_final, B, T, H,
                                            cu_seqlens, nseq, gate, workspace, workspace_bytes,
-                                           gdr_host::device_error_word(), s);
+                                           gdr_host::device_error_word(), s, chunk);
     } else {
         if (gdr_host::simt_smem_bytes(chunk, d_k, gate == GDR_GATE_PER_KEY_CHANNEL, true) >
             227u * 1024u)

@@ -54,8 +54,7 @@ typedef enum { GDR_GATE_SCALAR = 0, GDR_GATE_PER_KEY_CHANNEL = 1 } gdr_gate;
 
 /* Which kernels run the prefill.
  *  GDR_PATH_AUTO        tensor-core path when it applies (bf16, d_k = d_v = 128,
- *                       chunk = 64, or chunk = 16 in gdr_fwd), else the SIMT
- *                       path.
+ *                       chunk = 64 or 16), else the SIMT path.
  *  GDR_PATH_SIMT        fp32 CUDA-core kernels (any supported shape; the only
  *                       path for fp32 inputs).
  *  GDR_PATH_TENSORCORE  tcgen05/TMEM + TMA kernels; GDR_ERR_UNSUPPORTED where

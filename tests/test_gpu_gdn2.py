@@ -173,3 +173,12 @@ def test_gdn2_prefill_full_size_sampled(cuda_device):
     assert np.isfinite(O).all() and np.isfinite(SF).all()
     eo, es = prefill_out_rel(O[:, :, hs], Or), state_rel(SF[:, hs], SFr)
     assert eo <= 1e-2 and es <= 1e-2, (eo, es)
+
+
+@pytest.mark.parametrize("gate", ["channel", "scalar"])
+@pytest.mark.parametrize("T", [64, 300])
+def test_gdn2_tc_chunk16_against_oracle(cuda_device, T, gate):
+    """Gated DeltaNet-2 with 16-token chunks on the tensor cores."""
+    cfg = cfg_of(B=2, T=T, H=3, s0_var=0.01, gate=gate, chunk=16,
+                 gate_scale=0.05 if gate == "channel" else 0.1)
+    check(inputs.gdn2_inputs(cfg, seed=612), cuda_device, chunk=16, path="tc")

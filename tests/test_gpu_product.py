@@ -85,3 +85,13 @@ def test_gdp_prefill_full_size_sampled(cuda_device):
     assert np.isfinite(O).all() and np.isfinite(SF).all()
     eo, es = prefill_out_rel(O[:, :, heads], Or), state_rel(SF[:, heads], SFr)
     assert eo <= 1e-2 and es <= 1e-2, (eo, es)
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("n_h", [2, 3])
+def test_gdp_tc_bf16_chunk16(cuda_device, gate, n_h):
+    """Gated DeltaProduct with 16-step chunks of the virtual sequence on the
+    tensor cores (four chunks per 64-step tile)."""
+    cfg = cfg_of(B=2, T=150, H=3, gate=gate, n_h=n_h, chunk=16,
+                 gate_scale=0.1 if gate == "scalar" else 0.05)
+    check(inputs.product_inputs(cfg, seed=505), cuda_device, "tc")
