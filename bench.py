@@ -43,8 +43,8 @@ _TC_SRC = ('csrc/fwd_tc.cu', 'csrc/sm100.cuh', 'csrc/common.cuh')
 _DEC_SRC = ('csrc/decode.cu', 'csrc/common.cuh')
 _FR_SRC = ('csrc/frame.cu', 'csrc/sm100.cuh', 'csrc/tmap.cuh', 'csrc/common.cuh')
 NCU_TRAFFIC = {
-    ("tc_wy", "gdn_prefill"): (_TC_SRC, "31ad39eb861feed8", 206.273024e6 + 255.766016e6),
-    ("tc_state", "gdn_prefill"): (_TC_SRC, "31ad39eb861feed8", 308.367360e6 + 56.410112e6),
+    ("tc_wy", "gdn_prefill"): (_TC_SRC, "0ab89a53881ca31f", 206.257408e6 + 255.669760e6),
+    ("tc_state", "gdn_prefill"): (_TC_SRC, "0ab89a53881ca31f", 308.456960e6 + 56.687104e6),
     ("tc_wy", "kda_prefill"): (_TC_SRC, "31ad39eb861feed8", 681.934848e6 + 578.909184e6),
     ("decode", "decode"): (_DEC_SRC, "82e1f5016f476188", 543.250944e6 + 482.361600e6),
     ("decode", "kda_decode"): (_DEC_SRC, "82e1f5016f476188", 547.403264e6 + 482.458624e6),
