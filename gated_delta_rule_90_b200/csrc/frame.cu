@@ -21,11 +21,12 @@
 //   frame_chain   (batch*head, row block) S_t = (S_{t-1} D_t + C_t) W_t over
 //                                         the frames (rows of S are independent)
 //   frame_out     (token tile, head, batch) o_i = S_t q_i
-// The inverse and the chain are fp32 on the CUDA cores.
-// The two dense contractions over tokens -- the Gram pass and the output pass
-// -- run on the tensor cores for bf16 inputs with d_k = d_v = 128 (tcgen05,
-// operands staged by TMA, fp32 accumulators in TMEM), and on the CUDA cores
-// in fp32 otherwise.
+// The inverse is fp32 on the CUDA cores.  For bf16 inputs with
+// d_k = d_v = 128 the two dense contractions over tokens -- the Gram pass and
+// the output pass -- run on the tensor cores (tcgen05, operands staged by TMA,
+// fp32 accumulators in TMEM), and so does the chain, in a three-term bf16
+// split that keeps its products at fp32 accuracy; otherwise all four passes
+// are fp32 on the CUDA cores.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -125,7 +126,10 @@ constexpr int kSwThreads = 512;  // (d_k / 4) x (d_k / 8) tiles of 4 x 8, d_k <=
 // Thread (row group rg, column group cg) holds rows 4 rg .. 4 rg + 3 and the
 // columns 4 cg .. 4 cg + 3 and d_k/2 + 4 cg .. + 3, so that the float4 reads of
 // a pivot row by the column groups cover contiguous bytes (no bank conflicts).
-template <int DK>
+// With SPLIT the result is written as two bf16 matrices instead, W_hi = bf16(W)
+// and W_lo = bf16(W - W_hi), one after the other in the slot's first half
+// (the operands of the tensor-core chain).
+template <int DK, bool SPLIT>
 __global__ void __launch_bounds__(kSwThreads, 2)
 frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
     __shared__ __align__(16) float buf[2][128];  // pivot rows
@@ -204,7 +208,7 @@ frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
             }
         }
     }
-    if (act) {
+    if (act && !SPLIT) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float *o = Gp + (size_t)(r0 + i) * DK;
@@ -212,13 +216,43 @@ frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
             *reinterpret_cast<float4 *>(o + jB) = make_float4(-a[i][4], -a[i][5], -a[i][6], -a[i][7]);
         }
     }
+    if (act && SPLIT) {  // every read of G happened before the first barrier
+        __nv_bfloat16 *wh = reinterpret_cast<__nv_bfloat16 *>(Gp), *wl = wh + DK * DK;
+        // two consecutive entries of -a as packed bf16 pairs (hi, lo)
+        auto split2 = [](float x, float y, uint32_t &hi, uint32_t &lo) {
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(-x, -y);
+            const float2 hf = __bfloat1622float2(h2);
+            const __nv_bfloat162 l2 = __floats2bfloat162_rn(-x - hf.x, -y - hf.y);
+            hi = *reinterpret_cast<const uint32_t *>(&h2);
+            lo = *reinterpret_cast<const uint32_t *>(&l2);
+        };
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint2 h0, h1, l0, l1;
+            split2(a[i][0], a[i][1], h0.x, l0.x);
+            split2(a[i][2], a[i][3], h0.y, l0.y);
+            split2(a[i][4], a[i][5], h1.x, l1.x);
+            split2(a[i][6], a[i][7], h1.y, l1.y);
+            const size_t o = (size_t)(r0 + i) * DK;
+            *reinterpret_cast<uint2 *>(wh + o + jA) = h0;
+            *reinterpret_cast<uint2 *>(wh + o + jB) = h1;
+            *reinterpret_cast<uint2 *>(wl + o + jA) = l0;
+            *reinterpret_cast<uint2 *>(wl + o + jB) = l1;
+        }
+    }
 }
 
-static cudaError_t launch_inverse(float *GW, const Dims &d, unsigned int *err, cudaStream_t st) {
+static cudaError_t launch_inverse(float *GW, const Dims &d, bool split, unsigned int *err,
+                                  cudaStream_t st) {
     const dim3 gf((unsigned)d.F, (unsigned)d.H, (unsigned)d.B);
+    if (split) {
+        if (d.dk != 128) return cudaErrorInvalidValue;
+        frame_inverse_kernel<128, true><<<gf, kSwThreads, 0, st>>>(GW, d, err);
+        return cudaGetLastError();
+    }
     switch (d.dk) {
 #define GDR_INV(DK) \
-    case DK: frame_inverse_kernel<DK><<<gf, kSwThreads, 0, st>>>(GW, d, err); break
+    case DK: frame_inverse_kernel<DK, false><<<gf, kSwThreads, 0, st>>>(GW, d, err); break
         GDR_INV(16); GDR_INV(32); GDR_INV(48); GDR_INV(64);
         GDR_INV(80); GDR_INV(96); GDR_INV(112); GDR_INV(128);
 #undef GDR_INV
@@ -227,9 +261,8 @@ static cudaError_t launch_inverse(float *GW, const Dims &d, unsigned int *err, c
     return cudaGetLastError();
 }
 
-// S_t = (S_{t-1} D_t + C_t) W_t for kChainRows rows of S; every S_t is stored
-// for the output pass (fp32, or its bf16 copy for the tensor-core output pass),
-// the last one also as S_final.  W_t arrives by bulk copy into one of two
+// S_t = (S_{t-1} D_t + C_t) W_t for kChainRows rows of S in fp32 on the CUDA
+// cores; every S_t is stored for the output pass, the last one also as S_final.  W_t arrives by bulk copy into one of two
 // buffers, one frame ahead.  Thread (row pair rp = warp, column group cg =
 // lane) owns rows 2 rp, 2 rp + 1 and columns 4 cg .. 4 cg + 3: each float4 read
 // of a W_t row serves both rows (the chain is bound by shared-memory reads),
@@ -238,8 +271,7 @@ __global__ void __launch_bounds__(kThreads)
 frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
                    const float *__restrict__ g, int per_channel,
                    const float *__restrict__ S0, float *__restrict__ Sw,
-                   __nv_bfloat16 *__restrict__ Sb, float *__restrict__ S_final, Dims d,
-                   unsigned int *err) {
+                   float *__restrict__ S_final, Dims d, unsigned int *err) {
     extern __shared__ __align__(16) float sm[];
     const int bh = blockIdx.x, b = bh / d.H, h = bh % d.H;
     const int r0 = blockIdx.y * kChainRows;
@@ -334,17 +366,8 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
             *reinterpret_cast<float4 *>(Sr0 + c4) = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
             *reinterpret_cast<float4 *>(Sr1 + c4) = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
             const size_t o = sl * (size_t)d.dv * dk + (size_t)(r0 + 2 * rp) * dk + c4;
-            if (Sb) {  // operand of the tensor-core output pass
-                __nv_bfloat162 p0[2] = {__floats2bfloat162_rn(acc0[0], acc0[1]),
-                                        __floats2bfloat162_rn(acc0[2], acc0[3])};
-                __nv_bfloat162 p1[2] = {__floats2bfloat162_rn(acc1[0], acc1[1]),
-                                        __floats2bfloat162_rn(acc1[2], acc1[3])};
-                if (mine0) *reinterpret_cast<uint2 *>(Sb + o) = *reinterpret_cast<uint2 *>(p0);
-                if (mine1) *reinterpret_cast<uint2 *>(Sb + o + dk) = *reinterpret_cast<uint2 *>(p1);
-            } else {
-                if (mine0) *reinterpret_cast<float4 *>(Sw + o) = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
-                if (mine1) *reinterpret_cast<float4 *>(Sw + o + dk) = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
-            }
+            if (mine0) *reinterpret_cast<float4 *>(Sw + o) = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
+            if (mine1) *reinterpret_cast<float4 *>(Sw + o + dk) = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
         }
         __syncthreads();
     }
@@ -521,8 +544,206 @@ frame_gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// S_t = (S_{t-1} D_t + C_t) W_t on the tensor cores, for kCR rows of S per CTA.
+// Rows of S are independent, and W_t is symmetric, so the step is computed
+// transposed: S_t^T [128 x kCR] = W_t [128 x 128] * A_t^T with
+// A_t = S_{t-1} D_t + C_t.  W_t is the K-major A operand, A_t^T the MN-major B
+// operand (row m of it = key channel m over this CTA's rows of S), and the
+// accumulator's TMEM lane j holds column j of S_t.  So a thread on TMEM lane j
+// owns key channel j: its decay is one number, its C_t entries are column j of
+// the CTA's row block, and its piece of the B operand is contiguous.
+// kSplit threads share each channel (warps w, w + 4, ... reach the same TMEM
+// lanes), each with kCR / kSplit of the rows.
+//
+// fp32 accuracy from bf16 products by the three-term split (Henry, Tang and
+// Heinecke, "Leveraging the bfloat16 Artificial Intelligence Datatype For
+// Higher-Precision Computations", 2019): x = x_hi + x_lo with x_hi = bf16(x),
+// x_lo = bf16(x - x_hi), and
+//     A W ~ A_hi W_hi + A_hi W_lo + A_lo W_hi
+// (the dropped A_lo W_lo term is about 2^-16 of the product).  The inverse pass
+// writes W_hi and W_lo; the chain splits A_t itself.  A_hi^T and A_lo^T sit
+// side by side as one B operand of N = 2 kCR, so W_hi [A_hi^T A_lo^T] is one
+// MMA per K step (accumulator columns [0, kCR) and [kCR, 2 kCR)), and
+// W_lo A_hi^T adds into the first half: 16 MMAs per frame.
+//
+// Per frame: wait for the previous frame's MMAs, read S_{t-1} from TMEM (the
+// sum of the two halves), form A_t and its two parts in shared memory, issue
+// the MMAs, then -- while they run -- store S_{t-1} as the bf16 operand of the
+// output pass (transposed, key channel major).  W_t (TMA, 64 KB) and the CTA's
+// row block of C_t (one bulk copy, 32 KB) arrive together one frame ahead into
+// one of two stages.
+constexpr int kCR = 64;                      // rows of S per CTA
+constexpr int kSplit = 4;                    // threads per key channel
+constexpr int kChainThreads = 128 * kSplit;
+constexpr int kHR = kCR / kSplit;            // rows per thread
+constexpr int kWStages = 2;                  // stage ring depth
+constexpr uint32_t kWBytes = 4 * 16384;      // W_hi, W_lo: two 64-column atoms each
+constexpr uint32_t kCBytes = kCR * kTD * 4;  // C_t rows r0 .. r0 + kCR - 1, fp32
+constexpr uint32_t kStage = kWBytes + kCBytes;
+constexpr uint32_t kBBytes = 128 * kCR * 2;  // one part of A_t^T (MN-major, 128 B rows)
+constexpr size_t kChainTcSmem = 1024 + kWStages * kStage + 2 * kBBytes + 64;
+static_assert(kChainTcSmem <= 232448, "the chain's shared memory exceeds one CTA's limit");
+static_assert(kCR == 64, "one 128-byte swizzle atom of A_t^T rows per part");
+static_assert(kHR % 16 == 0, "whole 16-column TMEM loads per thread");
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+frame_chain_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__restrict__ Cw,
+                      const float *__restrict__ g, int per_channel, const float *__restrict__ S0,
+                      __nv_bfloat16 *__restrict__ Sb, float *__restrict__ S_final, Dims d,
+                      unsigned int *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *Bop = sm + kWStages * kStage;                                  // A_hi^T, then A_lo^T
+    uint64_t *wfull = reinterpret_cast<uint64_t *>(Bop + 2 * kBBytes);      // [kWStages]
+    uint64_t *mdone = wfull + kWStages;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mdone + 1);
+    const int bh = blockIdx.x, b = bh / d.H, h = bh % d.H;
+    const int r0 = blockIdx.y * kCR;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int j = (warp & 3) * 32 + (tid & 31);  // key channel = TMEM lane
+    const int hr = (warp >> 2) * kHR;            // this thread's rows: r0 + hr .. + kHR - 1
+    const size_t soff = ((size_t)b * d.H + h) * (size_t)kTD * kTD;
+    if (tid == 0) {
+        for (int i = 0; i < kWStages; ++i) mbar_init(&wfull[i], 1);
+        mbar_init(mdone, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 2 * kCR);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tslot;
+    const uint32_t tacc = tbase + ((uint32_t)((warp & 3) * 32) << 16) + hr;  // lanes, first column
+    auto load_w = [&](int f) {  // W_hi rows at slot * 256, W_lo rows 128 further; C_t block
+        const int st = f % kWStages;
+        uint8_t *wb = sm + st * kStage;
+        const size_t sl = slot(d, b, f, h);
+        const int y = (int)(sl * 2 * kTD);
+        mbar_arrive_expect_tx(&wfull[st], kStage);
+        tma_load_2d(wb, &tm_w, &wfull[st], 0, y);
+        tma_load_2d(wb + 16384, &tm_w, &wfull[st], 64, y);
+        tma_load_2d(wb + 32768, &tm_w, &wfull[st], 0, y + kTD);
+        tma_load_2d(wb + 49152, &tm_w, &wfull[st], 64, y + kTD);
+        bulk_load(wb + kWBytes, Cw + (sl * kTD + r0) * (size_t)kTD, kCBytes, &wfull[st]);
+    };
+    int issued = 0, committed = 0;  // stage loads issued, frames whose MMAs were committed (tid 0)
+    if (tid == 0) {
+        prefetch_tmap(&tm_w);
+        for (; issued < kWStages && issued < d.F; ++issued) load_w(issued);
+    }
+    float s[kHR];
+#pragma unroll
+    for (int r = 0; r < kHR; ++r) s[r] = S0 ? S0[soff + (size_t)(r0 + hr + r) * kTD + j] : 0.f;
+    auto decay = [&](int f) {
+        const size_t sl = slot(d, b, f, h);
+        return per_channel ? g[sl * kTD + j] : g[sl];
+    };
+    float gj = decay(0);
+    // this thread's piece of S_t^T (bf16, key channel major) for the output pass
+    auto store_sb = [&](int f) {
+        __nv_bfloat16 *o = Sb + (slot(d, b, f, h) * kTD + j) * kTD + r0 + hr;
+#pragma unroll
+        for (int q = 0; q < kHR / 8; ++q) reinterpret_cast<uint4 *>(o)[q] = pack8(s + 8 * q);
+    };
+    auto load_s = [&]() {  // S = columns [0, kCR) + columns [kCR, 2 kCR)
+#pragma unroll
+        for (int q = 0; q < kHR / 16; ++q) {
+            float x[16];
+            tmem_ld16(tacc + 16 * q, s + 16 * q);
+            tmem_ld16(tacc + kCR + 16 * q, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) s[16 * q + u] += x[u];
+        }
+    };
+    const uint32_t id2 = idesc_bf16(128, 2 * kCR, 0, 1), id1 = idesc_bf16(128, kCR, 0, 1);
+    bool ok = true;
+    for (int f = 0; f < d.F; ++f) {
+        if (f > 0) {
+            const bool okm = mbar_wait_bounded(mdone, (f - 1) & 1, kSpinF, err);
+            if (!__syncthreads_and(okm)) { ok = false; break; }
+            tc_fence_after();
+            if (tid == 0 && f + kWStages - 1 < d.F) {  // frame f - 1's stage is free
+                load_w(f + kWStages - 1);
+                issued = f + kWStages;
+            }
+            load_s();
+        }
+        const int st = f % kWStages;
+        const bool okw = mbar_wait_bounded(&wfull[st], (f / kWStages) & 1, kSpinF, err);
+        if (!__syncthreads_and(okw)) { ok = false; break; }
+        {  // A_t = S_{t-1} D_t + C_t, split; this thread's piece of row j of both parts
+            const float dj = expf(gj);
+            const float *cs = reinterpret_cast<const float *>(sm + st * kStage + kWBytes) + j;
+#pragma unroll
+            for (int q = 0; q < kHR / 8; ++q) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = 8 * q + 2 * u;
+                    const float a0 = fmaf(s[r], dj, cs[(hr + r) * kTD]);
+                    const float a1 = fmaf(s[r + 1], dj, cs[(hr + r + 1) * kTD]);
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+                    const float2 hf = __bfloat1622float2(h2);
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+                    hi[u] = *reinterpret_cast<const uint32_t *>(&h2);
+                    lo[u] = *reinterpret_cast<const uint32_t *>(&l2);
+                }
+                const int qg = (hr >> 3) + q;  // 16-byte chunk of the 128-byte row
+                const uint32_t off = (uint32_t)(j * 128 + ((qg ^ (j & 7)) << 4));
+                *reinterpret_cast<uint4 *>(Bop + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(Bop + kBBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t wb = smem_u32(sm + st * kStage);
+            const uint64_t dwh = sdesc_sw128(wb, 16, 1024), dwl = sdesc_sw128(wb + 32768, 16, 1024);
+            const uint64_t db = sdesc_sw128(smem_u32(Bop), kBBytes, 1024);  // lbo: A_hi^T -> A_lo^T
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // W_hi [A_hi^T A_lo^T]
+                mma_bf16_ss(tbase, sdesc_add(dwh, (kk >> 2) * 16384 + (kk & 3) * 32),
+                            sdesc_add(db, kk * 2048), id2, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // + W_lo A_hi^T
+                mma_bf16_ss(tbase, sdesc_add(dwl, (kk >> 2) * 16384 + (kk & 3) * 32),
+                            sdesc_add(db, kk * 2048), id1, 1);
+            mma_commit(mdone);
+            committed = f + 1;
+        }
+        if (f > 0) store_sb(f - 1);  // s still holds S_{t-1}
+        if (f + 1 < d.F) gj = decay(f + 1);
+    }
+    if (ok && d.F > 0) {
+        ok = __syncthreads_and(mbar_wait_bounded(mdone, (d.F - 1) & 1, kSpinF, err));
+        tc_fence_after();
+        if (ok) {
+            load_s();
+            store_sb(d.F - 1);
+            if (S_final)
+#pragma unroll
+                for (int r = 0; r < kHR; ++r) S_final[soff + (size_t)(r0 + hr + r) * kTD + j] = s[r];
+        }
+    }
+    if (tid == 0) {  // work still in flight on an error path lands before TMEM and smem go
+        if (committed > 0) mbar_wait_bounded(mdone, (committed - 1) & 1, kSpinF, err);
+        for (int i = max(0, issued - kWStages); i < issued; ++i)
+            mbar_wait_bounded(&wfull[i % kWStages], (i / kWStages) & 1, kSpinF, err);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 2 * kCR);
+}
+
 // o_i = S_t q_i for a tile of 128 tokens of one frame on the tensor cores:
-// D[128 tokens x 128] = Q (K-major A) * S_t^T (bf16 copy of S_t, K-major B).
+// D[128 tokens x 128] = Q (K-major A) * S_t^T, the B operand being the chain's
+// bf16 copy of S_t^T (key channel major, so MN-major: 64-column atoms 16 KB apart).
 __global__ void __launch_bounds__(128)
 frame_out_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_s,
                     __nv_bfloat16 *__restrict__ out, Dims d, unsigned int *err) {
@@ -550,7 +771,7 @@ frame_out_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    // Q: two 64-feature atoms of [128 tokens][64]; S_t: two atoms of [128 rows (d_v)][64 (d_k)]
+    // Q: two 64-feature atoms of [128 tokens][64]; S_t^T: two atoms of [128 rows (d_k)][64 (d_v)]
     if (tid == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_s);
@@ -567,13 +788,13 @@ frame_out_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bool ok = mbar_wait_bounded(&bar[0], 0, kSpinF, err);
     if (__syncthreads_and(ok) && tid == 0) {
         tc_fence_after();
-        const uint32_t id = idesc_bf16(128, 128, 0, 0);
+        const uint32_t id = idesc_bf16(128, 128, 0, 1);
         const uint64_t da = sdesc_sw128(smem_u32(sm), 16, 1024);
-        const uint64_t db = sdesc_sw128(smem_u32(sm + 32768), 16, 1024);
+        const uint64_t db = sdesc_sw128(smem_u32(sm + 32768), 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
             mma_bf16_ss(tmem, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32),
-                        sdesc_add(db, (kk >> 2) * 16384 + (kk & 3) * 32), id, kk > 0);
+                        sdesc_add(db, kk * 2048), id, kk > 0);
         mma_commit(&bar[1]);
     }
     ok = ok && mbar_wait_bounded(&bar[1], 0, kSpinF, err);
@@ -611,7 +832,10 @@ namespace {
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct FrameLayout {
-    size_t GM, CN, Sw, total;  // Sw holds fp32 S_t, or their bf16 copies on the tensor-core path
+    // GM: G_t, overwritten by W_t (fp32; on the tensor-core path W_hi and W_lo in bf16)
+    // CN: C_t (fp32)
+    // Sw: fp32 S_t (on the tensor-core path bf16 S_t^T)
+    size_t GM, CN, Sw, total;
 };
 
 FrameLayout frame_layout(int B, int T, int H, int dk, int dv, int n) {
@@ -643,7 +867,7 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
     __nv_bfloat16 *Sb = (__nv_bfloat16 *)(ws + L.Sw);
     const bool tc = frame_tc_applies(d, sizeof(Tin) == 2);
     cudaError_t e;
-    CUtensorMap mk, mv, mq, ms;
+    CUtensorMap mk, mv, mq, ms, mw;
     if (tc) {
         using namespace gdr_host::tmap;
         const uint64_t rows = (uint64_t)d.B * d.T, HD = (uint64_t)d.H * kTD;
@@ -651,7 +875,8 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
         if (!make_map(&mk, kBF, k, HD, rows, HD * 2, 64, 64, kSW) ||
             !make_map(&mv, kBF, v, HD, rows, HD * 2, 64, 64, kSW) ||
             !make_map(&mq, kBF, q, HD, rows, HD * 2, 64, 64, kSW) ||
-            !make_map(&ms, kBF, Sb, kTD, srows, kTD * 2, 64, 128, kSW))
+            !make_map(&ms, kBF, Sb, kTD, srows, kTD * 2, 64, 128, kSW) ||
+            !make_map(&mw, kBF, GM, kTD, 2 * srows, kTD * 2, 64, 128, kSW))  // W_hi, W_lo per slot
             return cudaErrorInvalidValue;
     }
     const size_t sm_gram = sizeof(float) * (size_t)(kTokTile * (d.dk + 1) + kTokTile * (d.dv + 1) + kTokTile);
@@ -665,6 +890,7 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
     const size_t sm_gram_tc = 1024 + 2 * kGStage + 1024, sm_out_tc = 1024 + 65536 + 64;
     if (tc &&
         ((e = cudaFuncSetAttribute(frame_gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gram_tc)) ||
+         (e = cudaFuncSetAttribute(frame_chain_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChainTcSmem)) ||
          (e = cudaFuncSetAttribute(frame_out_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out_tc))))
         return e;
     {
@@ -678,15 +904,21 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
     }
     {
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_SOLVE, st);
-        e = launch_inverse(GM, d, err, st);
+        e = launch_inverse(GM, d, tc, err, st);
         gdr_host::prof_end(tk, st);
         if (e != cudaSuccess) return e;
     }
     {
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_FRAME_CHAIN, st);
-        const dim3 gc((unsigned)(d.B * d.H), (unsigned)((d.dv + kChainRows - 1) / kChainRows));
-        frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, g, per_channel, S0, Sw,
-                                                           tc ? Sb : nullptr, S_final, d, err);
+        if (tc) {
+            const dim3 gc((unsigned)(d.B * d.H), (unsigned)(kTD / kCR));
+            frame_chain_tc_kernel<<<gc, kChainThreads, kChainTcSmem, st>>>(mw, CN, g, per_channel, S0,
+                                                                           Sb, S_final, d, err);
+        } else {
+            const dim3 gc((unsigned)(d.B * d.H), (unsigned)((d.dv + kChainRows - 1) / kChainRows));
+            frame_chain_kernel<<<gc, kThreads, sm_chain, st>>>(GM, CN, g, per_channel, S0, Sw,
+                                                               S_final, d, err);
+        }
         gdr_host::prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

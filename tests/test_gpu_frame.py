@@ -115,3 +115,24 @@ def test_frame_prefill_full_size_sampled(cuda_device):
     assert np.isfinite(O).all() and np.isfinite(SF).all()
     eo, es = prefill_out_rel(O[:, :, hs], Or), state_rel(SF[:, hs], SFr)
     assert eo <= 1e-2 and es <= 1e-2, (eo, es)
+
+
+def test_frame_tc_chain_keeps_fp32_accuracy(cuda_device):
+    """The tensor-core chain multiplies in a three-term bf16 split.  With every
+    writing strength a power of two, gamma * k is exact in bf16, so the
+    tensor-core Gram pass matches the fp32 one up to summation order, and the
+    gap between the two paths' S_final on the same (bf16-valued) inputs is the
+    chain's own rounding: about 1e-5 for the split, about 1e-3 had the chain
+    multiplied plain bf16 values."""
+    dev = cuda_device
+    cfg = cfg_of(B=1, T=4096, H=3, n=256, s0_var=0.01)
+    inp = inputs.frame_inputs(cfg, seed=706)
+    inp.gamma = np.exp2(np.round(np.log2(inp.gamma))).astype(np.float32)
+    _, SF_tc = run_gpu(inp, dev)
+    f = lambda x: to_dev(x, "f32", dev)
+    _, SF32 = binding.gdr_fwd_frame(f(inp.q), f(inp.k), f(inp.v), f(inp.g), f(inp.gamma), cfg.n,
+                                    f(inp.S0))  # fp32 inputs: the CUDA-core passes
+    torch.cuda.synchronize()
+    assert binding.device_status() == binding.GDR_OK
+    gap = state_rel(SF_tc, to_np(SF32))
+    assert gap <= 1e-4, gap
