@@ -15,8 +15,14 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdr.so")
+# The checked build (kernels guard their accesses; see gdr.h, gdr_checked_build).
+CHECKED_LIB_PATH = os.path.join(_HERE, "libgdr_check.so")
+# GDR_LIBRARY=<path> loads another build of the same library instead, e.g.
+# CHECKED_LIB_PATH.
+LIB_ENV = "GDR_LIBRARY"
 
-GDR_OK, GDR_ERR_INVALID, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT = range(5)
+GDR_OK, GDR_ERR_INVALID, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT, GDR_ERR_BOUNDS = \
+    range(6)
 GDR_F32, GDR_BF16 = 0, 1
 GDR_GATE_SCALAR, GDR_GATE_PER_KEY_CHANNEL = 0, 1
 PATHS = {"auto": 0, "simt": 1, "tc": 2}
@@ -33,13 +39,20 @@ class GdrError(RuntimeError):
         super().__init__(f"{what}: {status_string(status)}")
 
 
+def library_path() -> str:
+    """The library lib() loads: $GDR_LIBRARY if set, else libgdr.so."""
+    return os.environ.get(LIB_ENV) or LIB_PATH
+
+
 def lib() -> ctypes.CDLL:
     """Load libgdr.so (built in-tree by __graft_entry__.build())."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"libgdr.so is not built ({LIB_PATH}); run __graft_entry__.build()")
-        L = ctypes.CDLL(LIB_PATH)
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{os.path.basename(path)} is not built ({path}); "
+                               "run __graft_entry__.build()")
+        L = ctypes.CDLL(path)
         vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         L.gdr_status_string.restype = ctypes.c_char_p
         L.gdr_status_string.argtypes = [i]
@@ -54,6 +67,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_device_status.argtypes = [vp]
         L.gdr_selftest_wait_timeout.restype = i
         L.gdr_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+        L.gdr_checked_build.restype = i
+        L.gdr_checked_build.argtypes = []
+        L.gdr_selftest_bounds.restype = i
+        L.gdr_selftest_bounds.argtypes = [vp]
         L.gdr_fwd_product_workspace_size.restype = sz
         L.gdr_fwd_product_workspace_size.argtypes = [i] * 12
         L.gdr_fwd_product.restype = i
@@ -357,6 +374,15 @@ def device_status(stream=None) -> int:
 
 def selftest_wait_timeout(spin_limit: int, stream=None) -> int:
     return int(lib().gdr_selftest_wait_timeout(spin_limit, _stream(stream)))
+
+
+def checked_build() -> bool:
+    """True when the loaded library is the checked build (gdr.h, gdr_checked_build)."""
+    return bool(lib().gdr_checked_build())
+
+
+def selftest_bounds(stream=None) -> int:
+    return int(lib().gdr_selftest_bounds(_stream(stream)))
 
 
 def set_gram_spread_limit(limit: float) -> float:

@@ -9,10 +9,51 @@
 
 namespace gdr {
 
-// Device error word bits (see gdr_device_status).
-// Bits of the device error word: a bounded wait expired; a factorisation met a
-// non-positive pivot (a negative writing strength, or NaN input).
-enum : unsigned int { kErrTimeout = 1u, kErrNumeric = 2u };
+// Bits of the device error word (see gdr_device_status): a bounded wait
+// expired; a factorisation met a non-positive pivot (a negative writing
+// strength, or NaN input); a bounds guard of the checked build refused an access.
+enum : unsigned int { kErrTimeout = 1u, kErrNumeric = 2u, kErrBounds = 4u };
+
+// ---------------------------------------------------------------- checked build
+// Compiled with -DGDR_CHECK, every kernel checks, before it touches memory,
+// the spans of each global buffer that its CTA will read or write (and the
+// coordinates of its TMA copies) against the extents the entry point was
+// called with.  A miss sets kErrBounds in the device error word and the CTA
+// returns without touching anything, before any barrier, TMEM allocation or
+// copy, so the kernel ends normally and gdr_device_status reports
+// GDR_ERR_BOUNDS.  In the normal build the guards compile to nothing.
+#ifdef GDR_CHECK
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+// Is [first, first + count) inside [0, extent)?  (count = 0 always passes.)
+__device__ __forceinline__ bool chk_span(long long first, long long count, long long extent,
+                                         unsigned int *err) {
+    if (!kChecked || count <= 0) return true;
+    if (first >= 0 && first + count <= extent) return true;
+    if (err) atomicOr(err, kErrBounds);
+    return false;
+}
+// A shape condition the kernel's index arithmetic relies on.
+__device__ __forceinline__ bool chk_true(bool cond, unsigned int *err) {
+    if (!kChecked || cond) return true;
+    if (err) atomicOr(err, kErrBounds);
+    return false;
+}
+// A tiled TMA copy of a box_x x box_y box at (x, y) of a tensor with x_extent
+// elements per row (element size esz bytes) and `rows` rows: x must be >= 0
+// with x * esz a multiple of 16 (an unaligned x is an illegal instruction), the
+// box must start inside the tensor, and y >= 0 (loads may run past the end,
+// which the copy fills with zeros; stores are clipped there).
+__device__ __forceinline__ bool chk_tma(long long x, long long y, int esz, long long x_extent,
+                                        long long rows, unsigned int *err) {
+    if (!kChecked) return true;
+    if (x >= 0 && (x * esz) % 16 == 0 && x < x_extent && y >= 0 && y < rows) return true;
+    if (err) atomicOr(err, kErrBounds);
+    return false;
+}
 
 // Token-storage loads/stores: fp32 or bf16, converted to/from fp32.
 __device__ __forceinline__ float ld_in(const float *p, size_t i) { return p[i]; }

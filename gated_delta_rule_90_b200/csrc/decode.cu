@@ -45,11 +45,21 @@ __global__ void __launch_bounds__(kDecodeThreads)
 decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                    const float *__restrict__ g, const float *__restrict__ beta,
                    const float *__restrict__ eg, const float *__restrict__ wg,
-                   float *__restrict__ S, Tin *__restrict__ out, int dv) {
+                   float *__restrict__ S, Tin *__restrict__ out, int dv, long long nheads,
+                   unsigned int *err) {
     constexpr int VEC = DK / 32;
     using V = VecF<VEC>;
     const size_t head = blockIdx.x;  // flattened (sequence, head)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (kChecked) {  // checked build: this head's slices of every buffer, whole row batches
+        const long long hd = (long long)head;
+        if (!(chk_span(hd * DK, DK, nheads * DK, err) &&                              // q, k, g, eg
+              chk_span(hd * dv, dv, nheads * dv, err) &&                              // v, out, wg
+              chk_span(hd * dv * DK, (long long)dv * DK, nheads * dv * DK, err) &&    // S
+              chk_span(hd, 1, nheads, err) &&                                          // g, beta
+              chk_true(dv % (4 * kRowsInFlight) == 0, err)))
+            return;
+    }
 
     float kk[VEC], qq[VEC], aa[VEC], ee[VEC];  // ee: the reading direction
 #pragma unroll
@@ -132,7 +142,8 @@ static cudaError_t launch_decode(const void *q, const void *k, const void *v, co
                                  const float *wg = nullptr) {
     const unsigned int blocks = (unsigned int)((size_t)N * H);
     decode_step_kernel<Tin, DK, CH, DEC><<<blocks, kDecodeThreads, 0, st>>>(
-        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, eg, wg, S, (Tin *)out, dv);
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, eg, wg, S, (Tin *)out, dv,
+        (long long)N * H, kChecked ? gdr_host::device_error_word() : nullptr);
     return cudaGetLastError();
 }
 

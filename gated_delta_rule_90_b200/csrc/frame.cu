@@ -49,14 +49,23 @@ __host__ __device__ inline size_t slot(const Dims &d, int b, int f, int h) {
     return ((size_t)b * d.F + f) * d.H + h;
 }
 
+// Checked build: (b, f, h) names a frame-head of the call, and the frames tile
+// the T tokens (the last one may be shorter).  Every workspace slot a kernel
+// touches is slot(d, b, f, h) of such a triple.
+__device__ __forceinline__ bool frame_ok(const Dims &d, int b, int f, int h, unsigned int *err) {
+    return chk_span(b, 1, d.B, err) && chk_span(f, 1, d.F, err) && chk_span(h, 1, d.H, err) &&
+           chk_true(d.n >= 1 && (long long)(d.F - 1) * d.n < d.T && (long long)d.F * d.n >= d.T, err);
+}
+
 // G_t (d_k x d_k) then C_t (d_v x d_k): thread (ti, tj) owns an 8 x 8 block.
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads)
 frame_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
                   const float *__restrict__ gamma, float *__restrict__ Gw, float *__restrict__ Cw,
-                  Dims d) {
+                  Dims d, unsigned int *err) {
     extern __shared__ float sm[];
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    if (kChecked && !(frame_ok(d, b, f, h, err) && chk_true(d.dk <= 128 && d.dv <= 128, err))) return;
     const int kst = d.dk + 1, vst = d.dv + 1;
     float *Ks = sm, *Vs = Ks + kTokTile * kst, *gs = Vs + kTokTile * vst;
     const int tid = threadIdx.x, ti = tid >> 4, tj = tid & 15;
@@ -135,6 +144,7 @@ frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
     __shared__ __align__(16) float buf[2][128];  // pivot rows
     constexpr int NCG = DK / 8, NRG = DK / 4, HALF = DK / 2;  // column / row groups
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    if (kChecked && !(frame_ok(d, b, f, h, err) && chk_true(d.dk == DK, err))) return;
     const int tid = threadIdx.x, cg = tid % NCG, rg = tid / NCG;
     const bool act = rg < NRG;
     const int r0 = 4 * rg, jA = 4 * cg, jB = HALF + 4 * cg;
@@ -276,6 +286,7 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
     const int bh = blockIdx.x, b = bh / d.H, h = bh % d.H;
     const int r0 = blockIdx.y * kChainRows;
     const int nr = min(kChainRows, d.dv - r0);
+    if (kChecked && !(frame_ok(d, b, 0, h, err) && chk_true(nr >= 1 && d.dk <= 128, err))) return;
     const int dk = d.dk, sst = dk + 4;
     // W_t double buffer (unpadded, as copied), then S rows [16][dk + 4]
     float *Mb = sm, *S = Mb + 2 * dk * dk;
@@ -384,11 +395,12 @@ frame_chain_kernel(const float *__restrict__ Mw, const float *__restrict__ Cw,
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads)
 frame_out_kernel(const Tin *__restrict__ q, const float *__restrict__ Sw, Tin *__restrict__ out,
-                 Dims d) {
+                 Dims d, unsigned int *err) {
     extern __shared__ float sm[];
     const int tiles_per_frame = (d.n + kTokTile - 1) / kTokTile;
     const int f = blockIdx.x / tiles_per_frame, tile = blockIdx.x % tiles_per_frame;
     const int h = blockIdx.y, b = blockIdx.z;
+    if (kChecked && !frame_ok(d, b, f, h, err)) return;
     const int tt = f * d.n + tile * kTokTile;
     const int cnt = min(kTokTile, min(d.T, (f + 1) * d.n) - tt);
     if (cnt <= 0) return;  // whole CTA, before any barrier
@@ -435,6 +447,12 @@ frame_gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     const int ntiles = (t1 - t0 + kGT - 1) / kGT;
     const int x0 = h * kTD;
     const long yb = (long)b * d.T + t0;
+    if (kChecked) {  // checked build: the frame-head, and its first and last token tiles
+        const long long rows = (long long)d.B * d.T, xe = (long long)d.H * kTD;
+        if (!(frame_ok(d, b, f, h, err) && chk_tma(x0 + 64, yb, 2, xe, rows, err) &&
+              chk_tma(x0, yb + (long long)(ntiles - 1) * kGT, 2, xe, rows, err)))
+            return;
+    }
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
@@ -603,6 +621,8 @@ frame_chain_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__r
     const int j = (warp & 3) * 32 + (tid & 31);  // key channel = TMEM lane
     const int hr = (warp >> 2) * kHR;            // this thread's rows: r0 + hr .. + kHR - 1
     const size_t soff = ((size_t)b * d.H + h) * (size_t)kTD * kTD;
+    if (kChecked && !(frame_ok(d, b, 0, h, err) && chk_true(r0 + kCR <= kTD && d.dk == kTD && d.dv == kTD, err)))
+        return;  // whole CTA, before any sync
     if (tid == 0) {
         for (int i = 0; i < kWStages; ++i) mbar_init(&wfull[i], 1);
         mbar_init(mdone, 1);
@@ -757,6 +777,10 @@ frame_out_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int tt = f * d.n + tile * 128;
     const int cnt = min(128, min(d.T, (f + 1) * d.n) - tt);
     if (cnt <= 0) return;  // whole CTA, before any barrier
+    if (kChecked && !(frame_ok(d, b, f, h, err) &&
+                      chk_tma(h * kTD + 64, (long long)b * d.T + tt, 2, (long long)d.H * kTD,
+                              (long long)d.B * d.T, err)))
+        return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         mbar_init(&bar[0], 1);
@@ -898,7 +922,7 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
         if (tc)
             frame_gram_tc_kernel<<<gf, 256, sm_gram_tc, st>>>(mk, mv, gamma, GM, CN, d, err);
         else
-            frame_gram_kernel<Tin><<<gf, kThreads, sm_gram, st>>>((const Tin *)k, (const Tin *)v, gamma, GM, CN, d);
+            frame_gram_kernel<Tin><<<gf, kThreads, sm_gram, st>>>((const Tin *)k, (const Tin *)v, gamma, GM, CN, d, err);
         gdr_host::prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -930,7 +954,7 @@ cudaError_t frame_launch(const void *q, const void *k, const void *v, const floa
         } else {
             const int tiles = (d.n + kTokTile - 1) / kTokTile;
             const dim3 go((unsigned)(d.F * tiles), (unsigned)d.H, (unsigned)d.B);
-            frame_out_kernel<Tin><<<go, kThreads, sm_out, st>>>((const Tin *)q, Sw, (Tin *)out, d);
+            frame_out_kernel<Tin><<<go, kThreads, sm_out, st>>>((const Tin *)q, Sw, (Tin *)out, d, err);
         }
         gdr_host::prof_end(tk, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

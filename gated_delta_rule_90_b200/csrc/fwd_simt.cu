@@ -68,7 +68,8 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                 const float *__restrict__ g, const float *__restrict__ beta,
                 const float *__restrict__ eg, const float *__restrict__ wg,
                 const float *__restrict__ S0, Tin *__restrict__ out, float *__restrict__ S_final,
-                int T, int H, int dk, int dv, int C, const int32_t *__restrict__ cu, int T_total) {
+                int T, int H, int dk, int dv, int C, const int32_t *__restrict__ cu, int T_total,
+                int n_seq, unsigned int *err) {
     extern __shared__ float sm[];
     const SimtSmem L = simt_layout(C, dk, CH, DEC);
     float *Kc = sm + L.Kc, *Qc = sm + L.Qc, *Gc = sm + L.Gc, *Kx = sm + L.Kx, *bt = sm + L.bt;
@@ -82,6 +83,12 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     const int nr = min(kSimtRows, dv - r0);
     long t0, t1;
     seq_bounds(cu, s, T, T_total, t0, t1);
+    if (kChecked) {  // checked build: this CTA's tokens, state rows and state slot
+        const long long rows = cu ? (long long)T_total : (long long)n_seq * T;
+        if (!(chk_span(s, 1, n_seq, err) && chk_span(t0, t1 - t0, rows, err) &&
+              chk_true(nr >= 1 && r0 + nr <= dv, err)))
+            return;
+    }
 
     // state slice: rows r0 .. r0+nr of S (d_v x d_k)
     const size_t soff = ((size_t)s * H + h) * (size_t)dv * dk;
@@ -307,7 +314,7 @@ fwd_simt_wide_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const
                      const float *__restrict__ eg, const float *__restrict__ wg,
                      const float *__restrict__ S0, Tin *__restrict__ out, float *__restrict__ S_final,
                      int T, int H, int dk, int dv, int C, const int32_t *__restrict__ cu,
-                     int T_total) {
+                     int T_total, int n_seq, unsigned int *err) {
     extern __shared__ float sm[];
     const WideSmem L = wide_layout(C, dk, CH, DEC);
     float *NT = sm + L.NT, *Am = sm + L.Am, *Kb = sm + L.Kb, *Qb = sm + L.Qb, *Gb = sm + L.Gb;
@@ -322,6 +329,12 @@ fwd_simt_wide_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const
     const int seglen = (C + kWideSegs - 1) / kWideSegs;
     long t0, t1;
     seq_bounds(cu, s, T, T_total, t0, t1);
+    if (kChecked) {  // checked build: this CTA's tokens, state rows and state slot
+        const long long rows = cu ? (long long)T_total : (long long)n_seq * T;
+        if (!(chk_span(s, 1, n_seq, err) && chk_span(t0, t1 - t0, rows, err) &&
+              chk_true(nr >= 1 && r0 + nr <= dv, err)))
+            return;
+    }
 
     const size_t soff = ((size_t)s * H + h) * (size_t)dv * dk;
     for (int e = tid; e < kSimtRows * dk; e += kSimtThreads) {
@@ -552,7 +565,7 @@ static cudaError_t launch_simt(const void *q, const void *k, const void *v, cons
     dim3 grid((unsigned)(n_seq * H), (unsigned)((dv + kSimtRows - 1) / kSimtRows));
     kern<<<grid, kSimtThreads, smem, st>>>(
         (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, eg, wg, S0, (Tin *)out, S_final,
-        T, H, dk, dv, C, cu, T_total);
+        T, H, dk, dv, C, cu, T_total, n_seq, kChecked ? device_error_word() : nullptr);
     return cudaGetLastError();
 }
 

@@ -267,6 +267,14 @@ wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     if (!locate_chunk(geo, cu, ws, gcid, tstart, len)) return;  // whole CTA, before any sync
     const size_t slot = (size_t)gcid * geo.H + h;
     const int x0 = h * D, ytok = (int)tstart;
+    if (kChecked) {  // checked build: the chunk's tokens, its workspace slot, the TMA boxes
+        const long long rows = geo.varlen ? (long long)geo.T_total : (long long)geo.B * geo.T;
+        const long long xe = (long long)geo.H * D;
+        if (!(chk_span(tstart, len, rows, err) &&
+              chk_span((long long)slot, 1, (long long)geo.n_slots * geo.H, err) &&
+              chk_tma(x0, ytok, 2, xe, rows, err) && chk_tma(x0 + 64, ytok, 2, xe, rows, err)))
+            return;  // whole CTA, before any sync
+    }
 
     // The TMA thread initialises the barriers and issues the loads first, so
     // that their latency overlaps the TMEM allocation and the gate loads.
@@ -959,6 +967,15 @@ state_kernel(const __grid_constant__ CUtensorMap tm_W, const __grid_constant__ C
     seq_bounds(cu, s, geo.T, geo.T_total, t0, t1);
     const int gc0 = geo.varlen ? ws.chunk_start[s] : s * geo.nc;
     const int nch = (int)((t1 - t0 + C - 1) / C);
+    if (kChecked) {  // checked build: the sequence's tokens and the slots of its chunks
+        const long long rows = geo.varlen ? (long long)geo.T_total : (long long)geo.B * geo.T;
+        const long long nsl = (long long)geo.n_slots * geo.H;
+        const long long sl0 = (long long)gc0 * geo.H + h, sl1 = (long long)(gc0 + nch - 1) * geo.H + h;
+        if (!(chk_span(s, 1, geo.n_seq, err) && chk_span(t0, t1 - t0, rows, err) &&
+              (nch == 0 || (chk_span(sl0, 1, nsl, err) && chk_span(sl1, 1, nsl, err))) &&
+              chk_tma(h * D, 0, 2, (long long)geo.H * D, 1, err)))
+            return;  // whole CTA, before any sync
+    }
 
     // stage r & 1 <- chunk r's operands and decay rows; -W<- and Q<- arrive as
     // alternating SUB-row blocks (their maps have SUB-row boxes)

@@ -193,6 +193,7 @@ const char *gdr_status_string(gdr_status s) {
         case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: sizes or path not built";
         case GDR_ERR_CUDA: return "GDR_ERR_CUDA: CUDA runtime error";
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded device wait expired";
+        case GDR_ERR_BOUNDS: return "GDR_ERR_BOUNDS: a bounds guard refused an access";
     }
     return "GDR_ERR_UNKNOWN";
 }
@@ -384,7 +385,26 @@ static __global__ void wait_timeout_kernel(unsigned int spin_limit, unsigned int
     }
 }
 
+// A guarded write one element past a 16-float array: the guard refuses it.
+static __device__ float g_bounds_scratch[16];
+static __global__ void bounds_selftest_kernel(float *scratch, unsigned int *err) {
+    const long long i = 16 + threadIdx.x;
+    if (gdr::chk_span(i, 1, 16, err)) scratch[i] = 1.f;
+}
+
 extern "C" {
+
+int gdr_checked_build(void) { return gdr::kChecked ? 1 : 0; }
+
+gdr_status gdr_selftest_bounds(void *stream) {
+    if (!gdr::kChecked) return GDR_ERR_UNSUPPORTED;
+    unsigned int *err = gdr_host::device_error_word();
+    if (!err) return GDR_ERR_CUDA;
+    float *p = nullptr;
+    if (cudaGetSymbolAddress((void **)&p, g_bounds_scratch) != cudaSuccess) return GDR_ERR_CUDA;
+    bounds_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(p, err);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
 
 gdr_status gdr_device_status(void *stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
@@ -395,6 +415,7 @@ gdr_status gdr_device_status(void *stream) {
     if (word && cudaMemcpyToSymbol(g_gdr_device_error, &zero, sizeof(zero)) != cudaSuccess)
         return GDR_ERR_CUDA;
     if (word & gdr::kErrTimeout) return GDR_ERR_TIMEOUT;
+    if (word & gdr::kErrBounds) return GDR_ERR_BOUNDS;
     return (word & gdr::kErrNumeric) ? GDR_ERR_INVALID : GDR_OK;
 }
 

@@ -41,7 +41,10 @@ __global__ void __launch_bounds__(256) gdp_expand_kernel(const Tin *__restrict__
                                                          const float *__restrict__ g,
                                                          Tin *__restrict__ qv,
                                                          float *__restrict__ gv, long n_tokens,
-                                                         int H, int dk, int nh) {
+                                                         int H, int dk, int nh, unsigned int *err) {
+    // checked build: the 16-byte vectors tile every row exactly
+    if (kChecked && !chk_true((dk * (int)sizeof(Tin)) % 16 == 0 && (!CH || dk % 4 == 0) && nh >= 1, err))
+        return;
     const int hq = H * (dk * (int)sizeof(Tin) / 16);  // q vectors of one token
     const int hg = CH ? H * (dk / 4) : H;              // g floats4 (or floats) of one token
     const uint4 *q4 = reinterpret_cast<const uint4 *>(q);
@@ -73,7 +76,8 @@ __global__ void __launch_bounds__(256) gdp_expand_kernel(const Tin *__restrict__
 template <typename Tin>
 __global__ void __launch_bounds__(256) gdp_gather_kernel(const Tin *__restrict__ ov,
                                                          Tin *__restrict__ out, long n_tokens,
-                                                         int H, int dv, int nh) {
+                                                         int H, int dv, int nh, unsigned int *err) {
+    if (kChecked && !chk_true((dv * (int)sizeof(Tin)) % 16 == 0 && nh >= 1, err)) return;
     const int ho = H * (dv * (int)sizeof(Tin) / 16);
     const uint4 *ov4 = reinterpret_cast<const uint4 *>(ov);
     uint4 *out4 = reinterpret_cast<uint4 *>(out);
@@ -85,7 +89,8 @@ __global__ void __launch_bounds__(256) gdp_gather_kernel(const Tin *__restrict__
 }
 
 __global__ void gdp_scale_offsets_kernel(const int32_t *__restrict__ cu, int32_t *__restrict__ cuv,
-                                         int n, int nh) {
+                                         int n, int nh, unsigned int *err) {
+    if (kChecked && !chk_true(n >= 1 && nh >= 1, err)) return;
     for (int i = threadIdx.x; i <= n; i += blockDim.x) cuv[i] = cu[i] * nh;
 }
 
@@ -168,6 +173,7 @@ gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const fl
     float *gv = (float *)(ws + L.gv);
     int32_t *cuv = varlen ? (int32_t *)(ws + L.cuv) : nullptr;
     cudaStream_t st = (cudaStream_t)stream;
+    unsigned int *cerr = kChecked ? gdr_host::device_error_word() : nullptr;  // checked build
     const long ntok = (long)B * T;
     const bool ch = gate == GDR_GATE_PER_KEY_CHANNEL;
     if (ntok > 0) {
@@ -176,25 +182,25 @@ gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const fl
         if (dtype == GDR_BF16) {
             if (ch)
                 gdp_expand_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(
-                    (const __nv_bfloat16 *)q, g, (__nv_bfloat16 *)qv, gv, ntok, H, d_k, n_h);
+                    (const __nv_bfloat16 *)q, g, (__nv_bfloat16 *)qv, gv, ntok, H, d_k, n_h, cerr);
             else
                 gdp_expand_kernel<__nv_bfloat16, false><<<grid, 256, 0, st>>>(
-                    (const __nv_bfloat16 *)q, g, (__nv_bfloat16 *)qv, gv, ntok, H, d_k, n_h);
+                    (const __nv_bfloat16 *)q, g, (__nv_bfloat16 *)qv, gv, ntok, H, d_k, n_h, cerr);
         } else {
             if (ch)
                 gdp_expand_kernel<float, true><<<grid, 256, 0, st>>>((const float *)q, g,
                                                                      (float *)qv, gv, ntok, H,
-                                                                     d_k, n_h);
+                                                                     d_k, n_h, cerr);
             else
                 gdp_expand_kernel<float, false><<<grid, 256, 0, st>>>((const float *)q, g,
                                                                       (float *)qv, gv, ntok, H,
-                                                                      d_k, n_h);
+                                                                      d_k, n_h, cerr);
         }
         gdr_host::prof_end(tk, st);
         if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     }
     if (varlen) {
-        gdp_scale_offsets_kernel<<<1, 256, 0, st>>>(cu_seqlens, cuv, n_seq, n_h);
+        gdp_scale_offsets_kernel<<<1, 256, 0, st>>>(cu_seqlens, cuv, n_seq, n_h, cerr);
         if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     }
     // the tensor-core path writes the kept rows itself; otherwise gather them
@@ -212,10 +218,10 @@ gdr_status gdr_fwd_product(const void *q, const void *k, const void *v, const fl
         gdr_host::ProfToken tk = gdr_host::prof_begin(GDR_K_GDP_REMAP, st);
         if (dtype == GDR_BF16)
             gdp_gather_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-                (const __nv_bfloat16 *)ov, (__nv_bfloat16 *)out, ntok, H, d_v, n_h);
+                (const __nv_bfloat16 *)ov, (__nv_bfloat16 *)out, ntok, H, d_v, n_h, cerr);
         else
             gdp_gather_kernel<float><<<grid, 256, 0, st>>>((const float *)ov, (float *)out, ntok,
-                                                           H, d_v, n_h);
+                                                           H, d_v, n_h, cerr);
         gdr_host::prof_end(tk, st);
         if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     }

@@ -45,7 +45,8 @@ typedef enum {
     GDR_ERR_INVALID = 1,      /* bad shape, NULL where required, misalignment, bad enum */
     GDR_ERR_UNSUPPORTED = 2,  /* valid but not built: sizes or path outside the instantiated set */
     GDR_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
-    GDR_ERR_TIMEOUT = 4       /* a bounded device-side wait expired (see gdr_device_status) */
+    GDR_ERR_TIMEOUT = 4,      /* a bounded device-side wait expired (see gdr_device_status) */
+    GDR_ERR_BOUNDS = 5        /* checked build only: a kernel's bounds guard refused an access */
 } gdr_status;
 
 typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
@@ -138,7 +139,9 @@ gdr_status gdr_decode_step(const void *q, const void *k, const void *v, const fl
  * Synchronises `stream`, then reports (and clears) the device-side error word
  * of the current device: GDR_ERR_TIMEOUT if a bounded wait inside a kernel
  * gave up since the last call (that kernel skipped its remaining work and
- * returned), GDR_ERR_CUDA if the stream reports an error, else GDR_OK.
+ * returned), GDR_ERR_BOUNDS if a guard of the checked build refused an access,
+ * GDR_ERR_INVALID if a frame factorisation met a non-positive pivot,
+ * GDR_ERR_CUDA if the stream reports an error, else GDR_OK.
  */
 gdr_status gdr_device_status(void *stream);
 
@@ -149,6 +152,25 @@ gdr_status gdr_device_status(void *stream);
  * returns normally (the context stays usable).  Follow with gdr_device_status.
  */
 gdr_status gdr_selftest_wait_timeout(unsigned int spin_limit, void *stream);
+
+/*
+ * The checked build (compiled with -DGDR_CHECK; libgdr_check.so beside
+ * libgdr.so): every kernel checks the spans of the global buffers its CTA reads
+ * and writes, and its TMA coordinates (x >= 0 and 16-byte aligned, box origin
+ * inside the tensor), against the extents of the call before it touches
+ * memory.  A failed check sets a bit in the device error word, the CTA returns
+ * without touching anything, and gdr_device_status reports GDR_ERR_BOUNDS.
+ * The checks cost a few instructions per CTA; results are bit-identical to the
+ * normal build's.
+ *
+ * gdr_checked_build: 1 in the checked build, 0 in the normal one.
+ * gdr_selftest_bounds: checked build only (else GDR_ERR_UNSUPPORTED): launches
+ * one tiny kernel whose guard refuses an access past the end of a 16-float
+ * scratch array (the access is never made), so that the following
+ * gdr_device_status reports GDR_ERR_BOUNDS; the context stays usable.
+ */
+int gdr_checked_build(void);
+gdr_status gdr_selftest_bounds(void *stream);
 
 /*
  * Gated DeltaProduct prefill ("Linear Attention, Visualized", section "Gated

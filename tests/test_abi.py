@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for s in range(5):
+    for s in range(6):
         assert binding.status_string(s).startswith("GDR_")
     assert "UNKNOWN" in binding.status_string(99)
 
