@@ -43,13 +43,13 @@ _TC_SRC = ('csrc/fwd_tc.cu', 'csrc/sm100.cuh', 'csrc/common.cuh')
 _DEC_SRC = ('csrc/decode.cu', 'csrc/common.cuh')
 _FR_SRC = ('csrc/frame.cu', 'csrc/sm100.cuh', 'csrc/tmap.cuh', 'csrc/common.cuh')
 NCU_TRAFFIC = {
-    ("tc_wy", "gdn_prefill"): (_TC_SRC, "0ab89a53881ca31f", 206.257408e6 + 255.669760e6),
-    ("tc_state", "gdn_prefill"): (_TC_SRC, "0ab89a53881ca31f", 308.456960e6 + 56.687104e6),
-    ("tc_wy", "kda_prefill"): (_TC_SRC, "31ad39eb861feed8", 681.934848e6 + 578.909184e6),
-    ("decode", "decode"): (_DEC_SRC, "82e1f5016f476188", 543.250944e6 + 482.361600e6),
-    ("decode", "kda_decode"): (_DEC_SRC, "82e1f5016f476188", 547.403264e6 + 482.458624e6),
-    ("frame_chain", "frame_prefill"): (_FR_SRC, "2984ca0634014dc4", 33.711104e6 + 0.0),
-    ("frame_solve", "frame_prefill"): (_FR_SRC, "2984ca0634014dc4", 16.795136e6 + 0.002048e6),
+    ("tc_wy", "gdn_prefill"): (_TC_SRC, "90c504ae376e1600", 206.136064e6 + 253.452032e6),
+    ("tc_state", "gdn_prefill"): (_TC_SRC, "90c504ae376e1600", 308.366336e6 + 52.554752e6),
+    ("tc_wy", "kda_prefill"): (_TC_SRC, "90c504ae376e1600", 681.240832e6 + 565.438464e6),
+    ("decode", "decode"): (_DEC_SRC, "67d72f2db8183636", 543.343360e6 + 481.382144e6),
+    ("decode", "kda_decode"): (_DEC_SRC, "67d72f2db8183636", 547.481088e6 + 481.806848e6),
+    ("frame_chain", "frame_prefill"): (_FR_SRC, "d7a96b3509fa7060", 33.724160e6 + 0.0),
+    ("frame_solve", "frame_prefill"): (_FR_SRC, "d7a96b3509fa7060", 16.797184e6 + 0.0),
 }
 
 
@@ -614,9 +614,11 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                 "peak_source": peak_kind + " hbm_gbs", "algorithmic_bytes_per_launch": B_,
                 "frac_of_8TBps_spec": ach / 8000.0}
     elif is_frame:
-        # the dominant pass against its own roof: the token contractions (Gram,
-        # output) run on the tensor cores for bf16 d = 128, the factorisation and
-        # the chain are fp32 CUDA-core work
+        # the dominant pass against its own roof: for bf16 d = 128 the token
+        # contractions (Gram, output) and the chain run on the tensor cores (the
+        # chain's flops counted once, though its bf16 split executes three
+        # products); the factorisation, and every pass of the fp32 path, is
+        # fp32 CUDA-core work
         th = cfg.B * cfg.T * cfg.H
         fh = cfg.B * cfg.frames * cfg.H
         dk, dv = cfg.d_k, cfg.d_v
@@ -625,7 +627,7 @@ def measure(args, name, device, rank, world, peaks, peak_kind, path, steps, warm
                   "frame_solve": dk ** 3 / 3 * fh,
                   "frame_chain": 2 * dv * dk * dk * fh}
         flops = pflops.get(dom, 0)
-        on_tc = tc_path and dom in ("frame_gram", "frame_out")
+        on_tc = tc_path and dom in ("frame_gram", "frame_out", "frame_chain")
         alu_peak = SM_COUNT * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         peak = peaks["bf16_tflops"] if on_tc else alu_peak
         ach = flops / (dom_ms * 1e-3) / 1e12
