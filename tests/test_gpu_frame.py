@@ -72,6 +72,17 @@ def test_frame_bf16_d128(cuda_device, n):
     check(inputs.frame_inputs(cfg, seed=702), cuda_device)
 
 
+@pytest.mark.parametrize("gate,s0_var", [("scalar", 0.01), ("channel", 0.0), ("scalar", 0.0)])
+def test_frame_bf16_d128_gates_and_zero_state(cuda_device, gate, s0_var):
+    """The tensor-core passes with one scalar decay per frame (broadcast over
+    the key channels inside the chain) and with no initial state (S0 = 0);
+    two sequences, a partial last frame."""
+    cfg = cfg_of(B=2, T=700, H=2, n=128, gate=gate, s0_var=s0_var)
+    inp = inputs.frame_inputs(cfg, seed=707)
+    assert (inp.S0 is None) == (s0_var == 0.0)
+    check(inp, cuda_device)
+
+
 def test_frame_one_token_is_the_delta_rule_on_gpu(cuda_device):
     """n = 1 against gdr_fwd with beta = gamma / (1 + gamma) (Sherman-Morrison)."""
     cfg = cfg_of(B=1, T=96, H=2, d_k=64, d_v=64, n=1, dtype="f32", gate="channel", s0_var=0.01)
