@@ -260,9 +260,12 @@ gdr_status gdr_decode_step_gdn2(const void *q, const void *k, const void *v, con
  *  d_k a multiple of 16 in [16, 128]; d_v a multiple of 8 in [8, 128]
  *  workspace: gdr_fwd_frame_workspace_size(B, T, H, d_k, d_v, n) bytes,
  *           caller-owned device memory (per frame: G_t then W_t, C_t and S_t).
- * The Gram and output passes run on the tensor cores for bf16 with
- * d_k = d_v = 128 (bf16 operands, fp32 accumulation); the inverse and the
- * chain are fp32 on the CUDA cores.  Errors as gdr_fwd.
+ * For bf16 with d_k = d_v = 128 the Gram and output passes run on the tensor
+ * cores (bf16 operands, fp32 accumulation), and so does the chain, with each
+ * product split into three bf16 products (x = x_hi + x_lo, A W ~ A_hi W_hi +
+ * A_hi W_lo + A_lo W_hi) so that it keeps fp32 accuracy; the inverse is fp32
+ * on the CUDA cores.  Otherwise every pass is fp32 on the CUDA cores.  Errors
+ * as gdr_fwd.
  */
 size_t gdr_fwd_frame_workspace_size(int B, int T, int H, int d_k, int d_v, int n);
 gdr_status gdr_fwd_frame(const void *q, const void *k, const void *v, const float *g,
