@@ -83,6 +83,15 @@ def test_frame_bf16_d128_gates_and_zero_state(cuda_device, gate, s0_var):
     check(inp, cuda_device)
 
 
+@pytest.mark.parametrize("T,n", [(100, 128), (256, 128), (129, 128)])
+def test_frame_bf16_d128_few_frames(cuda_device, T, n):
+    """The tensor-core chain's pipeline ends: one frame (the loop runs only its
+    first step), exactly as many frames as it has stages, and a one-token last
+    frame."""
+    cfg = cfg_of(B=2, T=T, H=2, n=n, s0_var=0.01)
+    check(inputs.frame_inputs(cfg, seed=708), cuda_device)
+
+
 def test_frame_one_token_is_the_delta_rule_on_gpu(cuda_device):
     """n = 1 against gdr_fwd with beta = gamma / (1 + gamma) (Sherman-Morrison)."""
     cfg = cfg_of(B=1, T=96, H=2, d_k=64, d_v=64, n=1, dtype="f32", gate="channel", s0_var=0.01)
