@@ -126,109 +126,116 @@ frame_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v,
 // complement's diagonal) is >= 1 and no pivoting is needed.  G_t is
 // symmetrised as (G + G^T) / 2 on load; with s = a_kk^-1/2 and c = s b (b =
 // pivot row) the update a_ij -= c_i c_j is symmetric in i and j, so the matrix
-// stays exactly symmetric and row k stands in for column k.  A thread holds a
-// 4 x 8 tile in registers and reads 12 pivot-row values per step; the pivot
-// row passes through a double buffer in shared memory, written by its own
-// row's threads during the previous step: one barrier per pivot.  W_t
-// overwrites G_t.
-constexpr int kSwThreads = 512;  // (d_k / 4) x (d_k / 8) tiles of 4 x 8, d_k <= 128
-// Thread (row group rg, column group cg) holds rows 4 rg .. 4 rg + 3 and the
-// columns 4 cg .. 4 cg + 3 and d_k/2 + 4 cg .. + 3, so that the float4 reads of
-// a pivot row by the column groups cover contiguous bytes (no bank conflicts).
-// With SPLIT the result is written as two bf16 matrices instead, W_hi = bf16(W)
-// and W_lo = bf16(W - W_hi), one after the other in the slot's first half
-// (the operands of the tensor-core chain).
+// stays exactly symmetric and row k stands in for column k.  The pivot row
+// passes through a double buffer in shared memory, written by the threads that
+// hold it during the previous step: one barrier per pivot.  W_t overwrites
+// G_t; with SPLIT it is written as two bf16 matrices instead, W_hi = bf16(W)
+// and W_lo = bf16(W - W_hi), one after the other in the slot's first half (the
+// operands of the tensor-core chain).
+//
+// The sweep runs on the upper triangle only: the update a_ij -= c_i c_j and
+// the pivot's row and column give bit-identical values at (i, j) and (j, i),
+// so a thread holds one 4 x 4 block (bi, bj), bi <= bj, of the upper triangle
+// (a diagonal block in full), reads four pivot-row values for its rows and
+// four for its columns, and mirrors the block on output (a layout of 4 x 8
+// tiles over the whole matrix took 70 us against 64 us on the frame
+// workload).  The next pivot row k + 1 is published by the blocks of block
+// row (k + 1) / 4 (its columns from there on) and of block column (k + 1) / 4
+// above the diagonal (its earlier columns, by symmetry).
+constexpr int kSymThreads = 544;  // 17 warps >= 32 * 33 / 2 blocks (d_k = 128)
+
 template <int DK, bool SPLIT>
-__global__ void __launch_bounds__(kSwThreads, 2)
-frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
+__global__ void __launch_bounds__(kSymThreads, 2)
+frame_inverse_sym_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
+    constexpr int NB = DK / 4, NBLK = NB * (NB + 1) / 2;
+    static_assert(NBLK <= kSymThreads, "one block per thread");
     __shared__ __align__(16) float buf[2][128];  // pivot rows
-    constexpr int NCG = DK / 8, NRG = DK / 4, HALF = DK / 2;  // column / row groups
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     if (kChecked && !(frame_ok(d, b, f, h, err) && chk_true(d.dk == DK, err))) return;
-    const int tid = threadIdx.x, cg = tid % NCG, rg = tid / NCG;
-    const bool act = rg < NRG;
-    const int r0 = 4 * rg, jA = 4 * cg, jB = HALF + 4 * cg;
+    const int tid = threadIdx.x;
+    const bool act = tid < NBLK;
+    int bi = 0, rem = tid;  // row-major enumeration of the upper-triangle blocks
+    while (bi < NB && rem >= NB - bi) {
+        rem -= NB - bi;
+        ++bi;
+    }
+    const int bj = bi + rem, r0 = 4 * bi, c0 = 4 * bj;
     const size_t sl = slot(d, b, f, h);
     float *Gp = GW + sl * (size_t)DK * DK;
-    auto col = [&](int u) { return u < 4 ? jA + u : jB + u - 4; };
-    float a[4][8];
+    float a[4][4];
     if (act) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float4 x = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + jA);
-            const float4 y = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + jB);
+            const float4 x = *reinterpret_cast<const float4 *>(Gp + (size_t)(r0 + i) * DK + c0);
             a[i][0] = x.x; a[i][1] = x.y; a[i][2] = x.z; a[i][3] = x.w;
-            a[i][4] = y.x; a[i][5] = y.y; a[i][6] = y.z; a[i][7] = y.w;
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {  // G^T: column col(u), rows r0..r0+3
-            const float4 t = *reinterpret_cast<const float4 *>(Gp + (size_t)col(u) * DK + r0);
+        for (int u = 0; u < 4; ++u) {  // G^T: column c0 + u, rows r0..r0+3
+            const float4 t = *reinterpret_cast<const float4 *>(Gp + (size_t)(c0 + u) * DK + r0);
             const float tv[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                a[i][u] = 0.5f * (a[i][u] + tv[i]) + (r0 + i == col(u) ? 1.f : 0.f);
+                a[i][u] = 0.5f * (a[i][u] + tv[i]) + (r0 + i == c0 + u ? 1.f : 0.f);
         }
-        if (rg == 0) {
-            *reinterpret_cast<float4 *>(&buf[0][jA]) = make_float4(a[0][0], a[0][1], a[0][2], a[0][3]);
-            *reinterpret_cast<float4 *>(&buf[0][jB]) = make_float4(a[0][4], a[0][5], a[0][6], a[0][7]);
-        }
+        if (bi == 0)  // row 0 lies in block row 0
+            *reinterpret_cast<float4 *>(&buf[0][c0]) = make_float4(a[0][0], a[0][1], a[0][2], a[0][3]);
     }
     __syncthreads();
-    // pivot k: column k is local column (k >= d_k/2 ? 4 : 0) + k % 4 of column
-    // group (k % (d_k/2)) / 4; the two halves of the pivots are separate loops so
-    // that this index is a compile-time constant
+    for (int k4 = 0; k4 < DK; k4 += 4) {
+        const int kb = k4 >> 2;
 #pragma unroll
-    for (int hk = 0; hk < 2; ++hk) {
-        for (int k4 = 0; k4 < HALF; k4 += 4) {
+        for (int kk = 0; kk < 4; ++kk) {
+            const int k = k4 + kk;
+            const float *bk = buf[k & 1];
+            const float dkk = bk[k];
+            if (tid == 0 && !(dkk > 0.f)) atomicOr(err, kErrNumeric);
+            const float sq = rsqrtf(dkk);
+            if (act) {
+                const float4 br = *reinterpret_cast<const float4 *>(bk + r0);
+                const float4 bc = *reinterpret_cast<const float4 *>(bk + c0);
+                const float cr[4] = {br.x * sq, br.y * sq, br.z * sq, br.w * sq};
+                const float cc[4] = {bc.x * sq, bc.y * sq, bc.z * sq, bc.w * sq};
+                const bool krow = kb == bi, kcol = kb == bj;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const int k = hk * HALF + k4 + kk;
-                const int uk = 4 * hk + kk;  // the pivot's local column
-                const float *bk = buf[k & 1];
-                const float dkk = bk[k];
-                if (tid == 0 && !(dkk > 0.f)) atomicOr(err, kErrNumeric);
-                const float sq = rsqrtf(dkk);
-                if (act) {
-                    const float4 br4 = *reinterpret_cast<const float4 *>(bk + r0);
-                    const float4 bj0 = *reinterpret_cast<const float4 *>(bk + jA);
-                    const float4 bj1 = *reinterpret_cast<const float4 *>(bk + jB);
-                    const float cr[4] = {br4.x * sq, br4.y * sq, br4.z * sq, br4.w * sq};
-                    const float cj[8] = {bj0.x * sq, bj0.y * sq, bj0.z * sq, bj0.w * sq,
-                                         bj1.x * sq, bj1.y * sq, bj1.z * sq, bj1.w * sq};
-                    const bool krow = (k >> 2) == rg, kcol = (k4 >> 2) == cg;
+                for (int i = 0; i < 4; ++i) {
+                    if (krow && i == kk) {  // row k
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (i == kk && krow) {  // row k
+                        for (int u = 0; u < 4; ++u) a[i][u] = (kcol && u == kk) ? -(sq * sq) : cc[u] * sq;
+                    } else {
 #pragma unroll
-                            for (int u = 0; u < 8; ++u) a[i][u] = (u == uk && kcol) ? -(sq * sq) : cj[u] * sq;
-                        } else {
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) a[i][u] = fmaf(-cr[i], cj[u], a[i][u]);
-                            if (kcol) a[i][uk] = cr[i] * sq;  // column k
-                        }
-                    }
-                    if (((k + 1) >> 2) == rg && k + 1 < DK) {  // publish the next pivot row
-                        const int ni = (kk + 1) & 3;
-                        float *bn = buf[(k + 1) & 1];
-                        *reinterpret_cast<float4 *>(bn + jA) = make_float4(a[ni][0], a[ni][1], a[ni][2], a[ni][3]);
-                        *reinterpret_cast<float4 *>(bn + jB) = make_float4(a[ni][4], a[ni][5], a[ni][6], a[ni][7]);
+                        for (int u = 0; u < 4; ++u) a[i][u] = fmaf(-cr[i], cc[u], a[i][u]);
+                        if (kcol) a[i][kk] = cr[i] * sq;  // column k
                     }
                 }
-                __syncthreads();
+                if (k + 1 < DK) {  // publish row k + 1
+                    const int nb = (k + 1) >> 2, ni = (k + 1) & 3;
+                    float *bn = buf[(k + 1) & 1];
+                    if (bi == nb)
+                        *reinterpret_cast<float4 *>(bn + c0) =
+                            make_float4(a[ni][0], a[ni][1], a[ni][2], a[ni][3]);
+                    else if (bj == nb)
+                        *reinterpret_cast<float4 *>(bn + r0) =
+                            make_float4(a[0][ni], a[1][ni], a[2][ni], a[3][ni]);
+                }
             }
+            __syncthreads();
         }
     }
+    // the sweep leaves -W: the block and its mirror image
     if (act && !SPLIT) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float *o = Gp + (size_t)(r0 + i) * DK;
-            *reinterpret_cast<float4 *>(o + jA) = make_float4(-a[i][0], -a[i][1], -a[i][2], -a[i][3]);
-            *reinterpret_cast<float4 *>(o + jB) = make_float4(-a[i][4], -a[i][5], -a[i][6], -a[i][7]);
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(Gp + (size_t)(r0 + i) * DK + c0) =
+                make_float4(-a[i][0], -a[i][1], -a[i][2], -a[i][3]);
+        if (bi != bj) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                *reinterpret_cast<float4 *>(Gp + (size_t)(c0 + u) * DK + r0) =
+                    make_float4(-a[0][u], -a[1][u], -a[2][u], -a[3][u]);
         }
     }
     if (act && SPLIT) {  // every read of G happened before the first barrier
         __nv_bfloat16 *wh = reinterpret_cast<__nv_bfloat16 *>(Gp), *wl = wh + DK * DK;
-        // two consecutive entries of -a as packed bf16 pairs (hi, lo)
         auto split2 = [](float x, float y, uint32_t &hi, uint32_t &lo) {
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(-x, -y);
             const float2 hf = __bfloat1622float2(h2);
@@ -236,18 +243,18 @@ frame_inverse_kernel(float *__restrict__ GW, Dims d, unsigned int *err) {
             hi = *reinterpret_cast<const uint32_t *>(&h2);
             lo = *reinterpret_cast<const uint32_t *>(&l2);
         };
+        auto put = [&](int row, int col, float x0, float x1, float x2, float x3) {
+            uint2 hv, lv;
+            split2(x0, x1, hv.x, lv.x);
+            split2(x2, x3, hv.y, lv.y);
+            *reinterpret_cast<uint2 *>(wh + (size_t)row * DK + col) = hv;
+            *reinterpret_cast<uint2 *>(wl + (size_t)row * DK + col) = lv;
+        };
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint2 h0, h1, l0, l1;
-            split2(a[i][0], a[i][1], h0.x, l0.x);
-            split2(a[i][2], a[i][3], h0.y, l0.y);
-            split2(a[i][4], a[i][5], h1.x, l1.x);
-            split2(a[i][6], a[i][7], h1.y, l1.y);
-            const size_t o = (size_t)(r0 + i) * DK;
-            *reinterpret_cast<uint2 *>(wh + o + jA) = h0;
-            *reinterpret_cast<uint2 *>(wh + o + jB) = h1;
-            *reinterpret_cast<uint2 *>(wl + o + jA) = l0;
-            *reinterpret_cast<uint2 *>(wl + o + jB) = l1;
+        for (int i = 0; i < 4; ++i) put(r0 + i, c0, a[i][0], a[i][1], a[i][2], a[i][3]);
+        if (bi != bj) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) put(c0 + u, r0, a[0][u], a[1][u], a[2][u], a[3][u]);
         }
     }
 }
@@ -257,12 +264,12 @@ static cudaError_t launch_inverse(float *GW, const Dims &d, bool split, unsigned
     const dim3 gf((unsigned)d.F, (unsigned)d.H, (unsigned)d.B);
     if (split) {
         if (d.dk != 128) return cudaErrorInvalidValue;
-        frame_inverse_kernel<128, true><<<gf, kSwThreads, 0, st>>>(GW, d, err);
+        frame_inverse_sym_kernel<128, true><<<gf, kSymThreads, 0, st>>>(GW, d, err);
         return cudaGetLastError();
     }
     switch (d.dk) {
 #define GDR_INV(DK) \
-    case DK: frame_inverse_kernel<DK, false><<<gf, kSwThreads, 0, st>>>(GW, d, err); break
+    case DK: frame_inverse_sym_kernel<DK, false><<<gf, kSymThreads, 0, st>>>(GW, d, err); break
         GDR_INV(16); GDR_INV(32); GDR_INV(48); GDR_INV(64);
         GDR_INV(80); GDR_INV(96); GDR_INV(112); GDR_INV(128);
 #undef GDR_INV
