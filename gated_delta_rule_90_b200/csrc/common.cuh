@@ -42,11 +42,11 @@ __device__ __forceinline__ bool chk_true(bool cond, unsigned int *err) {
     if (err) atomicOr(err, kErrBounds);
     return false;
 }
-// A tiled TMA copy whose box starts at (x, y) in a tensor of x_extent elements
-// per row (element size esz bytes) and `rows` rows: x must be >= 0 with
-// x * esz a multiple of 16 (an unaligned x is an illegal instruction), and the
-// box must start inside the tensor (a load may run past the end, which the
-// copy fills with zeros; a store is clipped there).
+// A tiled TMA copy of a box_x x box_y box at (x, y) of a tensor with x_extent
+// elements per row (element size esz bytes) and `rows` rows: x must be >= 0
+// with x * esz a multiple of 16 (an unaligned x is an illegal instruction), the
+// box must start inside the tensor, and y >= 0 (loads may run past the end,
+// which the copy fills with zeros; stores are clipped there).
 __device__ __forceinline__ bool chk_tma(long long x, long long y, int esz, long long x_extent,
                                         long long rows, unsigned int *err) {
     if (!kChecked) return true;
